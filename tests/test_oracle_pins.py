@@ -1,0 +1,356 @@
+"""Pins of the CPU oracle to facts outside itself (no GPU).
+
+Each test fixes the oracle against something it does not compute itself: a
+hand-derived fixture, a closed form, brute force over all subsets, an
+independent library routine (torch's fp64 attention, torch's bf16 cast) or
+an invariant.  ``test_mutants_are_caught`` plants plausible mistakes in a
+copy of the oracle and checks that these pins reject each one.
+"""
+import itertools
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import rtp_oracle as ro
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _read_rows(name):
+    rows = []
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                rows.append(line.split())
+    return rows
+
+
+# --------------------------------------------------------------------------
+# hand-derived fixtures
+# --------------------------------------------------------------------------
+
+def test_topp_hand_fixture():
+    s = np.log(np.array([2.0, 4.0, 1.0, 4.0, 2.0]))
+    for p, count, tiepos, sel in _read_rows("topp_hand.txt"):
+        r = oracle.topp_select(s, float(p))
+        assert r.count == int(count)
+        assert r.tiepos == int(tiepos)
+        assert r.idx.tolist() == [int(x) for x in sel.split(",")]
+        assert r.tau == s[int(tiepos)]
+
+
+def test_attention_hand_fixture():
+    q = np.array([1.0, 0.0])
+    K = np.array([[0.0, 5.0], [math.log(3.0), 1.0], [math.log(2.0), -7.0]])
+    V = np.array([[1.0, 0.0], [0.0, 1.0], [2.0, 2.0]])
+    for sel, o0, o1 in _read_rows("attn_hand.txt"):
+        idx = np.array([int(x) for x in sel.split(",")])
+        o = oracle.attend(q, K, V, idx, 1.0)
+        np.testing.assert_allclose(o, [float(o0), float(o1)], rtol=0, atol=1e-14)
+
+
+# --------------------------------------------------------------------------
+# storage rounding: independent routine (torch's float32 -> bf16 cast) and hand cases
+# --------------------------------------------------------------------------
+
+def test_round_bf16_matches_torch_cast():
+    rng = np.random.default_rng(5)
+    x = np.concatenate([rng.standard_normal(20000), rng.standard_normal(2000) * 1e-30,
+                        rng.standard_normal(2000) * 1e30]).astype(np.float32)
+    ref = torch.from_numpy(x).to(torch.bfloat16).to(torch.float64).numpy()
+    np.testing.assert_array_equal(oracle.round_bf16(x.astype(np.float64)), ref)
+
+
+def test_round_bf16_hand_cases():
+    h = 2.0 ** -8
+    cases = {1.0 + h: 1.0, 1.0 + 3 * h: 1.0 + 4 * h, -(1.0 + h): -1.0, 0.0: 0.0,
+             2.0 ** -130: 2.0 ** -130, 3.0: 3.0, 255.5: 256.0, 1.0 + 1.5 * h: 1.0 + 2 * h}
+    for x, want in cases.items():
+        assert oracle.round_bf16(np.array([x]))[0] == want, x
+
+
+# --------------------------------------------------------------------------
+# indexer: special cases
+# --------------------------------------------------------------------------
+
+def test_index_project_coordinate_selection_is_a_gather():
+    from long_context_sparse_dim_b200.workloads import lowfreq_dims, lowfreq_projection
+    rng = np.random.default_rng(1)
+    x = rng.standard_normal((50, 128))
+    P = lowfreq_projection()
+    np.testing.assert_array_equal(oracle.index_project(x, P), x[:, lowfreq_dims()])
+
+
+def test_indexer_score_unit_query_reads_one_coordinate():
+    rng = np.random.default_rng(2)
+    k_idx = rng.standard_normal((40, 16))
+    for i in (0, 7, 15):
+        e = np.zeros(16)
+        e[i] = 1.0
+        np.testing.assert_array_equal(oracle.indexer_scores(e, k_idx), k_idx[:, i] / 4.0)
+
+
+def test_indexer_score_is_bilinear_and_symmetric():
+    rng = np.random.default_rng(3)
+    a, b = rng.standard_normal(16), rng.standard_normal(16)
+    K = rng.standard_normal((9, 16))
+    s_sum = oracle.indexer_scores(a + b, K)
+    np.testing.assert_allclose(s_sum, oracle.indexer_scores(a, K) + oracle.indexer_scores(b, K), atol=1e-12)
+    # s(a, b) == s(b, a)
+    assert abs(oracle.indexer_scores(a, b[None])[0] - oracle.indexer_scores(b, a[None])[0]) < 1e-14
+    # |a|^2 / 4 on itself
+    assert abs(oracle.indexer_scores(a, a[None])[0] - a @ a / 4) < 1e-12
+
+
+# --------------------------------------------------------------------------
+# top-p: minimality, brute force, closed forms
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("seed", range(6))
+@pytest.mark.parametrize("p", [0.05, 0.5, 0.9, 0.99])
+def test_topp_minimal_prefix(seed, p):
+    rng = np.random.default_rng(seed)
+    n = int(rng.integers(1, 400))
+    s = rng.standard_normal(n) * float(rng.choice([0.3, 1.0, 4.0]))
+    if seed % 2:
+        s = np.round(s, 1)                       # many exact ties
+    r = oracle.topp_select(s, p)
+    w = np.exp(s - s.max())
+    Z = w.sum()
+    # prefix of the (s desc, pos asc) order
+    order = sorted(range(n), key=lambda j: (-s[j], j))
+    assert sorted(order[: r.count]) == r.idx.tolist()
+    # mass reaches p and dropping the last key does not
+    assert w[r.idx].sum() >= p * Z * (1 - 1e-12)
+    assert w[order[: r.count - 1]].sum() < p * Z
+    # the threshold form describes the same set
+    pos = np.arange(n)
+    thr = (s > r.tau) | ((s == r.tau) & (pos <= r.tiepos))
+    assert np.flatnonzero(thr).tolist() == r.idx.tolist()
+
+
+@pytest.mark.parametrize("seed", range(30))
+def test_topp_brute_force_all_subsets(seed):
+    rng = np.random.default_rng(100 + seed)
+    n = int(rng.integers(1, 13))
+    s = np.round(rng.standard_normal(n) * 1.5, 1 if seed % 3 == 0 else 6)
+    p = float(rng.uniform(0.05, 0.999))
+    r = oracle.topp_select(s, p)
+    w = np.exp(s - s.max())
+    target = p * w.sum()
+    best = None
+    for size in range(1, n + 1):
+        masses = [w[list(c)].sum() for c in itertools.combinations(range(n), size)]
+        if max(masses) >= target:
+            best = size
+            break
+    assert r.count == best
+    # no other subset of that size carries more mass
+    top_mass = max(w[list(c)].sum() for c in itertools.combinations(range(n), best))
+    assert abs(w[r.idx].sum() - top_mass) <= 1e-12 * top_mass
+
+
+@pytest.mark.parametrize("n", [1, 2, 7, 100, 1001])
+@pytest.mark.parametrize("p", [0.013, 0.37, 0.5, 0.81, 0.999])
+def test_topp_all_equal_scores(n, p):
+    # equal weights: ceil(p n) keys, the lowest positions (pins the tie-break)
+    r = oracle.topp_select(np.full(n, 0.7), p)
+    k = math.ceil(p * n - 1e-9)
+    assert r.count == k
+    assert r.idx.tolist() == list(range(k))
+    assert r.tiepos == k - 1
+
+
+def test_topp_single_dominant_key():
+    s = np.zeros(50)
+    s[17] = 10.0                                  # e^10 / (e^10 + 49) > 0.99
+    r = oracle.topp_select(s, 0.99)
+    assert r.idx.tolist() == [17]
+    rng = np.random.default_rng(4)
+    V = rng.standard_normal((50, 8))
+    o = oracle.attend(np.zeros(8), rng.standard_normal((50, 8)), V, r.idx, 1.0)
+    np.testing.assert_array_equal(o, V[17])
+
+
+@pytest.mark.parametrize("na,nb,a,b,p", [(3, 40, 2.0, 0.0, 0.3), (3, 40, 2.0, 0.0, 0.9),
+                                         (10, 10, 1.0, -1.0, 0.5), (1, 99, 5.0, 0.0, 0.8),
+                                         (64, 4000, 1.0, 0.0, 0.95)])
+def test_topp_two_level_closed_form(na, nb, a, b, p):
+    # n_a keys at score a (> b), n_b at b: k* = ceil(pZ/e^a) if <= n_a, else n_a + ceil((pZ - n_a e^a)/e^b)
+    rng = np.random.default_rng(na * 7 + nb)
+    s = np.array([a] * na + [b] * nb)
+    perm = rng.permutation(na + nb)
+    s = s[perm]
+    Z = na * math.exp(a) + nb * math.exp(b)
+    k_a = math.ceil(p * Z / math.exp(a) - 1e-12)
+    k = k_a if k_a <= na else na + math.ceil((p * Z - na * math.exp(a)) / math.exp(b) - 1e-12)
+    r = oracle.topp_select(s, p)
+    assert r.count == k
+    hi = np.flatnonzero(s == a)
+    lo = np.flatnonzero(s == b)
+    want = sorted(hi[:k].tolist()) if k <= na else sorted(hi.tolist() + lo[: k - na].tolist())
+    assert r.idx.tolist() == want
+
+
+def test_topp_p_one_selects_everything_and_p_invalid():
+    s = np.random.default_rng(0).standard_normal(33) * 30.0   # weights underflow to ~0
+    assert oracle.topp_select(s, 1.0).count == 33
+    for bad in (0.0, -0.5, float("nan")):
+        with pytest.raises(ValueError):
+            oracle.topp_select(s, bad)
+
+
+def test_topp_signed_zero_and_negative_scores():
+    s = np.array([-0.0, 0.0, -1.5, -0.0, -3.0])
+    r = oracle.topp_select(s, 0.5)
+    # -0 == +0: the three zero scores tie and are taken by position
+    w = np.exp(s - 0.0)
+    k = 1
+    while w[[0, 1, 3][:k]].sum() < 0.5 * w.sum():
+        k += 1
+    assert r.idx.tolist() == [0, 1, 3][:k]
+
+
+# --------------------------------------------------------------------------
+# attention: p = 1 and W >= context reduce to full causal attention
+# (independent library routine: torch scaled_dot_product_attention in fp64)
+# --------------------------------------------------------------------------
+
+def _sdpa_causal(q, k, v, lens_b, T, scale):
+    """q [Hq, T, D], k/v [Hkv, n, D] -> [Hq, T, D]; queries are the last T of n positions."""
+    Hq, Hkv = q.shape[0], k.shape[0]
+    G = Hq // Hkv
+    n = lens_b
+    kk = torch.from_numpy(np.repeat(k[:, :n], G, axis=0)).double()
+    vv = torch.from_numpy(np.repeat(v[:, :n], G, axis=0)).double()
+    qq = torch.from_numpy(q).double()
+    qpos = torch.arange(T) + n - T
+    mask = torch.arange(n)[None, :] <= qpos[:, None]
+    return torch.nn.functional.scaled_dot_product_attention(qq, kk, vv, attn_mask=mask, scale=scale).numpy()
+
+
+def _layer(seed, B=2, Hq=4, Hkv=2, R=1, N=70, T=70, W=16, p=0.9, storage="f64"):
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((B, Hq, T, 32))
+    k = rng.standard_normal((B, Hkv, N, 32))
+    v = rng.standard_normal((B, Hkv, N, 32))
+    P = rng.standard_normal((R, 16, 32))
+    lens = np.array([N] * (B - 1) + [max(T, N - 9)])
+    return q, k, v, P, lens
+
+
+@pytest.mark.parametrize("T", [1, 5, 70])
+def test_p_one_and_wide_window_equal_full_causal_attention(T):
+    q, k, v, P, lens = _layer(7, T=T)
+    N = k.shape[2]
+    L = oracle.LayerOracle(q, k, v, P, lens, R=1, W=N + 5, p=1.0, storage="f64")
+    res = L.run()
+    for b in range(q.shape[0]):
+        ref = _sdpa_causal(q[b], k[b], v[b], int(lens[b]), T, L.scale)
+        got = np.stack([np.stack([res[(b, h, t)].o for t in range(T)]) for h in range(q.shape[1])])
+        np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_window_equals_sdpa_band():
+    q, k, v, P, lens = _layer(8, T=70, W=9)
+    L = oracle.LayerOracle(q, k, v, P, lens, R=0, W=9, p=0.5, storage="f64")
+    b, h = 1, 3
+    n = int(lens[b])
+    T = q.shape[2]
+    qpos = np.arange(T) + n - T
+    mask = (np.arange(n)[None, :] <= qpos[:, None]) & (np.arange(n)[None, :] > qpos[:, None] - 9)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q[b, h][None]), torch.from_numpy(k[b, h // 2, :n][None]),
+        torch.from_numpy(v[b, h // 2, :n][None]), attn_mask=torch.from_numpy(mask)[None], scale=L.scale)[0].numpy()
+    got = np.stack([L.query(b, h, t).o for t in range(T)])
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_window_one_returns_own_value():
+    q, k, v, P, lens = _layer(9, T=4)
+    L = oracle.LayerOracle(q, k, v, P, lens, R=0, W=1, p=0.5, storage="f64")
+    for t in range(4):
+        pos = L.pos(0, t)
+        np.testing.assert_array_equal(L.query(0, 1, t).o, v[0, 0, pos])
+
+
+def test_ragged_length_equals_truncated_cache():
+    q, k, v, P, lens = _layer(10, T=1, N=50)
+    lens = np.array([50, 31])
+    L = oracle.LayerOracle(q, k, v, P, lens, R=1, W=8, p=0.8, storage="f64")
+    Lt = oracle.LayerOracle(q[1:], k[1:, :, :31], v[1:, :, :31], P, [31], R=1, W=8, p=0.8, storage="f64")
+    for h in range(4):
+        np.testing.assert_array_equal(L.query(1, h, 0).o, Lt.query(0, h, 0).o)
+
+
+def test_empty_candidate_set_gives_zero():
+    q, k, v, P, lens = _layer(11, T=6, N=6)
+    lens = np.array([6, 6])
+    L = oracle.LayerOracle(q, k, v, P, lens, R=1, W=3, p=0.5, storage="f64")
+    L.lens = np.array([6, 4])                   # two of the six queries sit before position 0
+    assert L.query(1, 0, 0).sel.count == 0
+    np.testing.assert_array_equal(L.query(1, 0, 0).o, 0.0)
+    np.testing.assert_array_equal(L.query(1, 3, 1).o, 0.0)
+
+
+# --------------------------------------------------------------------------
+# needles: the planted keys are recalled (the pages' ">90% recall")
+# --------------------------------------------------------------------------
+
+def test_needle_recall_small_decode():
+    from long_context_sparse_dim_b200 import workloads as wl
+    inst = wl.generate(wl.DECODE_N4K_F32)
+    L = oracle.LayerOracle(inst.q, inst.k, inst.v, inst.P, inst.lens, R=1, W=512, p=0.9, storage="f32")
+    res = L.run()
+    hit, tot = oracle.needle_recall(res, inst.needles)
+    assert tot == 16
+    assert hit / tot >= 0.9
+
+
+# --------------------------------------------------------------------------
+# the pins reject planted mistakes
+# --------------------------------------------------------------------------
+
+def _mutant_tie_high(s, p):
+    s = np.asarray(s, dtype=np.float64)
+    n = s.shape[0]
+    w = np.exp(s - s.max())
+    order = np.lexsort((-np.arange(n), -s))      # wrong: higher position first
+    cum = np.cumsum(w[order])
+    k = n if p >= 1 else int(np.searchsorted(cum, p * w.sum())) + 1
+    return ro.Selection(np.sort(order[:k]), k, s[order[k - 1]], int(order[k - 1]), w.sum(), 0.0, order)
+
+
+_TRUE_TOPP = ro.topp_select
+
+
+def _mutant_off_by_one(s, p):
+    r = _TRUE_TOPP(s, p)
+    n = len(s)
+    k = min(n, r.count + 1)
+    return ro.Selection(np.sort(r.order[:k]), k, s[r.order[k - 1]], int(r.order[k - 1]), r.Z, 0.0, r.order)
+
+
+def _mutant_no_temperature_shift(s, p):
+    # wrong: weights exp(2 s) (a dropped /2 somewhere in the exponent)
+    return _TRUE_TOPP(2.0 * np.asarray(s, dtype=np.float64), p)
+
+
+@pytest.mark.parametrize("mutant", [_mutant_tie_high, _mutant_off_by_one, _mutant_no_temperature_shift])
+def test_mutants_are_caught(mutant, monkeypatch):
+    monkeypatch.setattr(ro, "topp_select", mutant)
+    monkeypatch.setattr(oracle, "topp_select", mutant)
+    failures = 0
+    for fn in (test_topp_hand_fixture,
+               lambda: test_topp_all_equal_scores(7, 0.37),
+               lambda: test_topp_two_level_closed_form(3, 40, 2.0, 0.0, 0.3)):
+        try:
+            fn()
+        except AssertionError:
+            failures += 1
+    assert failures >= 1
