@@ -1,0 +1,404 @@
+"""Benchmark of the RTPurbo decode path on B200 (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+
+A step is one decode step of one attention layer for the whole batch:
+project the newest key row and the queries (a1), score every cached key with
+the 16-dim indexer and cut at top-p (a2+a3), attend the selected keys
+(retrieval heads, a4) and the last W keys (local heads, a5).  All inputs are
+seeded synthetic tensors resident in HBM before the timed region; the timed
+region replays CUDA graphs of exactly K steps, bracketed by a barrier and a
+device synchronisation, and the step time is the max over ranks.  Each rank
+runs its own replica of the workload (weak scaling, no data-path collective).
+
+``value`` is decode tokens/s (sequences advanced by one token per second,
+summed over ranks).  ``e2e`` is the same metric through the public API with
+host buffers: each step copies the new token's q/k/v from pinned host memory,
+makes the C-ABI calls, and reads the output back.  ``--impl reference`` times
+the CPU oracle on the same workload instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from long_context_sparse_dim_b200 import workloads as wls  # noqa: E402
+
+DECODE_WORKLOADS = {w.name: w for w in (wls.DECODE_B8_N32K, wls.DECODE_N4K_F32, wls.DECODE_B4_N128K)}
+DEFAULT_WORKLOAD = wls.DECODE_B8_N32K.name
+METRIC = "decode sparse-attn tokens/s"
+ROW_BYTES = {"bf16": 2 * 128 * 2, "f32": 2 * 128 * 4}  # one K row + one V row
+L2_BYTES = 126 * 2 ** 20
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    if ws == 1:
+        return 0, 1, 0
+    import torch.distributed as dist
+    import datetime
+    backend = os.environ.get("RTP_BENCH_BACKEND", "nccl")
+    dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return dist.get_rank(), ws, int(os.environ.get("LOCAL_RANK", "0"))
+
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int, device=None):
+    if world > 1:
+        import torch.distributed as dist
+        if device is not None:
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# --------------------------------------------------------------------------
+# clocks
+# --------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out = ""
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------
+# reference arm: the CPU oracle
+# --------------------------------------------------------------------------
+
+def _oracle_cores():
+    try:
+        from threadpoolctl import threadpool_info
+        n = max([d.get("num_threads", 1) for d in threadpool_info()] or [1])
+        return int(n)
+    except Exception:
+        return 1
+
+
+def oracle_step_runner(inst, wl):
+    """Returns run(b) that computes every head of sequence b with the CPU oracle."""
+    import oracle
+    L = oracle.LayerOracle(inst.q, inst.k, inst.v, inst.P, inst.lens, R=wl.R, W=wl.W,
+                           p=float(np.float32(wl.p)), storage=wl.dtype)
+    for b in range(wl.B):            # the projected-key cache exists before decoding starts
+        for kvh in range(wl.R):
+            L.k_idx(b, kvh)
+
+    def run(b):
+        for h in range(wl.Hq):
+            L.query(b, h, 0)
+    return run
+
+
+def cpu_baseline(inst, wl, budget_s=10.0):
+    run = oracle_step_runner(inst, wl)
+    t0 = time.perf_counter()
+    done = 0
+    while True:
+        run(done % wl.B)
+        done += 1
+        if time.perf_counter() - t0 >= budget_s or done >= 4 * wl.B:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": done / dt, "unit": "tokens/s", "cores": _oracle_cores(), "kind": "oracle",
+            "sample": f"{done} sequences x all {wl.Hq} heads of {wl.name} (one token each), "
+                      f"projected-key cache prebuilt, {dt:.1f} s"}
+
+
+def run_reference(args, wl, rank):
+    if rank != 0:
+        return 0
+    inst = wls.generate(wl)
+    run = oracle_step_runner(inst, wl)
+    for i in range(args.warmup):
+        run(i % wl.B)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        run(i % wl.B)
+    dt = time.perf_counter() - t0
+    v = args.steps / dt
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": wl.name, "B": wl.B, "N": wl.N, "Hq": wl.Hq, "Hkv": wl.Hkv,
+                                             "retrieval_kv_heads": wl.R, "W": wl.W, "p": wl.p},
+            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": _oracle_cores(), "kind": "oracle",
+                             "sample": f"each step = all {wl.Hq} heads of one sequence of {wl.name}"},
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------------
+# our arm
+# --------------------------------------------------------------------------
+
+def _traffic_record(kernel: str):
+    """DRAM bytes per launch from a committed ncu summary, if the kernel source is unchanged."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)[kernel]
+        with open(os.path.join(ROOT, rec["source"]), "rb") as f:
+            sha = hashlib.sha1(f.read()).hexdigest()
+        if sha != rec["source_sha1"]:
+            return None
+        return rec
+    except Exception:
+        return None
+
+
+def run_ours(args, wl, rank, world, local_rank):
+    import torch
+    from long_context_sparse_dim_b200 import rtp  # noqa: F401  (fails loudly without librtp.so)
+    from long_context_sparse_dim_b200.layer import DecodeLayer
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    inst = wls.generate(wl)
+    dt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+    q = torch.from_numpy(inst.q).to(dev, dt)
+    k = torch.from_numpy(inst.k).to(dev, dt)
+    v = torch.from_numpy(inst.v).to(dev, dt)
+    P = torch.from_numpy(inst.P).to(dev, torch.float32)
+    layer = DecodeLayer(q, k, v, P, R=wl.R, W=wl.W, p=wl.p)
+    layer.build_index()
+    torch.cuda.synchronize()
+
+    # warm-up (also loads every kernel)
+    for _ in range(max(args.warmup, 1)):
+        layer.step()
+    torch.cuda.synchronize()
+
+    # graphs of the timed steps, events around the dominant kernel (sparse attention)
+    chunk = 500
+    graphs, ev = [], []
+    s = torch.cuda.Stream(dev)
+    s.wait_stream(torch.cuda.current_stream(dev))
+    remaining = args.steps
+    with torch.cuda.stream(s):
+        while remaining > 0:
+            n = min(chunk, remaining)
+            g = torch.cuda.CUDAGraph()
+            pairs = [(torch.cuda.Event(enable_timing=True, external=True),
+                      torch.cuda.Event(enable_timing=True, external=True)) for _ in range(n)]
+            with torch.cuda.graph(g, stream=s):
+                for i in range(n):
+                    _step_with_events(layer, pairs[i])
+            graphs.append(g)
+            ev.extend(pairs)
+            remaining -= n
+    torch.cuda.current_stream(dev).wait_stream(s)
+    torch.cuda.synchronize()
+    for g in graphs[:1]:
+        g.replay()                     # graph upload / first-launch costs stay untimed
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    time.sleep(0.2)
+    barrier(world, dev)
+    torch.cuda.synchronize()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record()
+    for g in graphs:
+        g.replay()
+    t_end.record()
+    torch.cuda.synchronize()
+    barrier(world, dev)
+    clock_info = clocks.stop()
+    step_ms_local = t_start.elapsed_time(t_end) / args.steps
+    step_ms = max_over_ranks(step_ms_local, world, dev)
+    attn_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+
+    # realised selection: union of the GQA group's masks per (sequence, KV head)
+    m = layer.sel.mask.view(torch.int32).cpu().numpy().view(np.uint32)
+    G, R = wl.G, wl.R
+    union_rows = 0
+    sel_rows = 0
+    for b in range(wl.B):
+        for kh in range(R):
+            rows = m[(b * R * G + kh * G):(b * R * G + (kh + 1) * G)]
+            u = np.bitwise_or.reduce(rows, axis=0)
+            union_rows += int(np.unpackbits(u.view(np.uint8)).sum())
+            sel_rows += int(np.unpackbits(rows.view(np.uint8)).sum())
+    row_b = ROW_BYTES[wl.dtype]
+    attn_bytes = union_rows * row_b
+    peak, peak_kind = _peaks()
+    achieved = attn_bytes / (attn_ms * 1e-3) / 1e9
+    idx_bytes = wl.B * R * wl.N * 16 * (2 if wl.dtype == "bf16" else 4)
+    win_bytes = wl.B * (wl.Hkv - R) * min(wl.W, wl.N) * row_b
+    step_bytes = idx_bytes + attn_bytes + win_bytes
+    tr = _traffic_record("attn_decode_bf16_kernel" if wl.dtype == "bf16" else "attn_decode_f32_kernel")
+
+    # end to end through the public API with host buffers
+    e2e = _e2e(layer, inst, wl, dev, max(min(args.steps, 200), 20))
+
+    line = {
+        "metric": METRIC, "value": world * wl.B / (step_ms * 1e-3), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic",
+        "config": {"workload": wl.name, "B": wl.B, "N": wl.N, "Hq": wl.Hq, "Hkv": wl.Hkv,
+                   "retrieval_kv_heads": R, "W": wl.W, "p": wl.p,
+                   "l2": f"inputs larger than L2: {step_bytes / 1e6:.0f} MB touched per step vs 126 MB L2, no flush",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": {"kernel": "attn_decode_bf16_kernel" if wl.dtype == "bf16" else "attn_decode_f32_kernel",
+                     "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "peak_kind": peak_kind, "traffic": tr["dram_bytes_per_launch"] if tr else None,
+                     "algorithmic_bytes": attn_bytes, "units": union_rows, "bytes_per_unit": row_b,
+                     "ms_per_launch": attn_ms},
+        "step_roofline": {"bytes": step_bytes, "achieved_gbs": step_bytes / (step_ms * 1e-3) / 1e9,
+                          "frac": step_bytes / (step_ms * 1e-3) / 1e9 / peak},
+        "selection": {"mean_selected_fraction": sel_rows / (wl.B * R * G * wl.N),
+                      "mean_group_union_fraction": union_rows / (wl.B * R * wl.N)},
+        "e2e": e2e,
+        "gpu_launches": 5 * args.steps,
+        "clocks": clock_info,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(inst, wl, args.cpu_budget)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del graphs
+    return 0
+
+
+def _step_with_events(layer, pair):
+    """One decode step with timing events around the sparse-attention launch."""
+    from long_context_sparse_dim_b200 import rtp
+    if layer.R:
+        n = layer.N
+        rtp.index_project(layer.k_ret[:, :, n - 1: n], layer.P, layer.k_idx[:, :, n - 1: n])
+        rtp.index_project(layer.q_ret, layer.P, layer.q_idx)
+        rtp.topp_select(layer.q_idx, layer.k_idx, layer.lens, layer.p, layer.sel, layer.ws_sel)
+        pair[0].record()
+        rtp.sparse_attn_decode(layer.q_ret, layer.k_ret, layer.v_ret, layer.lens, layer.sel, layer.scale,
+                               layer.o_ret, layer.ws_ret)
+        pair[1].record()
+    if layer.Hkv > layer.R:
+        rtp.window_attn(layer.q_loc, layer.k_loc, layer.v_loc, layer.lens, layer.W, layer.scale, layer.o_loc,
+                        layer.ws_loc)
+
+
+def _e2e(layer, inst, wl, dev, steps):
+    import torch
+    dt = layer.q.dtype
+    n = wl.N
+    h_q = torch.from_numpy(inst.q).to(dt).pin_memory()
+    h_k = torch.from_numpy(np.ascontiguousarray(inst.k[:, :, n - 1: n])).to(dt).pin_memory()
+    h_v = torch.from_numpy(np.ascontiguousarray(inst.v[:, :, n - 1: n])).to(dt).pin_memory()
+    h_o = torch.empty(layer.o.shape, dtype=layer.o.dtype).pin_memory()
+    h2d = h_q.numel() * h_q.element_size() + 2 * h_k.numel() * h_k.element_size()
+    d2h = h_o.numel() * h_o.element_size()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(steps):
+        layer.q.copy_(h_q, non_blocking=True)
+        layer.k[:, :, n - 1: n].copy_(h_k, non_blocking=True)
+        layer.v[:, :, n - 1: n].copy_(h_v, non_blocking=True)
+        layer.step()
+        h_o.copy_(layer.o, non_blocking=True)
+        torch.cuda.current_stream().synchronize()
+    t1.record()
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1) / steps
+    return {"value": wl.B / (ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h), "ms_per_step": ms, "steps": steps}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(DECODE_WORKLOADS))
+    ap.add_argument("--cpu-budget", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        args.warmup = 3
+    wl = DECODE_WORKLOADS[args.workload]
+    rank, world, local_rank = _dist()
+    try:
+        if args.impl == "reference":
+            return run_reference(args, wl, rank)
+        return run_ours(args, wl, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,56 @@
+// Host-side launcher interfaces between the C ABI (rtp_api.cu) and the kernels.
+// Arguments arrive here already validated.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace rtp {
+
+struct LaunchIndexProject {
+  View4 x;
+  const float* P;
+  MutView4 out;
+  int64_t B, H, HP, N;
+  bool in_bf16, out_bf16;
+};
+cudaError_t launch_index_project(const LaunchIndexProject& a, cudaStream_t stream);
+
+// Top-p selection, decode form (one query per (b, h)).
+struct LaunchToppDecode {
+  View4 q_idx;   // [B, Hq, 1, 16]
+  View4 k_idx;   // [B, Hk, N, 16]
+  const int32_t* lens;
+  int64_t B, Hq, Hk, N;
+  float p;
+  bool bf16;
+  uint32_t* tau_bits;
+  int32_t* tiepos;
+  int32_t* count;
+  uint32_t* mask;
+  int64_t mask_words;
+};
+cudaError_t launch_topp_decode(const LaunchToppDecode& a, cudaStream_t stream);
+bool topp_decode_supported(int64_t N);
+
+// Decode attention: sparse (mask given) or sliding window (W > 0).
+struct LaunchAttnDecode {
+  View4 q;       // [B, Hq, 1, 128]
+  View4 k, v;    // [B, Hk, N, 128]
+  const int32_t* lens;
+  const uint32_t* mask;  // sparse mode: [B*Hq, mask_words]
+  int64_t mask_words;
+  int64_t B, Hq, Hk, N;
+  int32_t W;             // > 0: window mode
+  float scale;
+  bool bf16;             // q/k/v dtype
+  MutView4 o;            // [B, Hq, 1, 128]
+  bool o_bf16;
+  void* ws;
+};
+size_t attn_decode_workspace_bytes(int64_t B, int64_t Hq, int64_t Hk, int64_t N, int32_t W);
+cudaError_t launch_attn_decode(const LaunchAttnDecode& a, cudaStream_t stream);
+
+}  // namespace rtp

@@ -1,0 +1,270 @@
+// C ABI of librtp.so: argument validation on the host, then dispatch to the
+// kernels.  Nothing is launched and nothing is written when a check fails.
+#include <math.h>
+#include <stdint.h>
+
+#include "launch.h"
+#include "rtp.h"
+
+namespace {
+
+thread_local int32_t g_last_cuda_error = 0;
+
+rtp_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return RTP_OK;
+  g_last_cuda_error = (int32_t)e;
+  return RTP_ERR_CUDA;
+}
+
+int64_t elt_size(int32_t dt) { return dt == RTP_F32 ? 4 : 2; }
+
+bool dtype_ok(int32_t dt) { return dt == RTP_F32 || dt == RTP_BF16; }
+
+// A 4-D tensor with the given last dimension, contiguous last dim, 16-byte
+// aligned base and (for dims longer than 1) 16-byte aligned strides.
+rtp_status check4(const rtp_tensor* t, int64_t last) {
+  if (!t || !t->data) return RTP_ERR_INVALID_ARG;
+  if (t->ndim != 4) return RTP_ERR_SHAPE;
+  if (!dtype_ok(t->dtype)) return RTP_ERR_DTYPE;
+  for (int i = 0; i < 4; ++i)
+    if (t->shape[i] < 0 || t->stride[i] < 0) return RTP_ERR_SHAPE;
+  if (t->shape[3] != last) return RTP_ERR_SHAPE;
+  if (t->shape[0] > INT32_MAX || t->shape[1] > INT32_MAX || t->shape[2] > INT32_MAX) return RTP_ERR_SHAPE;
+  if (t->stride[3] != 1) return RTP_ERR_ALIGNMENT;
+  if (((uintptr_t)t->data) % 16) return RTP_ERR_ALIGNMENT;
+  const int64_t es = elt_size(t->dtype);
+  for (int i = 0; i < 3; ++i)
+    if (t->shape[i] > 1 && (t->stride[i] * es) % 16) return RTP_ERR_ALIGNMENT;
+  return RTP_OK;
+}
+
+rtp::View4 view(const rtp_tensor* t) { return rtp::View4{t->data, t->stride[0], t->stride[1], t->stride[2]}; }
+rtp::MutView4 mview(const rtp_tensor* t) {
+  return rtp::MutView4{t->data, t->stride[0], t->stride[1], t->stride[2]};
+}
+
+bool same_bhn(const rtp_tensor* a, const rtp_tensor* b) {
+  return a->shape[0] == b->shape[0] && a->shape[1] == b->shape[1] && a->shape[2] == b->shape[2];
+}
+
+rtp_status check_workspace(void* ws, size_t bytes, size_t need) {
+  if (need == 0) return RTP_OK;
+  if (!ws) return RTP_ERR_WORKSPACE;
+  if (((uintptr_t)ws) % 256) return RTP_ERR_ALIGNMENT;
+  if (bytes < need) return RTP_ERR_WORKSPACE;
+  return RTP_OK;
+}
+
+// K and V of one layer: same shape/dtype, last dim 128.
+rtp_status check_kv(const rtp_tensor* k, const rtp_tensor* v) {
+  rtp_status s;
+  if ((s = check4(k, 128)) != RTP_OK) return s;
+  if ((s = check4(v, 128)) != RTP_OK) return s;
+  if (!same_bhn(k, v)) return RTP_ERR_SHAPE;
+  if (k->dtype != v->dtype) return RTP_ERR_DTYPE;
+  return RTP_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* rtp_status_string(rtp_status s) {
+  switch (s) {
+    case RTP_OK: return "ok";
+    case RTP_ERR_INVALID_ARG: return "invalid argument";
+    case RTP_ERR_SHAPE: return "bad shape";
+    case RTP_ERR_DTYPE: return "unsupported dtype";
+    case RTP_ERR_ALIGNMENT: return "misaligned pointer or stride";
+    case RTP_ERR_WORKSPACE: return "workspace missing or too small";
+    case RTP_ERR_CUDA: return "CUDA error";
+    case RTP_ERR_UNSUPPORTED: return "unsupported configuration";
+    default: return "unknown status";
+  }
+}
+
+int32_t rtp_last_cuda_error(void) { return g_last_cuda_error; }
+
+int32_t rtp_version(void) { return 100; }
+
+// ---- a1 ------------------------------------------------------------------------
+rtp_status rtp_index_project(const rtp_tensor* x, const rtp_tensor* P, const rtp_tensor* x_idx,
+                             rtp_stream_t stream) {
+  rtp_status s;
+  if ((s = check4(x, 128)) != RTP_OK) return s;
+  if ((s = check4(x_idx, 16)) != RTP_OK) return s;
+  if (!P || !P->data) return RTP_ERR_INVALID_ARG;
+  if (P->dtype != RTP_F32) return RTP_ERR_DTYPE;
+  if (P->ndim != 3 || P->shape[1] != 16 || P->shape[2] != 128 || P->shape[0] < 1) return RTP_ERR_SHAPE;
+  if (P->stride[2] != 1 || P->stride[1] != 128 || P->stride[0] != 16 * 128) return RTP_ERR_ALIGNMENT;
+  if (((uintptr_t)P->data) % 16) return RTP_ERR_ALIGNMENT;
+  if (!same_bhn(x, x_idx)) return RTP_ERR_SHAPE;
+  if (x->shape[1] % P->shape[0]) return RTP_ERR_SHAPE;
+  rtp::LaunchIndexProject a;
+  a.x = view(x);
+  a.P = static_cast<const float*>(P->data);
+  a.out = mview(x_idx);
+  a.B = x->shape[0];
+  a.H = x->shape[1];
+  a.HP = P->shape[0];
+  a.N = x->shape[2];
+  a.in_bf16 = x->dtype == RTP_BF16;
+  a.out_bf16 = x_idx->dtype == RTP_BF16;
+  return cuda_status(rtp::launch_index_project(a, (cudaStream_t)stream));
+}
+
+// ---- a2 + a3 ---------------------------------------------------------------------
+size_t rtp_topp_select_workspace_size(int64_t B, int64_t Hq, int64_t T, int64_t Hk, int64_t N) {
+  (void)B; (void)Hq; (void)Hk; (void)N;
+  if (T <= 1) return 0;  // the decode cut lives entirely in on-chip memory
+  return 0;
+}
+
+rtp_status rtp_topp_select(const rtp_tensor* q_idx, const rtp_tensor* k_idx, const int32_t* lens, float p,
+                           const rtp_selection* out, void* workspace, size_t workspace_bytes,
+                           rtp_stream_t stream) {
+  rtp_status s;
+  if ((s = check4(q_idx, 16)) != RTP_OK) return s;
+  if ((s = check4(k_idx, 16)) != RTP_OK) return s;
+  if (q_idx->dtype != k_idx->dtype) return RTP_ERR_DTYPE;
+  if (q_idx->shape[0] != k_idx->shape[0]) return RTP_ERR_SHAPE;
+  if (k_idx->shape[1] < 1 || q_idx->shape[1] % k_idx->shape[1]) return RTP_ERR_SHAPE;
+  if (!(p > 0.f) || isnan(p)) return RTP_ERR_INVALID_ARG;
+  if (!out || !out->tau_bits || !out->tiepos || !out->count) return RTP_ERR_INVALID_ARG;
+  const int64_t N = k_idx->shape[2];
+  if (out->mask && out->mask_words < (N + 31) / 32) return RTP_ERR_SHAPE;
+  const int64_t T = q_idx->shape[2];
+  if ((s = check_workspace(workspace, workspace_bytes,
+                           rtp_topp_select_workspace_size(q_idx->shape[0], q_idx->shape[1], T,
+                                                          k_idx->shape[1], N))) != RTP_OK)
+    return s;
+  if (T != 1) return RTP_ERR_UNSUPPORTED;
+  if (!rtp::topp_decode_supported(N)) return RTP_ERR_UNSUPPORTED;
+  rtp::LaunchToppDecode a;
+  a.q_idx = view(q_idx);
+  a.k_idx = view(k_idx);
+  a.lens = lens;
+  a.B = q_idx->shape[0];
+  a.Hq = q_idx->shape[1];
+  a.Hk = k_idx->shape[1];
+  a.N = N;
+  a.p = p;
+  a.bf16 = q_idx->dtype == RTP_BF16;
+  a.tau_bits = out->tau_bits;
+  a.tiepos = out->tiepos;
+  a.count = out->count;
+  a.mask = out->mask;
+  a.mask_words = out->mask_words;
+  return cuda_status(rtp::launch_topp_decode(a, (cudaStream_t)stream));
+}
+
+// ---- a4 decode -------------------------------------------------------------------
+size_t rtp_sparse_attn_decode_workspace_size(int64_t B, int64_t Hq, int64_t Hk, int64_t N) {
+  return rtp::attn_decode_workspace_bytes(B, Hq, Hk, N, 0);
+}
+
+static rtp_status check_decode_common(const rtp_tensor* q, const rtp_tensor* k, const rtp_tensor* v,
+                                      const rtp_tensor* o, float scale) {
+  rtp_status s;
+  if ((s = check4(q, 128)) != RTP_OK) return s;
+  if ((s = check_kv(k, v)) != RTP_OK) return s;
+  if ((s = check4(o, 128)) != RTP_OK) return s;
+  if (q->dtype != k->dtype) return RTP_ERR_DTYPE;
+  if (q->shape[0] != k->shape[0] || o->shape[0] != q->shape[0] || o->shape[1] != q->shape[1] ||
+      o->shape[2] != q->shape[2])
+    return RTP_ERR_SHAPE;
+  if (k->shape[1] < 1 || q->shape[1] % k->shape[1]) return RTP_ERR_SHAPE;
+  if (q->shape[1] / k->shape[1] > 8) return RTP_ERR_SHAPE;
+  if (!isfinite(scale)) return RTP_ERR_INVALID_ARG;
+  return RTP_OK;
+}
+
+rtp_status rtp_sparse_attn_decode(const rtp_tensor* q, const rtp_tensor* k, const rtp_tensor* v,
+                                  const int32_t* lens, const rtp_selection* sel, float scale,
+                                  const rtp_tensor* o, void* workspace, size_t workspace_bytes,
+                                  rtp_stream_t stream) {
+  rtp_status s;
+  if ((s = check_decode_common(q, k, v, o, scale)) != RTP_OK) return s;
+  if (q->shape[2] != 1) return RTP_ERR_SHAPE;
+  if (!sel || !sel->mask) return RTP_ERR_INVALID_ARG;
+  const int64_t N = k->shape[2];
+  if (sel->mask_words < (N + 31) / 32) return RTP_ERR_SHAPE;
+  const size_t need = rtp_sparse_attn_decode_workspace_size(q->shape[0], q->shape[1], k->shape[1], N);
+  if ((s = check_workspace(workspace, workspace_bytes, need)) != RTP_OK) return s;
+  rtp::LaunchAttnDecode a;
+  a.q = view(q);
+  a.k = view(k);
+  a.v = view(v);
+  a.lens = lens;
+  a.mask = sel->mask;
+  a.mask_words = sel->mask_words;
+  a.B = q->shape[0];
+  a.Hq = q->shape[1];
+  a.Hk = k->shape[1];
+  a.N = N;
+  a.W = 0;
+  a.scale = scale;
+  a.bf16 = q->dtype == RTP_BF16;
+  a.o = mview(o);
+  a.o_bf16 = o->dtype == RTP_BF16;
+  a.ws = workspace;
+  return cuda_status(rtp::launch_attn_decode(a, (cudaStream_t)stream));
+}
+
+// ---- a4 prefill --------------------------------------------------------------------
+size_t rtp_sparse_attn_prefill_workspace_size(int64_t B, int64_t Hq, int64_t T, int64_t Hk, int64_t N) {
+  (void)B; (void)Hq; (void)T; (void)Hk; (void)N;
+  return 0;
+}
+
+rtp_status rtp_sparse_attn_prefill(const rtp_tensor* q, const rtp_tensor* k, const rtp_tensor* v,
+                                   const rtp_tensor* q_idx, const rtp_tensor* k_idx, const int32_t* lens,
+                                   const rtp_selection* sel, float scale, const rtp_tensor* o,
+                                   void* workspace, size_t workspace_bytes, rtp_stream_t stream) {
+  (void)lens; (void)workspace; (void)workspace_bytes; (void)stream;
+  rtp_status s;
+  if ((s = check_decode_common(q, k, v, o, scale)) != RTP_OK) return s;
+  if ((s = check4(q_idx, 16)) != RTP_OK) return s;
+  if ((s = check4(k_idx, 16)) != RTP_OK) return s;
+  if (!sel || !sel->tau_bits || !sel->tiepos) return RTP_ERR_INVALID_ARG;
+  return RTP_ERR_UNSUPPORTED;
+}
+
+// ---- a5 ----------------------------------------------------------------------------
+size_t rtp_window_attn_workspace_size(int64_t B, int64_t Hq, int64_t T, int64_t Hk, int64_t N, int32_t W) {
+  if (T <= 1) return rtp::attn_decode_workspace_bytes(B, Hq, Hk, N, W < 1 ? 1 : W);
+  return 0;
+}
+
+rtp_status rtp_window_attn(const rtp_tensor* q, const rtp_tensor* k, const rtp_tensor* v, const int32_t* lens,
+                           int32_t W, float scale, const rtp_tensor* o, void* workspace,
+                           size_t workspace_bytes, rtp_stream_t stream) {
+  rtp_status s;
+  if ((s = check_decode_common(q, k, v, o, scale)) != RTP_OK) return s;
+  if (W < 1) return RTP_ERR_INVALID_ARG;
+  const int64_t T = q->shape[2];
+  const int64_t N = k->shape[2];
+  const size_t need = rtp_window_attn_workspace_size(q->shape[0], q->shape[1], T, k->shape[1], N, W);
+  if ((s = check_workspace(workspace, workspace_bytes, need)) != RTP_OK) return s;
+  if (T != 1) return RTP_ERR_UNSUPPORTED;
+  rtp::LaunchAttnDecode a;
+  a.q = view(q);
+  a.k = view(k);
+  a.v = view(v);
+  a.lens = lens;
+  a.mask = nullptr;
+  a.mask_words = 0;
+  a.B = q->shape[0];
+  a.Hq = q->shape[1];
+  a.Hk = k->shape[1];
+  a.N = N;
+  a.W = W;
+  a.scale = scale;
+  a.bf16 = q->dtype == RTP_BF16;
+  a.o = mview(o);
+  a.o_bf16 = o->dtype == RTP_BF16;
+  a.ws = workspace;
+  return cuda_status(rtp::launch_attn_decode(a, (cudaStream_t)stream));
+}
+
+}  // extern "C"

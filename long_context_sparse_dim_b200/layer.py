@@ -1,0 +1,78 @@
+"""One attention layer's RTPurbo decode step, sequenced over the C ABI.
+
+Holds the device buffers of one layer (KV cache views, projected-key cache,
+selection, outputs, workspaces) and issues the calls of one decode step:
+
+    a1  rtp_index_project   newest key row -> projected-key cache; queries -> q_idx
+    a3  rtp_topp_select     indexer scores + dynamic top-p cut (retrieval heads)
+    a4  rtp_sparse_attn_decode   attention over the selected keys
+    a5  rtp_window_attn     sliding-window attention (local heads)
+
+The first R KV heads are the retrieval heads ("RTPurbo: Turning Dense LLMs
+into Sparse Attention Models ...", "Three Key Insights" 1); every step of the
+computation runs in librtp.so.
+"""
+from __future__ import annotations
+
+from typing import Optional
+
+import torch
+
+from . import rtp
+
+
+class DecodeLayer:
+    def __init__(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, P: torch.Tensor,
+                 R: int, W: int, p: float, lens: Optional[torch.Tensor] = None,
+                 out_dtype: torch.dtype = torch.float32, scale: Optional[float] = None):
+        B, Hq, T, D = q.shape
+        _, Hkv, N, _ = k.shape
+        if T != 1:
+            raise ValueError("decode takes one query token per sequence")
+        self.B, self.Hq, self.Hkv, self.N, self.D = B, Hq, Hkv, N, D
+        self.G = Hq // Hkv
+        self.R, self.W, self.p = R, W, float(p)
+        self.scale = (D ** -0.5) if scale is None else scale
+        dev = q.device
+        G = self.G
+        self.q, self.k, self.v, self.P = q, k, v, P
+        self.lens = lens
+        self.lens_host = None if lens is None else [int(x) for x in lens.cpu().tolist()]
+        self.q_ret, self.q_loc = q[:, : R * G], q[:, R * G:]
+        self.k_ret, self.v_ret = k[:, :R], v[:, :R]
+        self.k_loc, self.v_loc = k[:, R:], v[:, R:]
+        self.o = torch.zeros(B, Hq, 1, D, dtype=out_dtype, device=dev)
+        self.o_ret, self.o_loc = self.o[:, : R * G], self.o[:, R * G:]
+        idx_dtype = k.dtype
+        self.k_idx = torch.zeros(B, R, N, 16, dtype=idx_dtype, device=dev)
+        self.q_idx = torch.zeros(B, R * G, 1, 16, dtype=idx_dtype, device=dev)
+        self.sel = rtp.Selection.empty(B * R * G, N, dev)
+        self.ws_sel = rtp.workspace(rtp.topp_select_workspace_size(B, R * G, 1, R, N), dev)
+        self.ws_ret = rtp.workspace(rtp.sparse_attn_decode_workspace_size(B, R * G, R, N), dev) if R else None
+        self.ws_loc = (rtp.workspace(rtp.window_attn_workspace_size(B, Hq - R * G, 1, Hkv - R, N, W), dev)
+                       if Hkv > R else None)
+
+    def build_index(self, stream=None) -> None:
+        """Project every cached key of the retrieval heads (done once, before decoding)."""
+        if self.R:
+            rtp.index_project(self.k_ret, self.P, self.k_idx, stream)
+
+    def step(self, stream=None) -> torch.Tensor:
+        """One decode step over the resident cache; returns o [B, Hq, 1, D]."""
+        if self.R:
+            if self.lens_host is None:
+                n = self.N
+                rtp.index_project(self.k_ret[:, :, n - 1: n], self.P, self.k_idx[:, :, n - 1: n], stream)
+            else:
+                for b, n in enumerate(self.lens_host):
+                    if n > 0:
+                        rtp.index_project(self.k_ret[b: b + 1, :, n - 1: n], self.P,
+                                          self.k_idx[b: b + 1, :, n - 1: n], stream)
+            rtp.index_project(self.q_ret, self.P, self.q_idx, stream)
+            rtp.topp_select(self.q_idx, self.k_idx, self.lens, self.p, self.sel, self.ws_sel, stream)
+            rtp.sparse_attn_decode(self.q_ret, self.k_ret, self.v_ret, self.lens, self.sel, self.scale,
+                                   self.o_ret, self.ws_ret, stream)
+        if self.Hkv > self.R:
+            rtp.window_attn(self.q_loc, self.k_loc, self.v_loc, self.lens, self.W, self.scale, self.o_loc,
+                            self.ws_loc, stream)
+        return self.o

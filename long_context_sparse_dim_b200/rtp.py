@@ -1,0 +1,227 @@
+"""ctypes binding of librtp.so (include/rtp.h): argument marshalling only.
+
+Every function here has the C name without the ``rtp_`` prefix, takes torch
+tensors that already live on the GPU, turns them into ``rtp_tensor``
+descriptors and calls the library on the current torch stream (or the given
+one).  A non-OK status raises :class:`RtpError`.  There is no fallback: if
+the shared library is missing, importing this module raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "librtp.so")
+
+RTP_OK = 0
+RTP_F32, RTP_BF16 = 0, 1
+STATUS_NAMES = {0: "RTP_OK", 1: "RTP_ERR_INVALID_ARG", 2: "RTP_ERR_SHAPE", 3: "RTP_ERR_DTYPE",
+                4: "RTP_ERR_ALIGNMENT", 5: "RTP_ERR_WORKSPACE", 6: "RTP_ERR_CUDA", 7: "RTP_ERR_UNSUPPORTED"}
+
+EXPORTED = ("rtp_index_project", "rtp_topp_select", "rtp_topp_select_workspace_size",
+            "rtp_sparse_attn_decode", "rtp_sparse_attn_decode_workspace_size",
+            "rtp_sparse_attn_prefill", "rtp_sparse_attn_prefill_workspace_size",
+            "rtp_window_attn", "rtp_window_attn_workspace_size",
+            "rtp_status_string", "rtp_last_cuda_error", "rtp_version")
+
+
+class RtpTensor(ctypes.Structure):
+    _fields_ = [("data", ctypes.c_void_p), ("dtype", ctypes.c_int32), ("ndim", ctypes.c_int32),
+                ("shape", ctypes.c_int64 * 4), ("stride", ctypes.c_int64 * 4)]
+
+
+class RtpSelection(ctypes.Structure):
+    _fields_ = [("tau_bits", ctypes.c_void_p), ("tiepos", ctypes.c_void_p), ("count", ctypes.c_void_p),
+                ("mask", ctypes.c_void_p), ("mask_words", ctypes.c_int64)]
+
+
+class RtpError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = f"{where}: {STATUS_NAMES.get(status, status)} ({_lib.rtp_status_string(status).decode()})"
+        if status == 6:
+            msg += f", cudaError {_lib.rtp_last_cuda_error()}"
+        super().__init__(msg)
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is not built; run python -m long_context_sparse_dim_b200.build")
+    lib = ctypes.CDLL(LIB_PATH)
+    P = ctypes.POINTER
+    T, S = P(RtpTensor), P(RtpSelection)
+    vp, i32, i64, f32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+    sig = {
+        "rtp_index_project": ([T, T, T, vp], i32),
+        "rtp_topp_select": ([T, T, vp, f32, S, vp, sz, vp], i32),
+        "rtp_topp_select_workspace_size": ([i64, i64, i64, i64, i64], sz),
+        "rtp_sparse_attn_decode": ([T, T, T, vp, S, f32, T, vp, sz, vp], i32),
+        "rtp_sparse_attn_decode_workspace_size": ([i64, i64, i64, i64], sz),
+        "rtp_sparse_attn_prefill": ([T, T, T, T, T, vp, S, f32, T, vp, sz, vp], i32),
+        "rtp_sparse_attn_prefill_workspace_size": ([i64, i64, i64, i64, i64], sz),
+        "rtp_window_attn": ([T, T, T, vp, i32, f32, T, vp, sz, vp], i32),
+        "rtp_window_attn_workspace_size": ([i64, i64, i64, i64, i64, i32], sz),
+        "rtp_status_string": ([i32], ctypes.c_char_p),
+        "rtp_last_cuda_error": ([], i32),
+        "rtp_version": ([], i32),
+    }
+    for name, (args, res) in sig.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = res
+    return lib
+
+
+_lib = _load()
+
+
+def lib() -> ctypes.CDLL:
+    return _lib
+
+
+# --------------------------------------------------------------------------
+# marshalling
+# --------------------------------------------------------------------------
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return RTP_F32
+    if t.dtype == torch.bfloat16:
+        return RTP_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def tensor_desc(t: torch.Tensor, ndim: int = 4) -> RtpTensor:
+    if t.dim() != ndim:
+        raise ValueError(f"expected a {ndim}-D tensor, got {tuple(t.shape)}")
+    d = RtpTensor()
+    d.data = t.data_ptr()
+    d.dtype = _dt(t)
+    d.ndim = ndim
+    for i in range(ndim):
+        d.shape[i] = t.shape[i]
+        d.stride[i] = t.stride(i)
+    return d
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _check(status: int, where: str):
+    if status != RTP_OK:
+        raise RtpError(status, where)
+
+
+@dataclass
+class Selection:
+    """Device arrays of rtp_selection for ``rows`` queries and ``N`` keys."""
+
+    tau_bits: torch.Tensor
+    tiepos: torch.Tensor
+    count: torch.Tensor
+    mask: Optional[torch.Tensor]
+
+    @staticmethod
+    def empty(rows: int, N: int, device, with_mask: bool = True) -> "Selection":
+        words = max((N + 31) // 32, 1)
+        return Selection(
+            tau_bits=torch.empty(rows, dtype=torch.int32, device=device),
+            tiepos=torch.empty(rows, dtype=torch.int32, device=device),
+            count=torch.empty(rows, dtype=torch.int32, device=device),
+            mask=torch.empty(rows, words, dtype=torch.int32, device=device) if with_mask else None)
+
+    def desc(self) -> RtpSelection:
+        s = RtpSelection()
+        s.tau_bits = self.tau_bits.data_ptr()
+        s.tiepos = self.tiepos.data_ptr()
+        s.count = self.count.data_ptr()
+        s.mask = self.mask.data_ptr() if self.mask is not None else None
+        s.mask_words = self.mask.shape[1] if self.mask is not None else 0
+        return s
+
+
+def workspace(nbytes: int, device) -> Optional[torch.Tensor]:
+    """A zero-filled workspace (256-byte aligned by the caching allocator)."""
+    if nbytes == 0:
+        return None
+    return torch.zeros(nbytes, dtype=torch.uint8, device=device)
+
+
+def _ws(ws: Optional[torch.Tensor]):
+    return (None, 0) if ws is None else (ctypes.c_void_p(ws.data_ptr()), ws.numel() * ws.element_size())
+
+
+# --------------------------------------------------------------------------
+# the five calls
+# --------------------------------------------------------------------------
+
+def index_project(x: torch.Tensor, P: torch.Tensor, x_idx: torch.Tensor, stream=None) -> None:
+    _check(_lib.rtp_index_project(ctypes.byref(tensor_desc(x)), ctypes.byref(tensor_desc(P, 3)),
+                                  ctypes.byref(tensor_desc(x_idx)), _stream(stream)), "rtp_index_project")
+
+
+def topp_select_workspace_size(B, Hq, T, Hk, N) -> int:
+    return int(_lib.rtp_topp_select_workspace_size(B, Hq, T, Hk, N))
+
+
+def topp_select(q_idx: torch.Tensor, k_idx: torch.Tensor, lens: Optional[torch.Tensor], p: float,
+                sel: Selection, ws: Optional[torch.Tensor] = None, stream=None) -> None:
+    w, nb = _ws(ws)
+    _check(_lib.rtp_topp_select(ctypes.byref(tensor_desc(q_idx)), ctypes.byref(tensor_desc(k_idx)),
+                                _ptr(lens), float(p), ctypes.byref(sel.desc()), w, nb, _stream(stream)),
+           "rtp_topp_select")
+
+
+def sparse_attn_decode_workspace_size(B, Hq, Hk, N) -> int:
+    return int(_lib.rtp_sparse_attn_decode_workspace_size(B, Hq, Hk, N))
+
+
+def sparse_attn_decode(q, k, v, lens, sel: Selection, scale: float, o, ws=None, stream=None) -> None:
+    w, nb = _ws(ws)
+    _check(_lib.rtp_sparse_attn_decode(ctypes.byref(tensor_desc(q)), ctypes.byref(tensor_desc(k)),
+                                       ctypes.byref(tensor_desc(v)), _ptr(lens), ctypes.byref(sel.desc()),
+                                       float(scale), ctypes.byref(tensor_desc(o)), w, nb, _stream(stream)),
+           "rtp_sparse_attn_decode")
+
+
+def sparse_attn_prefill_workspace_size(B, Hq, T, Hk, N) -> int:
+    return int(_lib.rtp_sparse_attn_prefill_workspace_size(B, Hq, T, Hk, N))
+
+
+def sparse_attn_prefill(q, k, v, q_idx, k_idx, lens, sel: Selection, scale: float, o, ws=None,
+                        stream=None) -> None:
+    w, nb = _ws(ws)
+    _check(_lib.rtp_sparse_attn_prefill(ctypes.byref(tensor_desc(q)), ctypes.byref(tensor_desc(k)),
+                                        ctypes.byref(tensor_desc(v)), ctypes.byref(tensor_desc(q_idx)),
+                                        ctypes.byref(tensor_desc(k_idx)), _ptr(lens), ctypes.byref(sel.desc()),
+                                        float(scale), ctypes.byref(tensor_desc(o)), w, nb, _stream(stream)),
+           "rtp_sparse_attn_prefill")
+
+
+def window_attn_workspace_size(B, Hq, T, Hk, N, W) -> int:
+    return int(_lib.rtp_window_attn_workspace_size(B, Hq, T, Hk, N, W))
+
+
+def window_attn(q, k, v, lens, W: int, scale: float, o, ws=None, stream=None) -> None:
+    w, nb = _ws(ws)
+    _check(_lib.rtp_window_attn(ctypes.byref(tensor_desc(q)), ctypes.byref(tensor_desc(k)),
+                                ctypes.byref(tensor_desc(v)), _ptr(lens), int(W), float(scale),
+                                ctypes.byref(tensor_desc(o)), w, nb, _stream(stream)), "rtp_window_attn")
+
+
+def version() -> int:
+    return int(_lib.rtp_version())

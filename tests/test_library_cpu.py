@@ -1,0 +1,162 @@
+"""librtp.so without a GPU: it loads, exports every declared symbol, and its
+host-side validation rejects bad arguments before touching the device.
+
+Every call below is built to FAIL validation (the pointers are fake), so
+nothing here ever reaches a CUDA call.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _lib():
+    from long_context_sparse_dim_b200 import build
+    if not os.path.exists(build.LIB):
+        build.build()
+    from long_context_sparse_dim_b200 import rtp
+    return rtp
+
+
+def _declared():
+    with open(os.path.join(ROOT, "include", "rtp.h")) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"RTP_API\s+[\w\s\*]+?\b(rtp_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_five_calls():
+    names = _declared()
+    for n in ("rtp_index_project", "rtp_topp_select", "rtp_sparse_attn_decode", "rtp_sparse_attn_prefill",
+              "rtp_window_attn"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    rtp = _lib()
+    lib = rtp.lib()
+    for name in _declared():
+        assert hasattr(lib, name), name
+    assert set(_declared()) == set(rtp.EXPORTED)
+    assert rtp.version() >= 100
+
+
+def test_exports_only_the_c_abi():
+    from long_context_sparse_dim_b200 import build
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", build.LIB], capture_output=True, text=True).stdout
+    syms = {ln.split()[-1] for ln in out.splitlines() if " T " in ln}
+    ours = {s for s in syms if s.startswith("rtp_")}
+    assert ours == set(_declared())
+
+
+def _desc(rtp, shape, dtype=1, data=0x10000, strides=None):
+    d = rtp.RtpTensor()
+    d.data = data
+    d.dtype = dtype
+    d.ndim = len(shape)
+    if strides is None:
+        strides, acc = [], 1
+        for s in reversed(shape):
+            strides.insert(0, acc)
+            acc *= s
+    for i, s in enumerate(shape):
+        d.shape[i] = s
+        d.stride[i] = strides[i]
+    return d
+
+
+def test_status_strings():
+    rtp = _lib()
+    for s in range(0, 8):
+        assert rtp.lib().rtp_status_string(s)
+    assert rtp.lib().rtp_status_string(99) == b"unknown status"
+
+
+def test_index_project_validation():
+    rtp = _lib()
+    L = rtp.lib()
+    by = ctypes.byref
+    x = _desc(rtp, [2, 2, 64, 128])
+    P = _desc(rtp, [2, 16, 128], dtype=0)
+    xi = _desc(rtp, [2, 2, 64, 16])
+    assert L.rtp_index_project(None, by(P), by(xi), None) == 1
+    assert L.rtp_index_project(by(_desc(rtp, [2, 2, 64, 128], data=0)), by(P), by(xi), None) == 1
+    assert L.rtp_index_project(by(_desc(rtp, [2, 2, 64, 64])), by(P), by(xi), None) == 2          # D != 128
+    assert L.rtp_index_project(by(x), by(P), by(_desc(rtp, [2, 2, 64, 8])), None) == 2          # d != 16
+    assert L.rtp_index_project(by(x), by(P), by(_desc(rtp, [2, 2, 63, 16])), None) == 2         # N mismatch
+    assert L.rtp_index_project(by(x), by(_desc(rtp, [3, 16, 128], dtype=0)), by(xi), None) == 2  # H % HP
+    assert L.rtp_index_project(by(x), by(_desc(rtp, [2, 16, 128], dtype=1)), by(xi), None) == 3  # P not f32
+    assert L.rtp_index_project(by(_desc(rtp, [2, 2, 64, 128], dtype=7)), by(P), by(xi), None) == 3
+    assert L.rtp_index_project(by(_desc(rtp, [2, 2, 64, 128], data=0x10008)), by(P), by(xi), None) == 4
+    bad_stride = _desc(rtp, [2, 2, 64, 128], strides=[2 * 64 * 130, 64 * 130, 130, 1])  # 260 B rows
+    assert L.rtp_index_project(by(bad_stride), by(P), by(xi), None) == 4
+    non_contig = _desc(rtp, [2, 2, 64, 128], strides=[2 * 64 * 256, 64 * 256, 256, 2])
+    assert L.rtp_index_project(by(non_contig), by(P), by(xi), None) == 4
+
+
+def _sel(rtp, mask=True, words=2):
+    s = rtp.RtpSelection()
+    s.tau_bits = 0x20000
+    s.tiepos = 0x30000
+    s.count = 0x40000
+    s.mask = 0x50000 if mask else None
+    s.mask_words = words
+    return s
+
+
+def test_topp_select_validation():
+    rtp = _lib()
+    L = rtp.lib()
+    by = ctypes.byref
+    qi = _desc(rtp, [2, 8, 1, 16])
+    ki = _desc(rtp, [2, 2, 64, 16])
+    s = _sel(rtp)
+    assert L.rtp_topp_select(by(qi), by(ki), None, 0.0, by(s), None, 0, None) == 1      # p <= 0
+    assert L.rtp_topp_select(by(qi), by(ki), None, -1.0, by(s), None, 0, None) == 1
+    assert L.rtp_topp_select(by(qi), by(ki), None, float("nan"), by(s), None, 0, None) == 1
+    assert L.rtp_topp_select(by(qi), by(ki), None, 0.9, None, None, 0, None) == 1
+    assert L.rtp_topp_select(by(qi), by(ki), None, 0.9, by(_sel(rtp, words=1)), None, 0, None) == 2
+    assert L.rtp_topp_select(by(_desc(rtp, [2, 7, 1, 16])), by(ki), None, 0.9, by(s), None, 0, None) == 2
+    assert L.rtp_topp_select(by(_desc(rtp, [3, 8, 1, 16])), by(ki), None, 0.9, by(s), None, 0, None) == 2
+    assert L.rtp_topp_select(by(_desc(rtp, [2, 8, 1, 16], dtype=0)), by(ki), None, 0.9, by(s), None, 0,
+                             None) == 3
+
+
+def test_attention_validation():
+    rtp = _lib()
+    L = rtp.lib()
+    by = ctypes.byref
+    q = _desc(rtp, [2, 8, 1, 128])
+    k = _desc(rtp, [2, 2, 64, 128])
+    o = _desc(rtp, [2, 8, 1, 128], dtype=0)
+    s = _sel(rtp)
+    # no workspace
+    assert L.rtp_sparse_attn_decode(by(q), by(k), by(k), None, by(s), 0.088, by(o), None, 0, None) == 5
+    assert L.rtp_sparse_attn_decode(by(q), by(k), by(k), None, by(s), 0.088, by(o), 0x100000, 16, None) == 5
+    assert L.rtp_sparse_attn_decode(by(q), by(k), by(k), None, by(s), 0.088, by(o), 0x100010, 1 << 30, None) == 4
+    assert L.rtp_sparse_attn_decode(by(q), by(k), by(k), None, by(_sel(rtp, mask=False)), 0.088, by(o), None, 0,
+                                    None) == 1
+    assert L.rtp_sparse_attn_decode(by(q), by(k), by(k), None, by(s), float("inf"), by(o), None, 0, None) == 1
+    assert L.rtp_sparse_attn_decode(by(_desc(rtp, [2, 18, 1, 128])), by(_desc(rtp, [2, 2, 64, 128])),
+                                    by(_desc(rtp, [2, 2, 64, 128])), None, by(s), 0.088,
+                                    by(_desc(rtp, [2, 18, 1, 128], dtype=0)), None, 0, None) == 2   # G = 9 > 8
+    assert L.rtp_sparse_attn_decode(by(q), by(k), by(_desc(rtp, [2, 2, 65, 128])), None, by(s), 0.088, by(o),
+                                    None, 0, None) == 2
+    assert L.rtp_sparse_attn_decode(by(q), by(k), by(_desc(rtp, [2, 2, 64, 128], dtype=0)), None, by(s), 0.088,
+                                    by(o), None, 0, None) == 3
+    assert L.rtp_window_attn(by(q), by(k), by(k), None, 0, 0.088, by(o), None, 0, None) == 1       # W < 1
+    assert L.rtp_window_attn(by(q), by(k), by(k), None, 16, 0.088, by(o), None, 0, None) == 5
+    assert L.rtp_window_attn(by(q), by(k), by(k), None, 16, 0.088, by(_desc(rtp, [2, 8, 2, 128], dtype=0)),
+                             None, 0, None) == 2
+
+
+def test_workspace_sizes_are_monotone():
+    rtp = _lib()
+    a = rtp.sparse_attn_decode_workspace_size(8, 8, 2, 32768)
+    b = rtp.sparse_attn_decode_workspace_size(8, 8, 2, 131072)
+    assert 0 < a <= b
+    assert rtp.window_attn_workspace_size(8, 24, 1, 6, 32768, 4096) > 0
+    assert rtp.topp_select_workspace_size(8, 8, 1, 2, 32768) == 0
