@@ -38,6 +38,8 @@ constexpr int kStages = 3;
 constexpr int kRowBytes = kHeadDim * 2;  // 256 B per bf16 row
 constexpr int kTileBytes = kTileKeys * kRowBytes;
 constexpr int kMaxGroup = 8;
+constexpr int kMaxChunk = 8192;                 // keys per CTA at most
+constexpr int kMaxChunkWords = kMaxChunk / 32;  // mask words per head per CTA
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct AttnArgs {
@@ -115,9 +117,12 @@ RTP_DEVICE KeyRange key_range(const AttnArgs& A, int b, int split) {
 }
 
 // ---- split partial write + last-CTA merge (shared by both variants) --------
-// part_o[h][d] (unnormalised), part_m[h] (log2 domain), part_l[h] are in smem.
+// part_o[h][d] (unnormalised), part_m[h] (log2 domain), part_l[h] are in smem;
+// `scratch` holds at least 2 * kMaxSplits * kMaxGroup + 2 * kMaxGroup floats.
+constexpr int kMaxSplits = 64;
+
 __device__ void finish_split(const AttnArgs& A, int grp, int split, const float* part_o,
-                             const float* part_m, const float* part_l, int* flag_smem) {
+                             const float* part_m, const float* part_l, int* flag_smem, float* scratch) {
   const int tid = threadIdx.x;
   const int G = A.G;
   float* wo = A.ws_o + ((int64_t)grp * A.splits + split) * kMaxGroup * kHeadDim;
@@ -136,23 +141,52 @@ __device__ void finish_split(const AttnArgs& A, int grp, int split, const float*
   __syncthreads();
   if (!*flag_smem) return;
   __threadfence();
+  const int S = A.splits;
   const int b = grp / A.Hk, kvh = grp % A.Hk;
-  const float* go = A.ws_o + (int64_t)grp * A.splits * kMaxGroup * kHeadDim;
-  const float* gml = A.ws_ml + (int64_t)grp * A.splits * kMaxGroup * 2;
+  const float* go = A.ws_o + (int64_t)grp * S * kMaxGroup * kHeadDim;
+  const float* gml = A.ws_ml + (int64_t)grp * S * kMaxGroup * 2;
+  float* fm = scratch;                       // [S][G]: split max, then its weight
+  float* fl = scratch + kMaxSplits * kMaxGroup;  // [S][G]: split sum
+  float* Mh = fl + kMaxSplits * kMaxGroup;   // [G]
+  float* Lh = Mh + kMaxGroup;                // [G]
+  for (int i = tid; i < S * G; i += blockDim.x) {
+    const int s = i / G, h = i % G;
+    fm[i] = __ldcg(gml + (s * kMaxGroup + h) * 2);
+    fl[i] = __ldcg(gml + (s * kMaxGroup + h) * 2 + 1);
+  }
+  __syncthreads();
+  if (tid < G) {
+    float M = -INFINITY;
+    for (int s = 0; s < S; ++s) M = fmaxf(M, fm[s * G + tid]);
+    float L = 0.f;
+    if (M != -INFINITY)
+      for (int s = 0; s < S; ++s) {
+        const float ms = fm[s * G + tid];
+        if (ms != -INFINITY) L += ex2(ms - M) * fl[s * G + tid];
+      }
+    Mh[tid] = M;
+    Lh[tid] = L;
+  }
+  __syncthreads();
+  for (int i = tid; i < S * G; i += blockDim.x) {
+    const float ms = fm[i], M = Mh[i % G];
+    fm[i] = (ms == -INFINITY || M == -INFINITY) ? 0.f : ex2(ms - M);
+  }
+  __syncthreads();
   for (int i = tid; i < G * kHeadDim; i += blockDim.x) {
     const int h = i / kHeadDim, d = i % kHeadDim;
-    float M = -INFINITY;
-    for (int s = 0; s < A.splits; ++s) M = fmaxf(M, __ldcg(gml + (s * kMaxGroup + h) * 2));
-    float num = 0.f, den = 0.f;
-    if (M != -INFINITY) {
-      for (int s = 0; s < A.splits; ++s) {
-        const float ms = __ldcg(gml + (s * kMaxGroup + h) * 2);
-        if (ms == -INFINITY) continue;
-        const float f = ex2(ms - M);
-        num += f * __ldcg(go + (s * kMaxGroup + h) * kHeadDim + d);
-        den += f * __ldcg(gml + (s * kMaxGroup + h) * 2 + 1);
-      }
+    const float* src = go + h * kHeadDim + d;
+    float num = 0.f;
+    int s = 0;
+    for (; s + 8 <= S; s += 8) {
+      float v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = __ldcg(src + (int64_t)(s + u) * kMaxGroup * kHeadDim);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) num += fm[(s + u) * G + h] * v[u];
     }
+    for (; s < S; ++s) num += fm[s * G + h] * __ldcg(src + (int64_t)s * kMaxGroup * kHeadDim);
+    const float den = Lh[h];
     const float val = den > 0.f ? num / den : 0.f;
     const int hq = kvh * G + h;
     if (A.o_bf16) {
@@ -201,19 +235,34 @@ attn_decode_bf16_kernel(AttnArgs A) {
   auto stageK = [&](int st) { return sbase + st * 2 * kTileBytes; };
   auto stageV = [&](int st) { return sbase + st * 2 * kTileBytes + kTileBytes; };
 
+  // Sparse mode: the chunk's mask words (per head, and their union over the
+  // group) are staged once; R.c0 is a multiple of 64 there.
+  uint32_t* umask = reinterpret_cast<uint32_t*>(smem + kStages * 2 * kTileBytes);
+  uint32_t* hmask = umask + kMaxChunkWords;  // [G][kMaxChunkWords]
+  const int nw = (R.c1 - R.c0 + 31) >> 5;
+  if (sparse) {
+    const int w0 = R.c0 >> 5;
+    for (int i = tid; i < nw; i += kAttnThreads) {
+      uint32_t u = 0;
+      for (int hh = 0; hh < G; ++hh) {
+        const uint32_t x = __ldg(mrow0 + (int64_t)hh * A.mask_words + w0 + i);
+        hmask[hh * kMaxChunkWords + i] = x;
+        u |= x;
+      }
+      umask[i] = u;
+    }
+    __syncthreads();
+  }
+
   // Load tile t into stage st: 64 rows x 16 chunks for K and for V, 8 + 8 per thread.
   auto load_tile = [&](int t, int st) {
     const int tb = R.c0 + t * kTileKeys;
     uint64_t uni = ~0ull;
     if (sparse) {
-      uni = 0ull;
-      const int w0 = tb >> 5;  // tb is a multiple of 64 in sparse mode
-      for (int hh = 0; hh < G; ++hh) {
-        const uint32_t* mr = mrow0 + (int64_t)hh * A.mask_words;
-        const uint32_t lo = __ldg(mr + w0);
-        const uint32_t hi = (tb + 32 < A.N) ? __ldg(mr + w0 + 1) : 0u;
-        uni |= (uint64_t)lo | ((uint64_t)hi << 32);
-      }
+      const int wl = (tb - R.c0) >> 5;
+      const uint32_t lo = umask[wl];
+      const uint32_t hi = (wl + 1 < nw) ? umask[wl + 1] : 0u;
+      uni = (uint64_t)lo | ((uint64_t)hi << 32);
     }
     const int ch = tid & 15;
 #pragma unroll
@@ -253,10 +302,10 @@ attn_decode_bf16_kernel(AttnArgs A) {
       const int kg0 = kw + g, kg1 = kw + g + 8;
       const bool v0 = kg0 < R.c1, v1 = kg1 < R.c1;
       if (sparse) {
-        const int wi = kw >> 5, sh = (kw & 31) + g;
-        const bool wv = kw < R.c1;  // the word exists (kw < N)
-        const uint32_t w0 = (wv && h0 < G) ? __ldg(mrow0 + (int64_t)h0 * A.mask_words + wi) : 0u;
-        const uint32_t w1 = (wv && h1 < G) ? __ldg(mrow0 + (int64_t)h1 * A.mask_words + wi) : 0u;
+        const int wi = (kw - R.c0) >> 5, sh = (kw & 31) + g;
+        const bool wv = kw < R.c1;  // the word is inside the chunk
+        const uint32_t w0 = (wv && h0 < G) ? hmask[h0 * kMaxChunkWords + wi] : 0u;
+        const uint32_t w1 = (wv && h1 < G) ? hmask[h1 * kMaxChunkWords + wi] : 0u;
         a00 = v0 && ((w0 >> sh) & 1u);
         a01 = v0 && ((w1 >> sh) & 1u);
         a10 = v1 && ((w0 >> (sh + 8)) & 1u);
@@ -340,6 +389,7 @@ attn_decode_bf16_kernel(AttnArgs A) {
   float* part_m = part_o + kMaxGroup * kHeadDim;              // [8]
   float* part_l = part_m + kMaxGroup;                         // [8]
   int* flag = reinterpret_cast<int*>(part_l + kMaxGroup);
+  float* scratch = reinterpret_cast<float*>(flag + 4);
 #pragma unroll
   for (int o = 4; o < 32; o <<= 1) {
     l0 += __shfl_xor_sync(0xffffffffu, l0, o);
@@ -381,7 +431,7 @@ attn_decode_bf16_kernel(AttnArgs A) {
     }
   }
   __syncthreads();
-  finish_split(A, grp, split, part_o, part_m, part_l, flag);
+  finish_split(A, grp, split, part_o, part_m, part_l, flag, scratch);
 }
 
 // ---- fp32 CUDA-core variant -----------------------------------------------
@@ -392,6 +442,7 @@ attn_decode_f32_kernel(AttnArgs A) {
   __shared__ __align__(16) float part_o[kMaxGroup * kHeadDim];
   __shared__ float part_m[kMaxGroup], part_l[kMaxGroup];
   __shared__ int flag;
+  __shared__ float scratch[2 * kMaxSplits * kMaxGroup + 2 * kMaxGroup];
   const int split = blockIdx.x, grp = blockIdx.y;
   const int b = grp / A.Hk, kvh = grp % A.Hk;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -474,25 +525,29 @@ attn_decode_f32_kernel(AttnArgs A) {
     }
   }
   __syncthreads();
-  finish_split(A, grp, split, part_o, part_m, part_l, &flag);
+  finish_split(A, grp, split, part_o, part_m, part_l, &flag, scratch);
 }
 
 // ---- host side ---------------------------------------------------------------
-static int attn_chunk(int64_t groups, int64_t range, int sms) {
-  // enough CTAs for ~4 per SM, chunks a multiple of the tile, at least 256 keys
-  const int64_t want_splits = (4 * (int64_t)sms + groups - 1) / (groups > 0 ? groups : 1);
-  int64_t chunk = (range + want_splits - 1) / (want_splits > 0 ? want_splits : 1);
-  chunk = (chunk + kTileKeys - 1) / kTileKeys * kTileKeys;
-  if (chunk < 256) chunk = 256;
-  if (chunk > 8192) chunk = 8192;
-  return (int)chunk;
-}
-
+// One wave: about two CTAs per SM over all (sequence, KV head) groups; chunks a
+// multiple of the tile, between 256 and kMaxChunk keys, at most kMaxSplits.
 static void attn_layout(int64_t B, int64_t Hk, int64_t N, int32_t W, int sms, int* chunk, int* splits) {
-  const int64_t range = W > 0 ? (W < N ? W : N) : N;
-  *chunk = attn_chunk(B * Hk, range > 0 ? range : 1, sms);
-  *splits = (int)((range + *chunk - 1) / *chunk);
-  if (*splits < 1) *splits = 1;
+  int64_t range = W > 0 ? (W < N ? W : N) : N;
+  if (range < 1) range = 1;
+  const int64_t groups = B * Hk > 0 ? B * Hk : 1;
+  int64_t want = (2 * (int64_t)sms) / groups;
+  if (want < 1) want = 1;
+  int64_t c = (range + want - 1) / want;
+  c = (c + kTileKeys - 1) / kTileKeys * kTileKeys;
+  if (c < 256) c = 256;
+  if (c > kMaxChunk) c = kMaxChunk;
+  int64_t s = (range + c - 1) / c;
+  while (s > kMaxSplits) {  // very long ranges: grow the chunk beyond the one-wave target
+    c *= 2;
+    s = (range + c - 1) / c;
+  }
+  *chunk = (int)c;
+  *splits = (int)s;
 }
 
 size_t attn_decode_workspace_bytes(int64_t B, int64_t Hq, int64_t Hk, int64_t N, int32_t W) {
@@ -507,11 +562,18 @@ size_t attn_decode_workspace_bytes(int64_t B, int64_t Hq, int64_t Hk, int64_t N,
   return ((o_bytes + 255) / 256 * 256) + ((ml_bytes + 255) / 256 * 256) + ((t_bytes + 255) / 256 * 256);
 }
 
+bool attn_decode_supported(int64_t B, int64_t Hk, int64_t N, int32_t W) {
+  int chunk = 0, splits = 0;
+  attn_layout(B, Hk, N, W, 148, &chunk, &splits);
+  return W > 0 || chunk <= kMaxChunk;  // the sparse form stages a chunk's masks on chip
+}
+
 cudaError_t launch_attn_decode(const LaunchAttnDecode& a, cudaStream_t stream) {
   const int64_t groups = a.B * a.Hk;
   if (groups == 0) return cudaSuccess;
   int chunk = 0, splits = 0;
   attn_layout(a.B, a.Hk, a.N, a.W, 148, &chunk, &splits);
+  if (a.W <= 0 && chunk > kMaxChunk) return cudaErrorInvalidValue;
   AttnArgs A;
   A.q = a.q;
   A.k = a.k;
@@ -537,7 +599,7 @@ cudaError_t launch_attn_decode(const LaunchAttnDecode& a, cudaStream_t stream) {
   A.tickets = reinterpret_cast<uint32_t*>(ws + (o_bytes + 255) / 256 * 256 + (ml_bytes + 255) / 256 * 256);
   dim3 grid((unsigned)splits, (unsigned)groups);
   if (a.bf16) {
-    const size_t smem = (size_t)kStages * 2 * kTileBytes;
+    const size_t smem = (size_t)kStages * 2 * kTileBytes + (size_t)(kMaxGroup + 1) * kMaxChunkWords * 4;
     cudaFuncSetAttribute(attn_decode_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     attn_decode_bf16_kernel<<<grid, kAttnThreads, smem, stream>>>(A);
   } else {

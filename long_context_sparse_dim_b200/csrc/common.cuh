@@ -84,6 +84,41 @@ RTP_DEVICE void load_idx_row<float>(const float* row, float (&k)[kIdxDim]) {
   }
 }
 
+// A projected-key row as raw 16-byte vectors (2 for bf16, 4 for fp32), so that
+// several rows can be in flight per thread before any conversion.
+template <typename T>
+struct IdxRaw {
+  static constexpr int kVec = sizeof(T) == 2 ? 2 : 4;
+  uint4 v[kVec];
+};
+
+template <typename T>
+RTP_DEVICE void load_idx_raw(const T* row, IdxRaw<T>& r) {
+  const uint4* p = reinterpret_cast<const uint4*>(row);
+#pragma unroll
+  for (int i = 0; i < IdxRaw<T>::kVec; ++i) r.v[i] = __ldg(p + i);
+}
+
+template <typename T>
+RTP_DEVICE void idx_raw_to_float(const IdxRaw<T>& r, float (&k)[kIdxDim]) {
+  if constexpr (sizeof(T) == 2) {
+    const uint32_t w[8] = {r.v[0].x, r.v[0].y, r.v[0].z, r.v[0].w, r.v[1].x, r.v[1].y, r.v[1].z, r.v[1].w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      k[2 * i] = bf16_lo(w[i]);
+      k[2 * i + 1] = bf16_hi(w[i]);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      k[4 * i] = __uint_as_float(r.v[i].x);
+      k[4 * i + 1] = __uint_as_float(r.v[i].y);
+      k[4 * i + 2] = __uint_as_float(r.v[i].z);
+      k[4 * i + 3] = __uint_as_float(r.v[i].w);
+    }
+  }
+}
+
 // Fixed-point top-p weight: round(exp(s - m) * 2^frac) as an unsigned 64-bit
 // integer.  With frac = 63 - ceil(log2 n) a sum over n keys cannot overflow,
 // and integer sums do not depend on the order of accumulation.

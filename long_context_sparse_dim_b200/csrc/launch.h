@@ -50,6 +50,7 @@ struct LaunchAttnDecode {
   bool o_bf16;
   void* ws;
 };
+bool attn_decode_supported(int64_t B, int64_t Hk, int64_t N, int32_t W);
 size_t attn_decode_workspace_bytes(int64_t B, int64_t Hq, int64_t Hk, int64_t N, int32_t W);
 cudaError_t launch_attn_decode(const LaunchAttnDecode& a, cudaStream_t stream);
 

@@ -191,6 +191,7 @@ rtp_status rtp_sparse_attn_decode(const rtp_tensor* q, const rtp_tensor* k, cons
   if (sel->mask_words < (N + 31) / 32) return RTP_ERR_SHAPE;
   const size_t need = rtp_sparse_attn_decode_workspace_size(q->shape[0], q->shape[1], k->shape[1], N);
   if ((s = check_workspace(workspace, workspace_bytes, need)) != RTP_OK) return s;
+  if (!rtp::attn_decode_supported(q->shape[0], k->shape[1], N, 0)) return RTP_ERR_UNSUPPORTED;
   rtp::LaunchAttnDecode a;
   a.q = view(q);
   a.k = view(k);

@@ -9,16 +9,21 @@
 // Design (B200): one thread-block CLUSTER per query.  Each CTA of the cluster
 // owns a contiguous slice of the keys, computes their scores once from the
 // projected-key cache (32-byte rows, 16-byte vector loads) and keeps them in
-// shared memory.  The cut is found without sorting by a three-digit radix
-// search on the order-preserving uint32 image of the fp32 scores (11 + 11 + 10
-// bits, most significant first).  Each digit pass builds a weighted histogram
-// (64-bit fixed-point mass + count) per CTA; the cluster reduces it through
-// distributed shared memory, each CTA summing one slice of the bins, and the
-// CTA holding the cut bin broadcasts it.  After the last digit the cut bin is
-// one score value tau; ties at tau are resolved by position with a prefix
-// count over the cluster.  Finally every CTA writes its bits of the selection
-// mask.  There are no global-memory atomics and no spin waits: all
-// synchronisation is the hardware cluster barrier.
+// shared memory.  The cut is found without sorting, by narrowing a bracket:
+//   pass 0   256 bins linear in (max - s) (1/16 nat wide; the last bin holds
+//            the tail) -- scores spread over many bins, so the per-warp
+//            shared-memory histograms see few same-bin collisions;
+//   pass 1.. 256 bins over the order-preserving uint32 image of the fp32
+//            score (8-bit digits of the offset inside the bracket), only for
+//            keys still inside the bracket, until the bracket is one score
+//            value tau.
+// Every pass accumulates 64-bit fixed-point masses (integer sums, so the
+// result does not depend on thread order).  After each pass every CTA reads
+// all CTAs' 256 bins through distributed shared memory and finds the same cut
+// bin by itself, so a pass costs one cluster barrier.  Ties at tau are
+// resolved by position with a prefix count over the cluster; then every CTA
+// writes its bits of the selection mask.  No global-memory atomics and no spin
+// waits: all synchronisation is the hardware cluster barrier.
 #include <cooperative_groups.h>
 
 #include <math.h>
@@ -32,39 +37,44 @@ namespace rtp {
 
 constexpr int kSelThreads = 256;
 constexpr int kSelWarps = kSelThreads / 32;
-constexpr int kBins = 2048;            // 11-bit digits; the last pass uses 1024 bins
+constexpr int kBins = 256;
 constexpr int kMaxCluster = 16;
 constexpr int kMaxKeysPerCta = 32768;  // scores of one CTA held in shared memory (128 KB)
-
-struct SelDecision {
-  uint64_t mass_above;  // mass of this pass's bins above the cut bin
-  uint64_t bin_mass;
-  uint32_t bin;         // cut bin (digit value)
-  uint32_t bin_cnt;
-  uint32_t cnt_above;
-  uint32_t pad;
-};
+constexpr float kLinBinsPerNat = 16.f; // pass 0 bin width 1/16 nat
+static_assert(kSelThreads == kBins, "one thread per histogram bin");
 
 struct SelSmem {
-  uint64_t hist_mass[kBins];
-  uint32_t hist_cnt[kBins];
-  uint64_t red_mass[kBins];
-  uint32_t red_cnt[kBins];
-  uint64_t slice_mass[kMaxCluster];
-  uint32_t slice_cnt[kMaxCluster];
-  uint32_t tcount[kMaxCluster];
-  SelDecision dec;
+  uint64_t whist[kSelWarps][kBins];  // per-warp private histograms
+  uint64_t hist[2][kBins];           // this CTA's histogram, double-buffered by pass parity
+  uint64_t red[kBins];               // cluster-wide histogram (each CTA holds a copy)
+  uint64_t wsum[kSelWarps];
+  uint32_t tcount[kMaxCluster];      // keys equal to tau, per CTA
+  uint32_t gcount[kMaxCluster];      // keys above tau, per CTA
   float cmax_self;
   float wmax[kSelWarps];
-  uint64_t wmass[kSelWarps];
   uint32_t wcnt[kSelWarps];
-  uint32_t wtot[kSelWarps];
+  uint32_t wcnt2[kSelWarps];
+  int cut_bin;
+  uint64_t cut_above;
 };
 
-RTP_DEVICE int ceil_log2(int64_t n) {
-  int r = 0;
-  while ((int64_t(1) << r) < n) ++r;
-  return r;
+RTP_DEVICE float ex2f_fast(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Fixed-point top-p weight round(2^((s - m) log2 e) * 2^frac).  Every use of a
+// weight in the cut goes through this one function.
+RTP_DEVICE uint64_t sel_weight(float s, float m, float two_pow_frac) {
+  const float e = ex2f_fast(__fmul_rn(__fsub_rn(s, m), 1.4426950408889634f));
+  return __float2ull_rn(__fmul_rn(e, two_pow_frac));
+}
+
+// pass-0 bin of a score: floor((m - s) * 16), the tail folded into the last bin
+RTP_DEVICE int lin_bin(float s, float m) {
+  const float t = __fmul_rn(__fsub_rn(m, s), kLinBinsPerNat);
+  return t >= (float)(kBins - 1) ? kBins - 1 : (int)t;
 }
 
 template <typename T>
@@ -115,182 +125,192 @@ topp_decode_kernel(View4 qv, View4 kv, const int32_t* __restrict__ lens, int Hq,
     return;
   }
 
-  // ---- scores of this CTA's keys -------------------------------------------
+  // ---- scores of this CTA's keys (eight independent row loads in flight per thread)
   float qf[kIdxDim];
   load_idx_row<T>(static_cast<const T*>(qv.data) + b * qv.sb + h * qv.sh, qf);
   const T* kb = static_cast<const T*>(kv.data) + b * kv.sb + kvh * kv.sh;
   float lmax = -INFINITY;
-  for (int i = tid; i < nloc; i += kSelThreads) {
-    float kf[kIdxDim];
-    load_idx_row<T>(kb + (int64_t)(c0 + i) * kv.sn, kf);
-    const float s = indexer_dot16(qf, kf);
-    scores[i] = s;
-    lmax = fmaxf(lmax, s);
+  constexpr int U = sizeof(T) == 2 ? 8 : 4;
+  for (int base = 0; base < nloc; base += U * kSelThreads) {
+    IdxRaw<T> raw[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int i = base + u * kSelThreads + tid;
+      if (i < nloc) load_idx_raw<T>(kb + (int64_t)(c0 + i) * kv.sn, raw[u]);
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int i = base + u * kSelThreads + tid;
+      if (i < nloc) {
+        float kf[kIdxDim];
+        idx_raw_to_float<T>(raw[u], kf);
+        const float sc = indexer_dot16(qf, kf);
+        scores[i] = sc;
+        lmax = fmaxf(lmax, sc);
+      }
+    }
   }
   lmax = warp_max(lmax);
   if (lane == 0) S.wmax[warp] = lmax;
   __syncthreads();
   if (tid == 0) {
-    float m = S.wmax[0];
-    for (int w = 1; w < kSelWarps; ++w) m = fmaxf(m, S.wmax[w]);
-    S.cmax_self = m;
+    float mm = S.wmax[0];
+    for (int w = 1; w < kSelWarps; ++w) mm = fmaxf(mm, S.wmax[w]);
+    S.cmax_self = mm;
   }
   cluster.sync();
   float m = -INFINITY;
-  for (int r = 0; r < C; ++r) m = fmaxf(m, *cluster.map_shared_rank(&S.cmax_self, r));
-
-  // ---- three radix passes ----------------------------------------------------
-  uint64_t target = 0, mass_above = 0;
-  uint32_t cnt_above = 0, prefix = 0, tau_cnt = 0;
-  for (int pass = 0; pass < 3; ++pass) {
-    const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
-    const int nb = pass == 2 ? 1024 : 2048;
-    const int pshift = pass == 1 ? 21 : 10;  // bits of the prefix fixed by earlier passes
-    for (int i = tid; i < nb; i += kSelThreads) {
-      S.hist_mass[i] = 0;
-      S.hist_cnt[i] = 0;
-    }
-    __syncthreads();
-    for (int i = tid; i < nloc; i += kSelThreads) {
-      const float s = scores[i];
-      const uint32_t k = score_key(s);
-      if (pass == 0 || (k >> pshift) == prefix) {
-        const uint32_t d = (k >> shift) & (uint32_t)(nb - 1);
-        atomicAdd(reinterpret_cast<unsigned long long*>(&S.hist_mass[d]),
-                  (unsigned long long)fixed_weight(s, m, two_pow_frac));
-        atomicAdd(&S.hist_cnt[d], 1u);
-      }
-    }
-    cluster.sync();  // (A) every CTA's histogram is complete
-
-    // Reduce the bins this CTA owns across the cluster.
-    const int sl = nb / C;
-    const int lo = rank * sl;
-    uint64_t tm = 0;
-    uint32_t tc = 0;
-    for (int i = tid; i < sl; i += kSelThreads) {
-      uint64_t am = 0;
-      uint32_t ac = 0;
-      for (int r = 0; r < C; ++r) {
-        am += cluster.map_shared_rank(S.hist_mass, r)[lo + i];
-        ac += cluster.map_shared_rank(S.hist_cnt, r)[lo + i];
-      }
-      S.red_mass[i] = am;
-      S.red_cnt[i] = ac;
-      tm += am;
-      tc += ac;
-    }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      tm += __shfl_xor_sync(0xffffffffu, tm, o);
-      tc += __shfl_xor_sync(0xffffffffu, tc, o);
-    }
-    if (lane == 0) {
-      S.wmass[warp] = tm;
-      S.wcnt[warp] = tc;
+  for (int r = 0; r < kMaxCluster; ++r)
+    if (r < C) m = fmaxf(m, *cluster.map_shared_rank(&S.cmax_self, r));
+
+  // ---- bracket narrowing --------------------------------------------------------
+  // pass 0: linear bins; then key-window bins [base, base + 256 << shift).
+  uint64_t target = 0, mass_above = 0;
+  int lin = -1;               // cut bin of pass 0
+  uint32_t kbase = 0;         // key window [kbase, kend) of the refinement passes
+  uint64_t kend = 0;
+  int shift = 0;
+  for (int pass = 0;; ++pass) {
+    uint64_t* wh = S.whist[warp];
+    for (int i = lane; i < kBins; i += 32) wh[i] = 0;
+    __syncwarp();
+    for (int i = tid; i < nloc; i += kSelThreads) {
+      const float sc = scores[i];
+      int d = -1;
+      if (pass == 0) {
+        d = lin_bin(sc, m);
+      } else if (lin_bin(sc, m) == lin) {
+        const uint32_t k = score_key(sc);
+        if (k >= kbase && (uint64_t)k < kend) d = (int)((uint64_t)(k - kbase) >> shift);
+      }
+      if (d >= 0) atomicAdd(reinterpret_cast<unsigned long long*>(&wh[d]),
+                            (unsigned long long)sel_weight(sc, m, two_pow_frac));
     }
     __syncthreads();
-    if (tid < C) {
-      uint64_t sm = 0;
-      uint32_t sc = 0;
-      for (int w = 0; w < kSelWarps; ++w) {
-        sm += S.wmass[w];
-        sc += S.wcnt[w];
-      }
-      cluster.map_shared_rank(S.slice_mass, tid)[rank] = sm;
-      cluster.map_shared_rank(S.slice_cnt, tid)[rank] = sc;
+    uint64_t* hb = S.hist[pass & 1];
+    {
+      uint64_t a = 0;
+#pragma unroll
+      for (int w = 0; w < kSelWarps; ++w) a += S.whist[w][tid];
+      hb[tid] = a;
     }
-    cluster.sync();  // (B) all slice totals are known everywhere
-
+    cluster.sync();  // every CTA's histogram of this pass is complete
+    // cluster-wide histogram, computed identically by every CTA
+    {
+      uint64_t a = 0;
+#pragma unroll
+      for (int r = 0; r < kMaxCluster; ++r)
+        if (r < C) a += cluster.map_shared_rank(hb, r)[tid];
+      S.red[tid] = a;
+    }
+    __syncthreads();
     if (pass == 0) {
+      // Z = total mass; target = ceil(p Z)
+      uint64_t a = S.red[tid];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+      if (lane == 0) S.wsum[warp] = a;
+      __syncthreads();
       uint64_t Z = 0;
-      for (int r = 0; r < C; ++r) Z += S.slice_mass[r];
-      double t = ceil((double)p * (double)Z);
-      uint64_t tt = t >= (double)Z ? Z : (uint64_t)t;
+      for (int w = 0; w < kSelWarps; ++w) Z += S.wsum[w];
+      const double t = ceil((double)p * (double)Z);
+      const uint64_t tt = t >= (double)Z ? Z : (uint64_t)t;
       target = tt < 1 ? 1 : tt;
+      __syncthreads();  // S.wsum is reused by the scan below
     }
     const uint64_t need = target - mass_above;  // >= 1
-    // The cut slice: walking slices from the highest scores down.
-    uint64_t cum = 0;
-    uint32_t cumc = 0;
-    int cut_r = 0;
-    for (int r = C - 1; r >= 0; --r) {
-      if (cum + S.slice_mass[r] >= need) {
-        cut_r = r;
-        break;
-      }
-      cum += S.slice_mass[r];
-      cumc += S.slice_cnt[r];
-    }
-    if (rank == cut_r && warp == 0) {
-      // lane l covers local bins [hi_l - per, hi_l), lane 0 the highest
-      const int per = (sl + 31) / 32;
-      const int hi_l = sl - lane * per;
-      const int lo_l = max(hi_l - per, 0);
-      uint64_t lm = 0;
-      uint32_t lc = 0;
-      for (int i = lo_l; i < hi_l; ++i) {
-        lm += S.red_mass[i];
-        lc += S.red_cnt[i];
-      }
-      uint64_t incl = lm;
-      uint32_t inclc = lc;
+    // Bins in descending score order: pass 0 bin 0 is the highest scores;
+    // refinement bin 255 is the highest key.  Position r in that order:
+    const int bin_of_r = pass == 0 ? tid : (kBins - 1 - tid);
+    const uint64_t mine = S.red[bin_of_r];
+    // inclusive prefix of the mass over the descending order (block scan)
+    uint64_t incl = mine;
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint64_t vm = __shfl_up_sync(0xffffffffu, incl, o);
-        const uint32_t vc = __shfl_up_sync(0xffffffffu, inclc, o);
-        if (lane >= o) {
-          incl += vm;
-          inclc += vc;
-        }
-      }
-      const uint64_t excl = incl - lm;
-      const uint32_t exclc = inclc - lc;
-      if (hi_l > lo_l && cum + excl < need && need <= cum + incl) {
-        uint64_t ma = cum + excl;
-        uint32_t ca = cumc + exclc;
-        int bin = lo_l;
-        for (int i = hi_l - 1; i >= lo_l; --i) {
-          if (ma + S.red_mass[i] >= need) {
-            bin = i;
-            break;
-          }
-          ma += S.red_mass[i];
-          ca += S.red_cnt[i];
-        }
-        SelDecision d;
-        d.mass_above = ma;
-        d.bin_mass = S.red_mass[bin];
-        d.bin = (uint32_t)(lo + bin);
-        d.bin_cnt = S.red_cnt[bin];
-        d.cnt_above = ca;
-        d.pad = 0;
-        for (int r = 0; r < C; ++r) *cluster.map_shared_rank(&S.dec, r) = d;
-      }
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint64_t v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
     }
-    cluster.sync();  // (C) the decision is everywhere
-    const SelDecision d = S.dec;
-    mass_above += d.mass_above;
-    cnt_above += d.cnt_above;
-    prefix = pass == 2 ? ((prefix << 10) | d.bin) : ((prefix << 11) | d.bin);
-    tau_cnt = d.bin_cnt;
+    if (lane == 31) S.wsum[warp] = incl;
+    __syncthreads();
+    uint64_t off = 0;
+    for (int w = 0; w < warp; ++w) off += S.wsum[w];
+    incl += off;
+    const uint64_t excl = incl - mine;
+    if (excl < need && need <= incl) {  // exactly one position holds the cut
+      S.cut_bin = bin_of_r;
+      S.cut_above = excl;
+    }
+    __syncthreads();
+    mass_above += S.cut_above;
+    const int cb = S.cut_bin;
+    __syncthreads();
+    if (pass == 0) {
+      lin = cb;
+      // key window holding every score of linear bin `lin` (with a margin)
+      const float hi_s = m - (float)lin / kLinBinsPerNat;
+      const float lo_s = m - (float)(lin + 1) / kLinBinsPerNat;
+      const float mg = 1e-5f * (fabsf(m) + (float)(lin + 1) / kLinBinsPerNat) + 1e-30f;
+      const uint32_t khi = score_key(__fadd_rn(hi_s + mg, 0.0f));
+      const uint32_t klo = lin == kBins - 1 ? 0u : score_key(__fadd_rn(lo_s - mg, 0.0f));
+      kbase = klo;
+      kend = (uint64_t)khi + 1;
+      const uint64_t range = kend - klo;
+      shift = 0;
+      while (((range - 1) >> shift) >= (uint64_t)kBins) ++shift;
+    } else {
+      kbase += (uint32_t)cb << shift;
+      const uint64_t e = (uint64_t)kbase + (uint64_t(1) << shift);
+      kend = e < kend ? e : kend;
+      if (shift == 0) break;            // the bracket is one score value
+      shift = shift >= 8 ? shift - 8 : 0;
+    }
   }
 
-  // ---- ties at tau, by position ---------------------------------------------
-  const uint32_t tau_key = prefix;
+  // ---- counts at tau: keys above and equal, per CTA, then over the cluster ----
+  const uint32_t tau_key = kbase;
   const float tau = key_score(tau_key);
-  const uint64_t w_tau = fixed_weight(tau, m, two_pow_frac);
+  uint32_t ngt = 0, neq = 0;
+  for (int i = tid; i < nloc; i += kSelThreads) {
+    const uint32_t k = score_key(scores[i]);
+    ngt += k > tau_key;
+    neq += k == tau_key;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    ngt += __shfl_xor_sync(0xffffffffu, ngt, o);
+    neq += __shfl_xor_sync(0xffffffffu, neq, o);
+  }
+  if (lane == 0) {
+    S.wcnt[warp] = ngt;
+    S.wcnt2[warp] = neq;
+  }
+  __syncthreads();
+  if (tid < C) {
+    uint32_t g = 0, e = 0;
+    for (int w = 0; w < kSelWarps; ++w) {
+      g += S.wcnt[w];
+      e += S.wcnt2[w];
+    }
+    cluster.map_shared_rank(S.gcount, tid)[rank] = g;
+    cluster.map_shared_rank(S.tcount, tid)[rank] = e;
+  }
+  cluster.sync();  // last distributed access
+  uint32_t cnt_above = 0, tau_cnt = 0;
+  int before = 0;
+  for (int r = 0; r < C; ++r) {
+    cnt_above += S.gcount[r];
+    tau_cnt += S.tcount[r];
+    if (r < rank) before += (int)S.tcount[r];
+  }
+  const uint64_t w_tau = sel_weight(tau, m, two_pow_frac);
   const uint64_t rem = target - mass_above;
   uint64_t n_tau64 = w_tau ? (rem + w_tau - 1) / w_tau : (uint64_t)tau_cnt;
   if (n_tau64 < 1) n_tau64 = 1;
   if (n_tau64 > tau_cnt) n_tau64 = tau_cnt;
   const int n_tau = (int)n_tau64;
-  const uint32_t my_tau = S.hist_cnt[tau_key & 1023u];  // this CTA's keys equal to tau
-  if (tid < C) cluster.map_shared_rank(S.tcount, tid)[rank] = my_tau;
-  cluster.sync();  // (D) last distributed access
-  int before = 0;
-  for (int r = 0; r < rank; ++r) before += (int)S.tcount[r];
-  const int want = n_tau - before;  // how many of this CTA's tau keys are taken
+  const int want = n_tau - before;           // how many of this CTA's tau keys are taken
+  const bool my_ties = S.tcount[rank] != 0;  // uniform over the CTA
 
   // ---- mask bits and the tie position ---------------------------------------
   int running = 0;
@@ -299,26 +319,29 @@ topp_decode_kernel(View4 qv, View4 kv, const int32_t* __restrict__ lens, int Hq,
     const bool valid = i < nloc;
     const uint32_t k = valid ? score_key(scores[i]) : 0u;
     const bool gt = valid && k > tau_key;
-    const bool eq = valid && k == tau_key;
-    const uint32_t beq = __ballot_sync(0xffffffffu, eq);
-    const int wpre = __popc(beq & ((1u << lane) - 1u));
-    if (lane == 0) S.wtot[warp] = __popc(beq);
-    __syncthreads();
-    int woff = 0, rtot = 0;
-    for (int w = 0; w < kSelWarps; ++w) {
-      const int t = (int)S.wtot[w];
-      woff += w < warp ? t : 0;
-      rtot += t;
+    bool sel = gt;
+    if (my_ties) {
+      const bool eq = valid && k == tau_key;
+      const uint32_t beq = __ballot_sync(0xffffffffu, eq);
+      const int wpre = __popc(beq & ((1u << lane) - 1u));
+      if (lane == 0) S.wcnt[warp] = __popc(beq);
+      __syncthreads();
+      int woff = 0, rtot = 0;
+      for (int w = 0; w < kSelWarps; ++w) {
+        const int t = (int)S.wcnt[w];
+        woff += w < warp ? t : 0;
+        rtot += t;
+      }
+      __syncthreads();
+      const int r_eq = running + woff + wpre;
+      sel = gt || (eq && r_eq < want);
+      if (eq && r_eq == want - 1) tiepos[qrow] = c0 + i;
+      running += rtot;
     }
-    __syncthreads();
-    const int r_eq = running + woff + wpre;
-    const bool sel = gt || (eq && r_eq < want);
-    if (eq && r_eq == want - 1) tiepos[qrow] = c0 + i;
     const uint32_t word = __ballot_sync(0xffffffffu, sel);
     const int wpos = base + warp * 32;
     const int w = (c0 + wpos) >> 5;
     if (lane == 0 && mrow && wpos < n_chunk && w < n_words_total) mrow[w] = word;
-    running += rtot;
   }
   if (rank == 0 && tid == 0) {
     tau_bits[qrow] = __float_as_uint(tau);
@@ -334,9 +357,9 @@ cudaError_t launch_topp_decode(const LaunchToppDecode& a, cudaStream_t stream) {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  // cluster size: enough CTAs to cover the GPU twice, and few enough keys per CTA
+  // cluster size: about one CTA per SM over all queries, and few enough keys per CTA
   int C = 1;
-  while (C < 8 && Q * C < 2 * sms) C <<= 1;
+  while (C < 8 && Q * C < sms) C <<= 1;
   while ((a.N + C - 1) / C > kMaxKeysPerCta && C < kMaxCluster) C <<= 1;
   int64_t n_chunk = (a.N + C - 1) / C;
   n_chunk = (n_chunk + 31) / 32 * 32;

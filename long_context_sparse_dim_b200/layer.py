@@ -57,8 +57,20 @@ class DecodeLayer:
         if self.R:
             rtp.index_project(self.k_ret, self.P, self.k_idx, stream)
 
-    def step(self, stream=None) -> torch.Tensor:
-        """One decode step over the resident cache; returns o [B, Hq, 1, D]."""
+    def step(self, stream=None, side_stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+        """One decode step over the resident cache; returns o [B, Hq, 1, D].
+
+        With ``side_stream`` the local heads' window attention (which does not
+        depend on the selection) runs there, forked from and joined back into
+        the main stream, so it overlaps the retrieval heads' chain."""
+        main = torch.cuda.current_stream() if stream is None else stream
+        local = self.Hkv > self.R
+        if side_stream is not None and local:
+            side_stream.wait_stream(main)
+            with torch.cuda.stream(side_stream):
+                rtp.window_attn(self.q_loc, self.k_loc, self.v_loc, self.lens, self.W, self.scale, self.o_loc,
+                                self.ws_loc, side_stream)
+            local = False
         if self.R:
             if self.lens_host is None:
                 n = self.N
@@ -72,7 +84,9 @@ class DecodeLayer:
             rtp.topp_select(self.q_idx, self.k_idx, self.lens, self.p, self.sel, self.ws_sel, stream)
             rtp.sparse_attn_decode(self.q_ret, self.k_ret, self.v_ret, self.lens, self.sel, self.scale,
                                    self.o_ret, self.ws_ret, stream)
-        if self.Hkv > self.R:
+        if local:
             rtp.window_attn(self.q_loc, self.k_loc, self.v_loc, self.lens, self.W, self.scale, self.o_loc,
                             self.ws_loc, stream)
+        if side_stream is not None and self.Hkv > self.R:
+            main.wait_stream(side_stream)
         return self.o
