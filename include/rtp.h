@@ -153,6 +153,30 @@ RTP_API rtp_status rtp_sparse_attn_decode(const rtp_tensor* q, const rtp_tensor*
                                   rtp_stream_t stream);
 RTP_API size_t rtp_sparse_attn_decode_workspace_size(int64_t B, int64_t Hq, int64_t Hk, int64_t N);
 
+/* ---- a4 (decode) without a caller workspace ------------------------------
+ * The pages have no counterpart to this call: it is a library-level variant
+ * of rtp_sparse_attn_decode (same arguments and results, minus the
+ * workspace) for callers that cannot allocate device memory -- for example a
+ * plugin inside a host framework that owns every device allocation and gives
+ * its plugins no allocator, or a runtime that reserves all device memory at
+ * start-up and forbids allocation afterwards.
+ *   - The split-K scratch lives in a fixed device array inside librtp.so,
+ *     RTP_NOALLOC_SCRATCH_BYTES long, which every GPU that loads the library
+ *     keeps until the process exits.  Shapes whose scratch would exceed it
+ *     (rtp_sparse_attn_decode_workspace_size() > RTP_NOALLOC_SCRATCH_BYTES)
+ *     return RTP_ERR_UNSUPPORTED.
+ *   - The first call on a device (with that device current) looks up the
+ *     array's device address; make that first call before any stream capture.
+ *   - All calls on a device share the array: calls that overlap on the GPU
+ *     race.  Order them on one stream.  Each call clears the part of the array
+ *     that must start at zero; the rest keeps the previous call's contents.
+ *   - Nothing is allocated: no cudaMalloc, cudaFree or allocating routine.
+ */
+#define RTP_NOALLOC_SCRATCH_BYTES (4u << 20)
+RTP_API rtp_status rtp_sparse_attn_decode_noalloc(const rtp_tensor* q, const rtp_tensor* k, const rtp_tensor* v,
+                                                  const int32_t* lens, const rtp_selection* sel, float scale,
+                                                  const rtp_tensor* o, rtp_stream_t stream);
+
 /* ---- a4 (prefill): causal attention over each query's selected keys ----
  *   q      [B, Hq, T, 128]  bf16;  k, v [B, Hk, N, 128] bf16
  *   q_idx  [B, Hq, T, 16], k_idx [B, Hk, N, 16]  bf16 (the inputs the selection used)

@@ -562,6 +562,16 @@ size_t attn_decode_workspace_bytes(int64_t B, int64_t Hq, int64_t Hk, int64_t N,
   return ((o_bytes + 255) / 256 * 256) + ((ml_bytes + 255) / 256 * 256) + ((t_bytes + 255) / 256 * 256);
 }
 
+void attn_decode_ticket_range(int64_t B, int64_t Hk, int64_t N, int32_t W, size_t* offset, size_t* bytes) {
+  int chunk = 0, splits = 0;
+  attn_layout(B, Hk, N, W, 148, &chunk, &splits);
+  const int64_t groups = B * Hk;
+  const size_t o_bytes = (size_t)groups * splits * kMaxGroup * kHeadDim * sizeof(float);
+  const size_t ml_bytes = (size_t)groups * splits * kMaxGroup * 2 * sizeof(float);
+  *offset = (o_bytes + 255) / 256 * 256 + (ml_bytes + 255) / 256 * 256;
+  *bytes = (size_t)(groups > 0 ? groups : 0) * sizeof(uint32_t);
+}
+
 bool attn_decode_supported(int64_t B, int64_t Hk, int64_t N, int32_t W) {
   int chunk = 0, splits = 0;
   attn_layout(B, Hk, N, W, 148, &chunk, &splits);

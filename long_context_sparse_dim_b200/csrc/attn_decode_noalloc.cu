@@ -1,0 +1,84 @@
+// rtp_sparse_attn_decode_noalloc: the decode sparse attention without a caller
+// workspace, for callers that cannot allocate device memory.
+//
+// Some callers of this library cannot call cudaMalloc: a plugin loaded into a
+// host framework that owns every device allocation and hands its plugins no
+// allocator, or a serving runtime that reserves all device memory at start-up
+// and forbids allocation afterwards.  Such a caller can pass its inputs and
+// outputs but has nowhere to put the split-K scratch that
+// rtp_sparse_attn_decode takes as a workspace.  This entry point keeps that
+// scratch in a fixed file-scope device array instead.
+//
+// Costs and limits of that choice:
+//   * every GPU that loads librtp.so holds RTP_NOALLOC_SCRATCH_BYTES of device
+//     memory for this array until the process exits;
+//   * shapes whose scratch would not fit are rejected (RTP_ERR_UNSUPPORTED);
+//   * all calls on a device share the one array, so calls that overlap on the
+//     GPU (different streams without ordering between them) race and give
+//     wrong results; order them on one stream;
+//   * the array's device address is looked up once per device, on the first
+//     call made with that device current (cudaGetSymbolAddress); make that
+//     first call before any stream capture.
+// The array keeps whatever the previous call left in it; the only part that
+// must start at zero (the per-group completion tickets) is cleared on the
+// stream by every call.  No cudaMalloc, cudaFree or allocating library routine
+// is called.
+#include <mutex>
+
+#include <cuda_runtime.h>
+
+#include "launch.h"
+#include "rtp.h"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[RTP_NOALLOC_SCRATCH_BYTES];
+
+std::mutex g_setup_mu;
+void* g_scratch_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device (looked up once).
+cudaError_t scratch_address(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_setup_mu);
+  if (!g_scratch_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    g_scratch_ptr[dev] = p;
+  }
+  *out = g_scratch_ptr[dev];
+  return cudaSuccess;
+}
+
+}  // namespace
+
+extern "C" rtp_status rtp_sparse_attn_decode_noalloc(const rtp_tensor* q, const rtp_tensor* k,
+                                                     const rtp_tensor* v, const int32_t* lens,
+                                                     const rtp_selection* sel, float scale,
+                                                     const rtp_tensor* o, rtp_stream_t stream) {
+  if (!q || !k || q->ndim != 4 || k->ndim != 4) return RTP_ERR_INVALID_ARG;
+  const size_t need = rtp_sparse_attn_decode_workspace_size(q->shape[0], q->shape[1], k->shape[1], k->shape[2]);
+  if (need > (size_t)RTP_NOALLOC_SCRATCH_BYTES) return RTP_ERR_UNSUPPORTED;
+  void* scratch = nullptr;
+  cudaError_t e = scratch_address(&scratch);
+  if (e != cudaSuccess) {
+    rtp::set_last_cuda_error((int32_t)e);
+    return RTP_ERR_CUDA;
+  }
+  size_t t_off = 0, t_bytes = 0;
+  rtp::attn_decode_ticket_range(q->shape[0], k->shape[1], k->shape[2], 0, &t_off, &t_bytes);
+  if (t_bytes) {
+    e = cudaMemsetAsync(static_cast<unsigned char*>(scratch) + t_off, 0, t_bytes, (cudaStream_t)stream);
+    if (e != cudaSuccess) {
+      rtp::set_last_cuda_error((int32_t)e);
+      return RTP_ERR_CUDA;
+    }
+  }
+  return rtp_sparse_attn_decode(q, k, v, lens, sel, scale, o, scratch, (size_t)RTP_NOALLOC_SCRATCH_BYTES, stream);
+}

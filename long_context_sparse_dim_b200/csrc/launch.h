@@ -53,5 +53,10 @@ struct LaunchAttnDecode {
 bool attn_decode_supported(int64_t B, int64_t Hk, int64_t N, int32_t W);
 size_t attn_decode_workspace_bytes(int64_t B, int64_t Hq, int64_t Hk, int64_t N, int32_t W);
 cudaError_t launch_attn_decode(const LaunchAttnDecode& a, cudaStream_t stream);
+// Byte range of the completion tickets inside a decode-attention workspace.
+void attn_decode_ticket_range(int64_t B, int64_t Hk, int64_t N, int32_t W, size_t* offset, size_t* bytes);
+
+// Records a CUDA error for rtp_last_cuda_error() on this thread.
+void set_last_cuda_error(int32_t e);
 
 }  // namespace rtp

@@ -67,6 +67,10 @@ rtp_status check_kv(const rtp_tensor* k, const rtp_tensor* v) {
 
 }  // namespace
 
+namespace rtp {
+void set_last_cuda_error(int32_t e) { g_last_cuda_error = e; }
+}  // namespace rtp
+
 extern "C" {
 
 const char* rtp_status_string(rtp_status s) {

@@ -24,7 +24,7 @@ STATUS_NAMES = {0: "RTP_OK", 1: "RTP_ERR_INVALID_ARG", 2: "RTP_ERR_SHAPE", 3: "R
                 4: "RTP_ERR_ALIGNMENT", 5: "RTP_ERR_WORKSPACE", 6: "RTP_ERR_CUDA", 7: "RTP_ERR_UNSUPPORTED"}
 
 EXPORTED = ("rtp_index_project", "rtp_topp_select", "rtp_topp_select_workspace_size",
-            "rtp_sparse_attn_decode", "rtp_sparse_attn_decode_workspace_size",
+            "rtp_sparse_attn_decode", "rtp_sparse_attn_decode_workspace_size", "rtp_sparse_attn_decode_noalloc",
             "rtp_sparse_attn_prefill", "rtp_sparse_attn_prefill_workspace_size",
             "rtp_window_attn", "rtp_window_attn_workspace_size",
             "rtp_status_string", "rtp_last_cuda_error", "rtp_version")
@@ -62,6 +62,7 @@ def _load() -> ctypes.CDLL:
         "rtp_topp_select_workspace_size": ([i64, i64, i64, i64, i64], sz),
         "rtp_sparse_attn_decode": ([T, T, T, vp, S, f32, T, vp, sz, vp], i32),
         "rtp_sparse_attn_decode_workspace_size": ([i64, i64, i64, i64], sz),
+        "rtp_sparse_attn_decode_noalloc": ([T, T, T, vp, S, f32, T, vp], i32),
         "rtp_sparse_attn_prefill": ([T, T, T, T, T, vp, S, f32, T, vp, sz, vp], i32),
         "rtp_sparse_attn_prefill_workspace_size": ([i64, i64, i64, i64, i64], sz),
         "rtp_window_attn": ([T, T, T, vp, i32, f32, T, vp, sz, vp], i32),
@@ -196,6 +197,20 @@ def sparse_attn_decode(q, k, v, lens, sel: Selection, scale: float, o, ws=None, 
                                        ctypes.byref(tensor_desc(v)), _ptr(lens), ctypes.byref(sel.desc()),
                                        float(scale), ctypes.byref(tensor_desc(o)), w, nb, _stream(stream)),
            "rtp_sparse_attn_decode")
+
+
+NOALLOC_SCRATCH_BYTES = 4 << 20
+
+
+def sparse_attn_decode_noalloc(q, k, v, lens, sel: Selection, scale: float, o, stream=None) -> None:
+    """rtp_sparse_attn_decode without a workspace, for callers that cannot
+    allocate device memory: the scratch is a fixed array inside the library
+    (NOALLOC_SCRATCH_BYTES per device, shared by all calls; keep calls ordered
+    on one stream, and make the first call on a device outside stream capture)."""
+    _check(_lib.rtp_sparse_attn_decode_noalloc(ctypes.byref(tensor_desc(q)), ctypes.byref(tensor_desc(k)),
+                                               ctypes.byref(tensor_desc(v)), _ptr(lens), ctypes.byref(sel.desc()),
+                                               float(scale), ctypes.byref(tensor_desc(o)), _stream(stream)),
+           "rtp_sparse_attn_decode_noalloc")
 
 
 def sparse_attn_prefill_workspace_size(B, Hq, T, Hk, N) -> int:
