@@ -44,7 +44,8 @@ constexpr float kLinBinsPerNat = 16.f; // pass 0 bin width 1/16 nat
 static_assert(kSelThreads == kBins, "one thread per histogram bin");
 
 struct SelSmem {
-  uint64_t whist[kSelWarps][kBins];  // per-warp private histograms
+  uint32_t whlo[kSelWarps][kBins];   // per-warp private histograms (64-bit masses as lo/hi words)
+  uint32_t whhi[kSelWarps][kBins];
   uint64_t hist[2][kBins];           // this CTA's histogram, double-buffered by pass parity
   uint64_t red[kBins];               // cluster-wide histogram (each CTA holds a copy)
   uint64_t wsum[kSelWarps];
@@ -57,6 +58,19 @@ struct SelSmem {
   int cut_bin;
   uint64_t cut_above;
 };
+
+// Exact 64-bit add into a (lo, hi) pair of 32-bit shared-memory words: native
+// 32-bit atomics, the carry out of the low word is added to the high word by the
+// one thread whose addition wrapped it.  (64-bit shared-memory atomics are far
+// slower on this part, more so under contention.)
+RTP_DEVICE void add_u64_pair(uint32_t* lo, uint32_t* hi, uint64_t w) {
+  const uint32_t l = (uint32_t)w;
+  uint32_t h = (uint32_t)(w >> 32);
+  const uint32_t old = atomicAdd(lo, l);
+  if (old + l < old) ++h;
+  if (h) atomicAdd(hi, h);
+}
+RTP_DEVICE uint64_t pair_value(uint32_t lo, uint32_t hi) { return ((uint64_t)hi << 32) | lo; }
 
 RTP_DEVICE float ex2f_fast(float x) {
   float y;
@@ -79,7 +93,7 @@ RTP_DEVICE int lin_bin(float s, float m) {
 
 template <typename T>
 __global__ void __launch_bounds__(kSelThreads)
-topp_decode_kernel(View4 qv, View4 kv, const int32_t* __restrict__ lens, int Hq, int G, int N,
+topp_query_kernel(View4 qv, View4 kv, const int32_t* __restrict__ lens, int Hq, int G, int N,
                    int n_chunk, float p, float two_pow_frac, uint32_t* __restrict__ tau_bits,
                    int32_t* __restrict__ tiepos, int32_t* __restrict__ count,
                    uint32_t* __restrict__ mask, int64_t mask_words) {
@@ -172,8 +186,12 @@ topp_decode_kernel(View4 qv, View4 kv, const int32_t* __restrict__ lens, int Hq,
   uint64_t kend = 0;
   int shift = 0;
   for (int pass = 0;; ++pass) {
-    uint64_t* wh = S.whist[warp];
-    for (int i = lane; i < kBins; i += 32) wh[i] = 0;
+    uint32_t* wlo = S.whlo[warp];
+    uint32_t* whi = S.whhi[warp];
+    for (int i = lane; i < kBins; i += 32) {
+      wlo[i] = 0;
+      whi[i] = 0;
+    }
     __syncwarp();
     for (int i = tid; i < nloc; i += kSelThreads) {
       const float sc = scores[i];
@@ -184,15 +202,14 @@ topp_decode_kernel(View4 qv, View4 kv, const int32_t* __restrict__ lens, int Hq,
         const uint32_t k = score_key(sc);
         if (k >= kbase && (uint64_t)k < kend) d = (int)((uint64_t)(k - kbase) >> shift);
       }
-      if (d >= 0) atomicAdd(reinterpret_cast<unsigned long long*>(&wh[d]),
-                            (unsigned long long)sel_weight(sc, m, two_pow_frac));
+      if (d >= 0) add_u64_pair(&wlo[d], &whi[d], sel_weight(sc, m, two_pow_frac));
     }
     __syncthreads();
     uint64_t* hb = S.hist[pass & 1];
     {
       uint64_t a = 0;
 #pragma unroll
-      for (int w = 0; w < kSelWarps; ++w) a += S.whist[w][tid];
+      for (int w = 0; w < kSelWarps; ++w) a += pair_value(S.whlo[w][tid], S.whhi[w][tid]);
       hb[tid] = a;
     }
     cluster.sync();  // every CTA's histogram of this pass is complete
@@ -351,28 +368,17 @@ topp_decode_kernel(View4 qv, View4 kv, const int32_t* __restrict__ lens, int Hq,
 
 bool topp_decode_supported(int64_t N) { return N <= (int64_t)kMaxKeysPerCta * kMaxCluster; }
 
-cudaError_t launch_topp_decode(const LaunchToppDecode& a, cudaStream_t stream) {
-  const int64_t Q = a.B * a.Hq;
-  if (Q == 0) return cudaSuccess;
+static int sm_count() {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  // cluster size: about one CTA per SM over all queries, and few enough keys per CTA
-  int C = 1;
-  while (C < 8 && Q * C < sms) C <<= 1;
-  while ((a.N + C - 1) / C > kMaxKeysPerCta && C < kMaxCluster) C <<= 1;
-  int64_t n_chunk = (a.N + C - 1) / C;
-  n_chunk = (n_chunk + 31) / 32 * 32;
-  if (n_chunk == 0) n_chunk = 32;
-  if (n_chunk > kMaxKeysPerCta) return cudaErrorInvalidValue;
-  const size_t smem = sizeof(SelSmem) + (size_t)n_chunk * sizeof(float);
-  int lg = 0;
-  while ((int64_t(1) << lg) < a.N) ++lg;
-  const float two_pow_frac = ldexpf(1.f, 63 - lg);
-  const int G = (int)(a.Hq / a.Hk);
+  return sms;
+}
 
+template <typename K, typename... Args>
+static cudaError_t launch_cluster(K kern, int grid, int C, size_t smem, cudaStream_t stream, Args... args) {
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(Q * C));
+  cfg.gridDim = dim3((unsigned)grid);
   cfg.blockDim = dim3(kSelThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
@@ -383,23 +389,38 @@ cudaError_t launch_topp_decode(const LaunchToppDecode& a, cudaStream_t stream) {
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-
-  cudaError_t e;
-  if (a.bf16) {
-    auto kern = topp_decode_kernel<__nv_bfloat16>;
-    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (C > 8) cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-    e = cudaLaunchKernelEx(&cfg, kern, a.q_idx, a.k_idx, a.lens, (int)a.Hq, G, (int)a.N, (int)n_chunk, a.p,
-                           two_pow_frac, a.tau_bits, a.tiepos, a.count, a.mask, a.mask_words);
-  } else {
-    auto kern = topp_decode_kernel<float>;
-    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (C > 8) cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-    e = cudaLaunchKernelEx(&cfg, kern, a.q_idx, a.k_idx, a.lens, (int)a.Hq, G, (int)a.N, (int)n_chunk, a.p,
-                           two_pow_frac, a.tau_bits, a.tiepos, a.count, a.mask, a.mask_words);
-  }
+  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (C > 8) cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, args...);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
+}
+
+cudaError_t launch_topp_decode(const LaunchToppDecode& a, cudaStream_t stream) {
+  const int64_t Q = a.B * a.Hq;
+  if (Q == 0) return cudaSuccess;
+  const int sms = sm_count();
+  int lg = 0;
+  while ((int64_t(1) << lg) < a.N) ++lg;
+  const float two_pow_frac = ldexpf(1.f, 63 - lg);
+  const int G = (int)(a.Hq / a.Hk);
+
+  // Query form: one cluster per query.
+  int C = 1;
+  while (C < 8 && Q * C < sms) C <<= 1;
+  while ((a.N + C - 1) / C > kMaxKeysPerCta && C < kMaxCluster) C <<= 1;
+  int64_t n_chunk = (a.N + C - 1) / C;
+  n_chunk = (n_chunk + 31) / 32 * 32;
+  if (n_chunk == 0) n_chunk = 32;
+  if (n_chunk > kMaxKeysPerCta) return cudaErrorInvalidValue;
+  const size_t smem = sizeof(SelSmem) + (size_t)n_chunk * sizeof(float);
+  if (a.bf16)
+    return launch_cluster(topp_query_kernel<__nv_bfloat16>, (int)(Q * C), C, smem, stream, a.q_idx, a.k_idx, a.lens,
+                          (int)a.Hq, G, (int)a.N, (int)n_chunk, a.p, two_pow_frac, a.tau_bits, a.tiepos, a.count,
+                          a.mask, a.mask_words);
+  return launch_cluster(topp_query_kernel<float>, (int)(Q * C), C, smem, stream, a.q_idx, a.k_idx, a.lens, (int)a.Hq,
+                        G, (int)a.N, (int)n_chunk, a.p, two_pow_frac, a.tau_bits, a.tiepos, a.count, a.mask,
+                        a.mask_words);
 }
 
 }  // namespace rtp
