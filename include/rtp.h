@@ -207,6 +207,16 @@ RTP_API rtp_status rtp_window_attn(const rtp_tensor* q, const rtp_tensor* k, con
                            void* workspace, size_t workspace_bytes, rtp_stream_t stream);
 RTP_API size_t rtp_window_attn_workspace_size(int64_t B, int64_t Hq, int64_t T, int64_t Hk, int64_t N, int32_t W);
 
+/* ---- device-side errors -------------------------------------------------
+ * Kernels that wait on asynchronous copies or tensor-core completions give up
+ * after about two seconds instead of hanging, and record a code in a device
+ * word.  rtp_poll_device_error synchronises the device, stores that code in
+ * *code (0: nothing happened; RTP_DEVICE_ERR_TIMEOUT: a wait gave up and the
+ * affected outputs are invalid) and clears it.
+ */
+#define RTP_DEVICE_ERR_TIMEOUT 1
+RTP_API rtp_status rtp_poll_device_error(int32_t* code);
+
 /* ---- utilities ---------------------------------------------------------- */
 RTP_API const char* rtp_status_string(rtp_status s);   /* static string, never NULL */
 RTP_API int32_t rtp_last_cuda_error(void);              /* cudaError_t of the last RTP_ERR_CUDA on this thread */

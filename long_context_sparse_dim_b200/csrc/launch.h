@@ -35,6 +35,42 @@ struct LaunchToppDecode {
 cudaError_t launch_topp_decode(const LaunchToppDecode& a, cudaStream_t stream);
 bool topp_decode_supported(int64_t N);
 
+// Top-p selection, prefill form (T query tokens per sequence), tcgen05 score tiles.
+struct LaunchToppPrefill {
+  View4 q_idx;   // [B, Hq, T, 16] bf16
+  View4 k_idx;   // [B, Hk, N, 16] bf16
+  const int32_t* lens;
+  int64_t B, Hq, Hk, T, N;
+  float p;
+  uint32_t* tau_bits;
+  int32_t* tiepos;
+  int32_t* count;
+  uint32_t* mask;
+  int64_t mask_words;
+  int* err;      // device error word
+};
+cudaError_t launch_topp_prefill(const LaunchToppPrefill& a, cudaStream_t stream);
+
+// Prefill attention (T query tokens per sequence, bf16): sparse form (threshold
+// selection + projected tiles) when W == 0, sliding window when W > 0.
+struct LaunchAttnPrefill {
+  View4 q, k, v;          // [B, Hq, T, 128], [B, Hk, N, 128]
+  View4 q_idx, k_idx;     // sparse form: [B, Hq, T, 16], [B, Hk, N, 16]
+  const int32_t* lens;
+  const uint32_t* tau_bits;
+  const int32_t* tiepos;
+  int64_t B, Hq, Hk, T, N;
+  int32_t W;
+  float scale;
+  MutView4 o;
+  bool o_bf16;
+  int* err;
+};
+cudaError_t launch_attn_prefill(const LaunchAttnPrefill& a, cudaStream_t stream);
+
+// Device address of the library's error word on the current device.
+cudaError_t device_error_word(int** out);
+
 // Decode attention: sparse (mask given) or sliding window (W > 0).
 struct LaunchAttnDecode {
   View4 q;       // [B, Hq, 1, 128]

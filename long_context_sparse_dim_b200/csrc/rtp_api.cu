@@ -142,7 +142,27 @@ rtp_status rtp_topp_select(const rtp_tensor* q_idx, const rtp_tensor* k_idx, con
                            rtp_topp_select_workspace_size(q_idx->shape[0], q_idx->shape[1], T,
                                                           k_idx->shape[1], N))) != RTP_OK)
     return s;
-  if (T != 1) return RTP_ERR_UNSUPPORTED;
+  if (T != 1) {
+    if (q_idx->dtype != RTP_BF16) return RTP_ERR_DTYPE;  // the tensor-core score tiles take bf16
+    rtp::LaunchToppPrefill a;
+    a.q_idx = view(q_idx);
+    a.k_idx = view(k_idx);
+    a.lens = lens;
+    a.B = q_idx->shape[0];
+    a.Hq = q_idx->shape[1];
+    a.Hk = k_idx->shape[1];
+    a.T = T;
+    a.N = N;
+    a.p = p;
+    a.tau_bits = out->tau_bits;
+    a.tiepos = out->tiepos;
+    a.count = out->count;
+    a.mask = out->mask;
+    a.mask_words = out->mask_words;
+    cudaError_t e = rtp::device_error_word(&a.err);
+    if (e != cudaSuccess) return cuda_status(e);
+    return cuda_status(rtp::launch_topp_prefill(a, (cudaStream_t)stream));
+  }
   if (!rtp::topp_decode_supported(N)) return RTP_ERR_UNSUPPORTED;
   rtp::LaunchToppDecode a;
   a.q_idx = view(q_idx);
@@ -226,13 +246,36 @@ rtp_status rtp_sparse_attn_prefill(const rtp_tensor* q, const rtp_tensor* k, con
                                    const rtp_tensor* q_idx, const rtp_tensor* k_idx, const int32_t* lens,
                                    const rtp_selection* sel, float scale, const rtp_tensor* o,
                                    void* workspace, size_t workspace_bytes, rtp_stream_t stream) {
-  (void)lens; (void)workspace; (void)workspace_bytes; (void)stream;
+  (void)workspace; (void)workspace_bytes;
   rtp_status s;
   if ((s = check_decode_common(q, k, v, o, scale)) != RTP_OK) return s;
   if ((s = check4(q_idx, 16)) != RTP_OK) return s;
   if ((s = check4(k_idx, 16)) != RTP_OK) return s;
   if (!sel || !sel->tau_bits || !sel->tiepos) return RTP_ERR_INVALID_ARG;
-  return RTP_ERR_UNSUPPORTED;
+  if (q->dtype != RTP_BF16 || q_idx->dtype != RTP_BF16 || k_idx->dtype != RTP_BF16) return RTP_ERR_DTYPE;
+  if (!same_bhn(q, q_idx) || !same_bhn(k, k_idx)) return RTP_ERR_SHAPE;
+  if (q->shape[2] > k->shape[2]) return RTP_ERR_SHAPE;
+  rtp::LaunchAttnPrefill a;
+  a.q = view(q);
+  a.k = view(k);
+  a.v = view(v);
+  a.q_idx = view(q_idx);
+  a.k_idx = view(k_idx);
+  a.lens = lens;
+  a.tau_bits = sel->tau_bits;
+  a.tiepos = sel->tiepos;
+  a.B = q->shape[0];
+  a.Hq = q->shape[1];
+  a.Hk = k->shape[1];
+  a.T = q->shape[2];
+  a.N = k->shape[2];
+  a.W = 0;
+  a.scale = scale;
+  a.o = mview(o);
+  a.o_bf16 = o->dtype == RTP_BF16;
+  cudaError_t e = rtp::device_error_word(&a.err);
+  if (e != cudaSuccess) return cuda_status(e);
+  return cuda_status(rtp::launch_attn_prefill(a, (cudaStream_t)stream));
 }
 
 // ---- a5 ----------------------------------------------------------------------------
@@ -251,7 +294,31 @@ rtp_status rtp_window_attn(const rtp_tensor* q, const rtp_tensor* k, const rtp_t
   const int64_t N = k->shape[2];
   const size_t need = rtp_window_attn_workspace_size(q->shape[0], q->shape[1], T, k->shape[1], N, W);
   if ((s = check_workspace(workspace, workspace_bytes, need)) != RTP_OK) return s;
-  if (T != 1) return RTP_ERR_UNSUPPORTED;
+  if (T != 1) {
+    if (q->dtype != RTP_BF16) return RTP_ERR_DTYPE;  // the prefill kernels take bf16
+    if (T > N) return RTP_ERR_SHAPE;
+    rtp::LaunchAttnPrefill a;
+    a.q = view(q);
+    a.k = view(k);
+    a.v = view(v);
+    a.q_idx = rtp::View4{nullptr, 0, 0, 0};
+    a.k_idx = rtp::View4{nullptr, 0, 0, 0};
+    a.lens = lens;
+    a.tau_bits = nullptr;
+    a.tiepos = nullptr;
+    a.B = q->shape[0];
+    a.Hq = q->shape[1];
+    a.Hk = k->shape[1];
+    a.T = T;
+    a.N = N;
+    a.W = W;
+    a.scale = scale;
+    a.o = mview(o);
+    a.o_bf16 = o->dtype == RTP_BF16;
+    cudaError_t e = rtp::device_error_word(&a.err);
+    if (e != cudaSuccess) return cuda_status(e);
+    return cuda_status(rtp::launch_attn_prefill(a, (cudaStream_t)stream));
+  }
   rtp::LaunchAttnDecode a;
   a.q = view(q);
   a.k = view(k);

@@ -90,3 +90,60 @@ class DecodeLayer:
         if side_stream is not None and self.Hkv > self.R:
             main.wait_stream(side_stream)
         return self.o
+
+
+class PrefillLayer:
+    """One attention layer's RTPurbo prefill: T query tokens per sequence (the
+    last T of its N-token context), causal.
+
+        a1  rtp_index_project   keys and queries of the retrieval heads -> 16-dim
+        a3  rtp_topp_select     per-token top-p over the causal prefix (tensor-core score tiles)
+        a4  rtp_sparse_attn_prefill   attention over each token's selected keys
+        a5  rtp_window_attn     sliding-window attention of the local heads
+    """
+
+    def __init__(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, P: torch.Tensor,
+                 R: int, W: int, p: float, lens: Optional[torch.Tensor] = None,
+                 out_dtype: torch.dtype = torch.float32, scale: Optional[float] = None,
+                 with_mask: bool = False):
+        B, Hq, T, D = q.shape
+        _, Hkv, N, _ = k.shape
+        self.B, self.Hq, self.Hkv, self.N, self.T, self.D = B, Hq, Hkv, N, T, D
+        self.G = Hq // Hkv
+        self.R, self.W, self.p = R, W, float(p)
+        self.scale = (D ** -0.5) if scale is None else scale
+        dev = q.device
+        G = self.G
+        self.q, self.k, self.v, self.P, self.lens = q, k, v, P, lens
+        self.q_ret, self.q_loc = q[:, : R * G], q[:, R * G:]
+        self.k_ret, self.v_ret = k[:, :R], v[:, :R]
+        self.k_loc, self.v_loc = k[:, R:], v[:, R:]
+        self.o = torch.zeros(B, Hq, T, D, dtype=out_dtype, device=dev)
+        self.o_ret, self.o_loc = self.o[:, : R * G], self.o[:, R * G:]
+        self.k_idx = torch.zeros(B, R, N, 16, dtype=torch.bfloat16, device=dev)
+        self.q_idx = torch.zeros(B, R * G, T, 16, dtype=torch.bfloat16, device=dev)
+        self.sel = rtp.Selection.empty(B * R * G * T, N, dev, with_mask=with_mask)
+        self.ws_loc = (rtp.workspace(rtp.window_attn_workspace_size(B, Hq - R * G, T, Hkv - R, N, W), dev)
+                       if Hkv > R else None)
+
+    def step(self, stream=None, side_stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+        main = torch.cuda.current_stream() if stream is None else stream
+        local = self.Hkv > self.R
+        if side_stream is not None and local:
+            side_stream.wait_stream(main)
+            with torch.cuda.stream(side_stream):
+                rtp.window_attn(self.q_loc, self.k_loc, self.v_loc, self.lens, self.W, self.scale, self.o_loc,
+                                self.ws_loc, side_stream)
+            local = False
+        if self.R:
+            rtp.index_project(self.k_ret, self.P, self.k_idx, stream)
+            rtp.index_project(self.q_ret, self.P, self.q_idx, stream)
+            rtp.topp_select(self.q_idx, self.k_idx, self.lens, self.p, self.sel, None, stream)
+            rtp.sparse_attn_prefill(self.q_ret, self.k_ret, self.v_ret, self.q_idx, self.k_idx, self.lens,
+                                    self.sel, self.scale, self.o_ret, None, stream)
+        if local:
+            rtp.window_attn(self.q_loc, self.k_loc, self.v_loc, self.lens, self.W, self.scale, self.o_loc,
+                            self.ws_loc, stream)
+        if side_stream is not None and self.Hkv > self.R:
+            main.wait_stream(side_stream)
+        return self.o

@@ -27,7 +27,7 @@ EXPORTED = ("rtp_index_project", "rtp_topp_select", "rtp_topp_select_workspace_s
             "rtp_sparse_attn_decode", "rtp_sparse_attn_decode_workspace_size", "rtp_sparse_attn_decode_noalloc",
             "rtp_sparse_attn_prefill", "rtp_sparse_attn_prefill_workspace_size",
             "rtp_window_attn", "rtp_window_attn_workspace_size",
-            "rtp_status_string", "rtp_last_cuda_error", "rtp_version")
+            "rtp_poll_device_error", "rtp_status_string", "rtp_last_cuda_error", "rtp_version")
 
 
 class RtpTensor(ctypes.Structure):
@@ -67,6 +67,7 @@ def _load() -> ctypes.CDLL:
         "rtp_sparse_attn_prefill_workspace_size": ([i64, i64, i64, i64, i64], sz),
         "rtp_window_attn": ([T, T, T, vp, i32, f32, T, vp, sz, vp], i32),
         "rtp_window_attn_workspace_size": ([i64, i64, i64, i64, i64, i32], sz),
+        "rtp_poll_device_error": ([P(i32)], i32),
         "rtp_status_string": ([i32], ctypes.c_char_p),
         "rtp_last_cuda_error": ([], i32),
         "rtp_version": ([], i32),
@@ -236,6 +237,13 @@ def window_attn(q, k, v, lens, W: int, scale: float, o, ws=None, stream=None) ->
     _check(_lib.rtp_window_attn(ctypes.byref(tensor_desc(q)), ctypes.byref(tensor_desc(k)),
                                 ctypes.byref(tensor_desc(v)), _ptr(lens), int(W), float(scale),
                                 ctypes.byref(tensor_desc(o)), w, nb, _stream(stream)), "rtp_window_attn")
+
+
+def poll_device_error() -> int:
+    """Synchronise, return and clear the device error word (0 = no error)."""
+    code = ctypes.c_int32(0)
+    _check(_lib.rtp_poll_device_error(ctypes.byref(code)), "rtp_poll_device_error")
+    return int(code.value)
 
 
 def version() -> int:
