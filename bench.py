@@ -36,8 +36,11 @@ sys.path.insert(0, ROOT)
 from long_context_sparse_dim_b200 import workloads as wls  # noqa: E402
 
 DECODE_WORKLOADS = {w.name: w for w in (wls.DECODE_B8_N32K, wls.DECODE_N4K_F32, wls.DECODE_B4_N128K)}
+PREFILL_WORKLOADS = {w.name: w for w in (wls.PREFILL_N32K, wls.PREFILL_N8K, wls.PREFILL_CHUNK_1M)}
+ALL_WORKLOADS = {**DECODE_WORKLOADS, **PREFILL_WORKLOADS}
 DEFAULT_WORKLOAD = wls.DECODE_B8_N32K.name
 METRIC = "decode sparse-attn tokens/s"
+METRIC_PREFILL = "prefill queries/s"
 ROW_BYTES = {"bf16": 2 * 128 * 2, "f32": 2 * 128 * 4}  # one K row + one V row
 L2_BYTES = 126 * 2 ** 20
 
@@ -49,6 +52,16 @@ def _peaks():
         return float(d["hbm_gbs"]), "measured"
     except Exception:
         return 6650.0, "fallback"
+
+
+def _tensor_peaks():
+    """(burst, sustained) dense bf16 TFLOP/s, and where they come from."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops"]), float(d["bf16_tflops_sustained"]), "measured"
+    except Exception:
+        return 1590.0, 1400.0, "fallback"
 
 
 def _dist():
@@ -387,23 +400,183 @@ def _e2e(layer, inst, wl, dev, steps):
             "d2h_bytes_per_step": int(d2h), "ms_per_step": ms, "steps": steps}
 
 
+# --------------------------------------------------------------------------
+# prefill
+# --------------------------------------------------------------------------
+
+def _prefill_calls(layer, side):
+    """The calls of one prefill step; returns (name, fn) pairs in launch order."""
+    from long_context_sparse_dim_b200 import rtp
+    L = layer
+    calls = []
+    if L.R:
+        calls += [("index_project_k", lambda: rtp.index_project(L.k_ret, L.P, L.k_idx)),
+                  ("index_project_q", lambda: rtp.index_project(L.q_ret, L.P, L.q_idx)),
+                  ("topp_select", lambda: rtp.topp_select(L.q_idx, L.k_idx, L.lens, L.p, L.sel)),
+                  ("sparse_attn_prefill", lambda: rtp.sparse_attn_prefill(
+                      L.q_ret, L.k_ret, L.v_ret, L.q_idx, L.k_idx, L.lens, L.sel, L.scale, L.o_ret))]
+    if L.Hkv > L.R:
+        calls += [("window_attn", lambda: rtp.window_attn(L.q_loc, L.k_loc, L.v_loc, L.lens, L.W, L.scale,
+                                                          L.o_loc, L.ws_loc))]
+    return calls
+
+
+def cpu_baseline_prefill(inst, wl, budget_s=10.0):
+    import oracle
+    L = oracle.LayerOracle(inst.q, inst.k, inst.v, inst.P, inst.lens, R=wl.R, W=wl.W,
+                           p=float(np.float32(wl.p)), storage=wl.dtype)
+    for kvh in range(wl.R):
+        L.k_idx(0, kvh)
+    rng = np.random.default_rng(0)
+    t0 = time.perf_counter()
+    done = 0
+    while time.perf_counter() - t0 < budget_s:
+        t = int(rng.integers(0, wl.T))
+        for h in range(wl.Hq):
+            L.query(0, h, t)
+        done += 1
+    dt = time.perf_counter() - t0
+    return {"value": done / dt, "unit": "queries/s", "cores": _oracle_cores(), "kind": "oracle",
+            "sample": f"{done} uniformly drawn query tokens x all {wl.Hq} heads of {wl.name}, "
+                      f"projected-key cache prebuilt, {dt:.1f} s"}
+
+
+def run_prefill(args, wl, rank, world, local_rank):
+    import torch
+    from long_context_sparse_dim_b200 import rtp  # noqa: F401
+    from long_context_sparse_dim_b200.layer import PrefillLayer
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    inst = wls.generate(wl)
+    q = torch.from_numpy(inst.q).to(dev, torch.bfloat16)
+    k = torch.from_numpy(inst.k).to(dev, torch.bfloat16)
+    v = torch.from_numpy(inst.v).to(dev, torch.bfloat16)
+    P = torch.from_numpy(inst.P).to(dev, torch.float32)
+    layer = PrefillLayer(q, k, v, P, R=wl.R, W=wl.W, p=wl.p)
+    side = torch.cuda.Stream(dev)
+    for _ in range(args.warmup):
+        layer.step(side_stream=side)
+    torch.cuda.synchronize()
+
+    # per-kernel times, serialised on one stream (events on the launching stream)
+    calls = _prefill_calls(layer, side)
+    reps = max(1, min(args.steps, 3))
+    times = {n: [] for n, _ in calls}
+    for _ in range(reps):
+        for n, fn in calls:
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            b.synchronize()
+            times[n].append(a.elapsed_time(b))
+    kernels_ms = {n: statistics.mean(v) for n, v in times.items()}
+
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    time.sleep(0.2)
+    barrier(world, dev)
+    torch.cuda.synchronize()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record()
+    for _ in range(args.steps):
+        layer.step(side_stream=side)
+    t_end.record()
+    torch.cuda.synchronize()
+    barrier(world, dev)
+    clock_info = clocks.stop()
+    assert rtp.poll_device_error() == 0, "a device wait timed out"
+    step_ms = max_over_ranks(t_start.elapsed_time(t_end) / args.steps, world, dev)
+
+    G, R = wl.G, wl.R
+    T, N = wl.T, wl.N
+    counts = layer.sel.count.cpu().numpy().astype(np.int64)
+    admitted = int(counts.sum())                       # (query, key) pairs the sparse attention runs
+    pos = np.arange(T) + N - T
+    causal = int((pos + 1).sum()) * R * G              # indexer (query, key) pairs
+    win = int(np.minimum(pos + 1, wl.W).sum()) * (wl.Hq - R * G)
+    burst, sustained, pk = _tensor_peaks()
+    attn_flop = 4.0 * 128 * admitted                   # QK^T + PV, 2 FLOP per MAC
+    win_flop = 4.0 * 128 * win
+    gemm_flop = 2.0 * 16 * causal                      # one pass of the depth-16 score GEMM
+    dom = max(("sparse_attn_prefill", attn_flop), ("window_attn", win_flop), key=lambda x: kernels_ms.get(x[0], 0))
+    dom_ach = dom[1] / (kernels_ms[dom[0]] * 1e-3) / 1e12
+    line = {
+        "metric": METRIC_PREFILL, "value": world * wl.B * T / (step_ms * 1e-3), "unit": "queries/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": wl.name, "B": wl.B, "T": T, "N": N, "Hq": wl.Hq, "Hkv": wl.Hkv,
+                   "retrieval_kv_heads": R, "W": wl.W, "p": wl.p,
+                   "l2": "inputs larger than L2 (K/V cache and score sweeps), no flush",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": {"kernel": dom[0], "bound": "tensor", "achieved": dom_ach, "peak": sustained,
+                     "unit": "TFLOP/s", "frac": dom_ach / sustained, "peak_kind": pk + " sustained",
+                     "traffic": None, "algorithmic_flop": dom[1], "ms_per_launch": kernels_ms[dom[0]]},
+        "score_gemm": {"kernel": "topp_select", "algorithmic_flop_one_pass": gemm_flop,
+                       "achieved_tflops_one_pass": gemm_flop / (kernels_ms["topp_select"] * 1e-3) / 1e12,
+                       "frac_of_burst": gemm_flop / (kernels_ms["topp_select"] * 1e-3) / 1e12 / burst},
+        "kernels_ms": kernels_ms,
+        "selection": {"mean_selected_fraction": admitted / max(causal, 1)},
+        "gpu_launches": len(calls) * args.steps,
+        "streams": "window attention (local heads) forked onto a second stream inside each step",
+        "clocks": clock_info,
+    }
+    line["e2e"] = _e2e_prefill(layer, inst, dev, side, max(1, min(args.steps, 3)))
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_prefill(inst, wl, args.cpu_budget)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def _e2e_prefill(layer, inst, dev, side, steps):
+    import torch
+    h_q = torch.from_numpy(inst.q).to(torch.bfloat16).pin_memory()
+    h_k = torch.from_numpy(inst.k).to(torch.bfloat16).pin_memory()
+    h_v = torch.from_numpy(inst.v).to(torch.bfloat16).pin_memory()
+    h_o = torch.empty(layer.o.shape, dtype=layer.o.dtype).pin_memory()
+    h2d = sum(x.numel() * x.element_size() for x in (h_q, h_k, h_v))
+    d2h = h_o.numel() * h_o.element_size()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(steps):
+        layer.q.copy_(h_q, non_blocking=True)
+        layer.k.copy_(h_k, non_blocking=True)
+        layer.v.copy_(h_v, non_blocking=True)
+        layer.step(side_stream=side)
+        h_o.copy_(layer.o, non_blocking=True)
+        torch.cuda.current_stream().synchronize()
+    t1.record()
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1) / steps
+    return {"value": inst.wl.B * inst.wl.T / (ms * 1e-3), "unit": "queries/s", "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h), "ms_per_step": ms, "steps": steps}
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(DECODE_WORKLOADS))
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(ALL_WORKLOADS))
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
-    wl = DECODE_WORKLOADS[args.workload]
+    wl = ALL_WORKLOADS[args.workload]
     rank, world, local_rank = _dist()
     try:
         if args.impl == "reference":
             return run_reference(args, wl, rank)
+        if wl.mode == "prefill":
+            return run_prefill(args, wl, rank, world, local_rank)
         return run_ours(args, wl, rank, world, local_rank)
     finally:
         if world > 1:

@@ -18,16 +18,20 @@
 //   warp 5     MMA issuer (one elected lane)
 // The cut of every row is found by sweeps over its causal prefix; each sweep
 // recomputes the score tiles (depth-16 MMAs are cheap) and narrows a bracket
-// around the cut score:
-//   MAX   row maximum m
-//   L0    Z = sum of 64-bit fixed-point weights; 32 bins of (m - s) 1/4 nat wide
-//   L1    32 sub-bins of the L0 cut bin (1/128 nat)
-//   KEY   5-bit digits of the order-preserving uint32 image of s inside the
-//         bracket, until the bracket is one score value tau
-//   TIE   keys above tau are counted, the n-th key equal to tau (position
-//         order) gives tiepos, and the optional selection mask is written
-// A row owns its 32-bin histogram column in shared memory, so no atomics are
-// needed.  Sweeps continue while any row of the block is unresolved.
+// around the cut score, every row on the same schedule:
+//   MAX      row maximum m
+//   LIN 0-3  32 bins of u = m - s, 1/4, 1/128, 1/4096, 1/131072 nat wide (each
+//            level splits the previous cut bin; power-of-two rescaling of u is
+//            exact), with 64-bit fixed-point masses (Z on level 0) and counts
+//   COLLECT  once the cut bin holds <= 32 keys, their (score, position) pairs
+//            are kept and an in-thread sort by (score desc, position asc)
+//            finishes the cut: tau, the number taken, tiepos, count
+// Fallbacks: the tail bin of level 0, or a bin still too full after level 3,
+// continue with 5-bit digits of the order-preserving uint32 image of the score
+// (KEY) until one value is left, then a TIE sweep counts and locates the ties;
+// the TIE sweep also writes the optional selection mask.
+// A row owns its 32-bin histogram columns in shared memory (no atomics); the
+// candidate list reuses the row's mass column.
 #include <cudaTypedefs.h>
 
 #include <math.h>
@@ -40,17 +44,18 @@ namespace rtp {
 constexpr int kPfRows = 128;      // query rows per CTA (TMEM lanes)
 constexpr int kPfKeys = 64;       // keys per score tile (MMA N)
 constexpr int kPfStages = 4;      // K_idx tile ring
-constexpr int kPfBins = 32;       // histogram bins per row
+constexpr int kPfBins = 32;       // histogram bins per row (also the candidate capacity)
 constexpr int kPfThreads = 192;   // 4 epilogue warps + producer + MMA
 constexpr int kPfTileBytes = kPfKeys * kIdxDim * 2;  // 2 KB
 constexpr int kPfTmemCols = 2 * kPfKeys;             // two accumulator buffers
 
-enum PfLevel : int { kLvMax = 0, kLvL0 = 1, kLvL1 = 2, kLvKey = 3, kLvTie = 4, kLvDone = 5 };
+enum PfLevel : int { kLvMax = 0, kLvLin = 1, kLvCollect = 2, kLvKey = 3, kLvTie = 4, kLvDone = 5 };
 
 struct PfSmem {
   alignas(1024) uint8_t qtile[kPfRows * kIdxDim * 2];            // A operand, 4 KB
   alignas(1024) uint8_t ktile[kPfStages][kPfTileBytes];           // B operand ring
-  uint64_t hist[kPfBins][kPfRows];                                // per-row mass histograms
+  uint64_t hist[kPfBins][kPfRows];                                // per-row masses / candidates
+  uint32_t hcnt[kPfBins][kPfRows];                                // per-row counts
   uint64_t q_full;
   uint64_t k_full[kPfStages];
   uint64_t k_empty[kPfStages];
@@ -78,12 +83,12 @@ RTP_DEVICE uint64_t pf_weight(float s, float m, float two_pow_frac) {
   return __float2ull_rn(__fmul_rn(e, two_pow_frac));
 }
 
-__global__ void __launch_bounds__(kPfThreads)
+__global__ void __launch_bounds__(kPfThreads, 3)
 topp_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap, PfArgs A) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   PfSmem& S = *reinterpret_cast<PfSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int t0 = blockIdx.x * kPfRows;
+  const int t0 = (gridDim.x - 1 - blockIdx.x) * kPfRows;  // the longest prefixes start first
   const int bh = blockIdx.y;
   const int b = bh / A.Hq, h = bh % A.Hq, kvh = h / A.G;
   int n_b = A.N;
@@ -127,7 +132,9 @@ topp_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
   }
   float m = -INFINITY;
   uint64_t Z = 0, target = 0, mass_above = 0;
-  int b0 = 0, b1 = 0, shift = 0, n_tau = 0, ngt = 0, neq = 0, tiepos = -1;
+  uint32_t cnt_above = 0;
+  int lin = 0, prefix = 0, tail = 0, shift = 0, n_tau = 0, ngt = 0, neq = 0, tiepos = -1, ncand = 0;
+  float lscale = 4.f;  // bins of level `lin`: floor(u * lscale)
   uint32_t kbase = 0, tau_key = 0;
   uint64_t kend = 0;
   uint32_t* mrow = (A.mask && is_row && t < A.T) ? A.mask + ((int64_t)bh * A.T + t) * A.mask_words : nullptr;
@@ -137,8 +144,12 @@ topp_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
     const int more = __syncthreads_or(is_row && level != kLvDone);
     const int abort = __syncthreads_or(!alive);
     if (!more || abort || ntiles == 0) break;
-    if (is_row && (level == kLvL0 || level == kLvL1 || level == kLvKey))
-      for (int i = 0; i < kPfBins; ++i) S.hist[i][row] = 0;
+    if (is_row && (level == kLvLin || level == kLvKey))
+      for (int i = 0; i < kPfBins; ++i) {
+        S.hist[i][row] = 0;
+        S.hcnt[i][row] = 0;
+      }
+    if (is_row) ncand = 0;
 
     if (warp == 4) {
       // ---------------- TMA producer ----------------
@@ -177,77 +188,112 @@ topp_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
         const uint32_t gi = g + i, buf = gi & 1;
         if (!mbar_wait(&S.t_full[buf], (gi >> 1) & 1, alive, A.err)) break;
         tc_fence_after();
-        uint32_t v[2][32];
         const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16) + buf * kPfKeys;
-        tmem_ld32(taddr, v[0]);
-        tmem_ld32(taddr + 32, v[1]);
-        tmem_ld_wait();
-        tc_fence_before();
-        mbar_arrive(&S.t_empty[buf]);
-        if (level == kLvDone) continue;
         const int key0 = i * kPfKeys;
-        const int nv = pos - key0 + 1;  // keys of this tile inside the row's causal prefix
-        uint32_t mbits[2] = {0u, 0u};
-        if (level == kLvMax) {
-#pragma unroll
-          for (int j = 0; j < kPfKeys; ++j)
-            if (j < nv) m = fmaxf(m, __fadd_rn(__fmul_rn(__uint_as_float(v[j >> 5][j & 31]), 0.25f), 0.0f));
-        } else if (level == kLvTie) {
-#pragma unroll
-          for (int j = 0; j < kPfKeys; ++j) {
-            if (j < nv) {
-              const float s = __fadd_rn(__fmul_rn(__uint_as_float(v[j >> 5][j & 31]), 0.25f), 0.0f);
-              const uint32_t k = score_key(s);
-              const bool gt = k > tau_key;
-              bool sel = gt;
-              ngt += gt;
-              if (k == tau_key) {
-                ++neq;
-                sel = neq <= n_tau;
-                if (neq == n_tau) tiepos = key0 + j;
-              }
-              mbits[j >> 5] |= (uint32_t)sel << (j & 31);
-            }
+        uint64_t mbits = 0ull;
+#pragma unroll 1
+        for (int half = 0; half < 2; ++half) {
+          uint32_t v[32];
+          tmem_ld32(taddr + half * 32, v);
+          tmem_ld_wait();
+          if (half == 1) {
+            tc_fence_before();
+            mbar_arrive(&S.t_empty[buf]);
           }
-        } else {
+          if (level == kLvDone) continue;
+          const int kb = key0 + half * 32;
+          const int nv = pos - kb + 1;  // keys of this chunk inside the row's causal prefix
+          if (nv <= 0) continue;
+          if (level == kLvMax) {
+            if (nv >= 32) {
 #pragma unroll
-          for (int j = 0; j < kPfKeys; ++j) {
-            if (j < nv) {
-              const float s = __fadd_rn(__fmul_rn(__uint_as_float(v[j >> 5][j & 31]), 0.25f), 0.0f);
-              const float u = __fsub_rn(mh, s);
-              const float u4 = __fmul_rn(u, 4.f);
-              const int l0 = u4 >= 31.f ? 31 : (int)u4;
-              int d = -1;
-              if (level == kLvL0) {
-                d = l0;
-              } else if (l0 == b0) {
-                if (level == kLvL1) {
-                  d = (int)__fmul_rn(u, 128.f) - 32 * b0;
-                } else {
-                  bool in = true;
-                  if (b0 < 31) in = ((int)__fmul_rn(u, 128.f) - 32 * b0) == b1;
-                  const uint32_t k = score_key(s);
-                  if (in && k >= kbase && (uint64_t)k < kend) d = (int)((k - kbase) >> shift);
+              for (int j = 0; j < 32; ++j) m = fmaxf(m, __uint_as_float(v[j]));
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (j < nv) m = fmaxf(m, __uint_as_float(v[j]));
+            }
+          } else if (level == kLvTie) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              if (j < nv) {
+                const float sv = __fadd_rn(__fmul_rn(__uint_as_float(v[j]), 0.25f), 0.0f);
+                const uint32_t k = score_key(sv);
+                const bool gt = k > tau_key;
+                bool sel = gt;
+                ngt += gt;
+                if (k == tau_key) {
+                  ++neq;
+                  sel = neq <= n_tau;
+                  if (neq == n_tau) tiepos = kb + j;
+                }
+                mbits |= (uint64_t)sel << (half * 32 + j);
+              }
+            }
+          } else if (level == kLvLin) {
+            const int nvc = nv < 32 ? nv : 32;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              if (j < nvc) {
+                const float sv = __fadd_rn(__fmul_rn(__uint_as_float(v[j]), 0.25f), 0.0f);
+                const float t = __fmul_rn(__fsub_rn(mh, sv), lscale);
+                const int ti = lin == 0 ? (t >= 31.f ? 31 : (int)t) : (t >= 2.0e9f ? -1 : (int)t);
+                if ((ti >> 5) == prefix && ti >= 0) {
+                  const int d = ti & 31;
+                  const uint64_t w = pf_weight(sv, mh, A.two_pow_frac);
+                  Z += w;
+                  S.hist[d][row] += w;
+                  S.hcnt[d][row] += 1u;
                 }
               }
-              if (d >= 0) {
-                const uint64_t w = pf_weight(s, mh, A.two_pow_frac);
-                if (level == kLvL0) Z += w;
-                S.hist[d][row] += w;
+            }
+          } else if (level == kLvCollect) {
+            const int nvc = nv < 32 ? nv : 32;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              if (j < nvc) {
+                const float sv = __fadd_rn(__fmul_rn(__uint_as_float(v[j]), 0.25f), 0.0f);
+                const float t = __fmul_rn(__fsub_rn(mh, sv), lscale);
+                const int ti = lin == 0 ? (t >= 31.f ? 31 : (int)t) : (t >= 2.0e9f ? -1 : (int)t);
+                if (ti == prefix && ncand < kPfBins) {
+                  S.hist[ncand][row] = ((uint64_t)(uint32_t)(kb + j) << 32) | __float_as_uint(sv);
+                  ++ncand;
+                }
+              }
+            }
+          } else {  // KEY fallback
+            const int nvc = nv < 32 ? nv : 32;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              if (j < nvc) {
+                const float sv = __fadd_rn(__fmul_rn(__uint_as_float(v[j]), 0.25f), 0.0f);
+                const float t = __fmul_rn(__fsub_rn(mh, sv), lscale);
+                const int ti = tail ? 31 : (t >= 2.0e9f ? -1 : (int)t);
+                const int tl = tail ? (__fmul_rn(__fsub_rn(mh, sv), 4.f) >= 31.f ? 31 : -1) : ti;
+                const uint32_t k = score_key(sv);
+                if (tl == prefix && k >= kbase && (uint64_t)k < kend) {
+                  const int d = (int)((k - kbase) >> shift);
+                  S.hist[d][row] += pf_weight(sv, mh, A.two_pow_frac);
+                  S.hcnt[d][row] += 1u;
+                }
               }
             }
           }
         }
         if (level == kLvTie && mrow) {
           const int w0 = key0 >> 5;
-          if (w0 < A.mask_words) mrow[w0] = mbits[0];
-          if (w0 + 1 < A.mask_words) mrow[w0 + 1] = mbits[1];
+          if (w0 < A.mask_words) mrow[w0] = (uint32_t)mbits;
+          if (w0 + 1 < A.mask_words) mrow[w0 + 1] = (uint32_t)(mbits >> 32);
         }
       }
       // ---- end of sweep: advance this row's bracket ----
       if (is_row && level != kLvDone && alive) {
         if (level == kLvMax) {
-          level = kLvL0;
+          m = __fadd_rn(__fmul_rn(m, 0.25f), 0.0f);  // same rounding as every score
+          level = kLvLin;
+          lin = 0;
+          prefix = 0;
+          lscale = 4.f;
         } else if (level == kLvTie) {
           if (mrow)  // words past the block's last tile
             for (int64_t w = 2 * (int64_t)ntiles; w < (A.N + 31) / 32; ++w) mrow[w] = 0u;
@@ -256,15 +302,59 @@ topp_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
           A.tiepos[qrow] = tiepos;
           A.count[qrow] = ngt + n_tau;
           level = kLvDone;
-        } else {
-          if (level == kLvL0) {
+        } else if (level == kLvCollect) {
+          // sort the candidates by (score desc, position asc), then take them in order
+          for (int a = 1; a < ncand; ++a) {
+            const uint64_t x = S.hist[a][row];
+            const uint32_t xk = score_key(__uint_as_float((uint32_t)x));
+            const uint32_t xp = (uint32_t)(x >> 32);
+            int bI = a - 1;
+            while (bI >= 0) {
+              const uint64_t y = S.hist[bI][row];
+              const uint32_t yk = score_key(__uint_as_float((uint32_t)y));
+              if (yk > xk || (yk == xk && (uint32_t)(y >> 32) < xp)) break;
+              S.hist[bI + 1][row] = y;
+              --bI;
+            }
+            S.hist[bI + 1][row] = x;
+          }
+          const uint64_t need = target - mass_above;
+          uint64_t cum = 0;
+          int taken = ncand;
+          for (int a = 0; a < ncand; ++a) {
+            cum += pf_weight(__uint_as_float((uint32_t)S.hist[a][row]), mh, A.two_pow_frac);
+            if (cum >= need) {
+              taken = a + 1;
+              break;
+            }
+          }
+          if (taken < 1) taken = 1;
+          const uint64_t last = S.hist[taken - 1][row];
+          tau_key = score_key(__uint_as_float((uint32_t)last));
+          n_tau = 0;
+          for (int a = 0; a < taken; ++a) n_tau += score_key(__uint_as_float((uint32_t)S.hist[a][row])) == tau_key;
+          const int cnt = (int)cnt_above + taken;
+          if (mrow) {  // the selection mask needs one more sweep
+            ngt = 0;
+            neq = 0;
+            tiepos = -1;
+            level = kLvTie;
+          } else {
+            const int64_t qrow = (int64_t)bh * A.T + t;
+            A.tau_bits[qrow] = __float_as_uint(key_score(tau_key));
+            A.tiepos[qrow] = (int)(last >> 32);
+            A.count[qrow] = cnt;
+            level = kLvDone;
+          }
+        } else {  // LIN or KEY: find the cut bin
+          if (level == kLvLin && lin == 0) {
             const double tt = ceil((double)A.p * (double)Z);
             uint64_t tg = tt >= (double)Z ? Z : (uint64_t)tt;
             target = tg < 1 ? 1 : tg;
           }
           const uint64_t need = target - mass_above;
-          // bins in descending score order: L0/L1 bin 0 first; KEY bin 31 first
           uint64_t cum = 0;
+          uint32_t cumc = 0;
           int cut = 0;
           for (int r = 0; r < kPfBins; ++r) {
             const int bin = level == kLvKey ? kPfBins - 1 - r : r;
@@ -274,13 +364,16 @@ topp_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
               break;
             }
             cum += hv;
+            cumc += S.hcnt[bin][row];
           }
           mass_above += cum;
-          if (level == kLvL0) {
-            b0 = cut;
-            if (b0 < 31) {
-              level = kLvL1;
-            } else {  // the tail bin: key window from the lowest key up to m - 7.75
+          cnt_above += cumc;
+          const uint32_t in_bin = S.hcnt[cut][row];
+          if (level == kLvLin) {
+            if (lin == 0 && cut == 31) {
+              // tail bin (u >= 7.75): exact digits over the keys up to m - 7.75
+              tail = 1;
+              prefix = 31;
               const float hi_s = mh - 7.75f;
               const float mg = 1e-5f * (fabsf(mh) + 8.f) + 1e-30f;
               kbase = 0u;
@@ -288,18 +381,25 @@ topp_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
               shift = 0;
               while (((kend - kbase - 1) >> shift) >= (uint64_t)kPfBins) ++shift;
               level = kLvKey;
+            } else {
+              prefix = (prefix << 5) | cut;
+              if (in_bin <= (uint32_t)kPfBins) {
+                level = kLvCollect;  // same scale: keys whose level-`lin` bin is `prefix`
+              } else if (lin < 3) {
+                ++lin;
+                lscale *= 32.f;
+              } else {
+                // still too many keys: exact digits inside the bracket of this bin
+                const float hi_s = mh - (float)prefix / lscale;
+                const float lo_s = mh - (float)(prefix + 1) / lscale;
+                const float mg = 1e-5f * (fabsf(mh) + (float)(prefix + 1) / lscale) + 1e-30f;
+                kbase = score_key(__fadd_rn(lo_s - mg, 0.0f));
+                kend = (uint64_t)score_key(__fadd_rn(hi_s + mg, 0.0f)) + 1;
+                shift = 0;
+                while (((kend - kbase - 1) >> shift) >= (uint64_t)kPfBins) ++shift;
+                level = kLvKey;
+              }
             }
-          } else if (level == kLvL1) {
-            b1 = cut;
-            const int fine = 32 * b0 + b1;  // u in [fine/128, (fine+1)/128)
-            const float hi_s = mh - (float)fine / 128.f;
-            const float lo_s = mh - (float)(fine + 1) / 128.f;
-            const float mg = 1e-5f * (fabsf(mh) + (float)(fine + 1) / 128.f) + 1e-30f;
-            kbase = score_key(__fadd_rn(lo_s - mg, 0.0f));
-            kend = (uint64_t)score_key(__fadd_rn(hi_s + mg, 0.0f)) + 1;
-            shift = 0;
-            while (((kend - kbase - 1) >> shift) >= (uint64_t)kPfBins) ++shift;
-            level = kLvKey;
           } else {  // KEY
             kbase += (uint32_t)cut << shift;
             const uint64_t e = (uint64_t)kbase + (uint64_t(1) << shift);
@@ -310,6 +410,9 @@ topp_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
               const uint64_t rem = target - mass_above;
               uint64_t nt = w_tau ? (rem + w_tau - 1) / w_tau : 1;
               n_tau = (int)(nt < 1 ? 1 : nt);
+              ngt = 0;
+              neq = 0;
+              tiepos = -1;
               level = kLvTie;
             } else {
               shift = shift >= 5 ? shift - 5 : 0;

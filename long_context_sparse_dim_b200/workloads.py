@@ -120,13 +120,18 @@ PREFILL_N32K = Workload(
     name="prefill_t32768_llama8b_2ret6loc", mode="prefill", B=1, Hq=32, Hkv=8, R=2,
     N=32768, T=32768, W=4096, p=0.95, dtype="bf16", needle_mode="fraction",
     needle_fraction=0.10, seed=3)
+# Same layer and recipe at 8192 tokens: small enough for detailed profiler captures.
+PREFILL_N8K = Workload(
+    name="prefill_t8192_llama8b_2ret6loc", mode="prefill", B=1, Hq=32, Hkv=8, R=2,
+    N=8192, T=8192, W=4096, p=0.95, dtype="bf16", needle_mode="fraction",
+    needle_fraction=0.10, seed=5)
 PREFILL_CHUNK_1M = Workload(
     name="prefill_chunk_t8192_n1048576_llama8b_2ret6loc", mode="prefill", B=1, Hq=32,
     Hkv=8, R=2, N=1048576, T=8192, W=8192, p=0.95, dtype="bf16", needle_mode="strata",
     needle_count=256, seed=4)
 
 WORKLOADS: Dict[str, Workload] = {w.name: w for w in (
-    DECODE_N4K_F32, DECODE_B8_N32K, DECODE_B4_N128K, PREFILL_N32K, PREFILL_CHUNK_1M)}
+    DECODE_N4K_F32, DECODE_B8_N32K, DECODE_B4_N128K, PREFILL_N32K, PREFILL_N8K, PREFILL_CHUNK_1M)}
 
 
 # --------------------------------------------------------------------------
