@@ -43,7 +43,7 @@ namespace rtp {
 
 constexpr int kPfRows = 128;      // query rows per CTA (TMEM lanes)
 constexpr int kPfKeys = 64;       // keys per score tile (MMA N)
-constexpr int kPfStages = 4;      // K_idx tile ring
+constexpr int kPfStages = 2;      // K_idx tile ring
 constexpr int kPfBins = 32;       // histogram bins per row (also the candidate capacity)
 constexpr int kPfThreads = 192;   // 4 epilogue warps + producer + MMA
 constexpr int kPfTileBytes = kPfKeys * kIdxDim * 2;  // 2 KB
@@ -52,10 +52,10 @@ constexpr int kPfTmemCols = 2 * kPfKeys;             // two accumulator buffers
 enum PfLevel : int { kLvMax = 0, kLvLin = 1, kLvCollect = 2, kLvKey = 3, kLvTie = 4, kLvDone = 5 };
 
 struct PfSmem {
-  alignas(1024) uint8_t qtile[kPfRows * kIdxDim * 2];            // A operand, 4 KB
-  alignas(1024) uint8_t ktile[kPfStages][kPfTileBytes];           // B operand ring
+  alignas(256) uint8_t qtile[kPfRows * kIdxDim * 2];             // A operand, 4 KB
+  alignas(256) uint8_t ktile[kPfStages][kPfTileBytes];            // B operand ring
   uint64_t hist[kPfBins][kPfRows];                                // per-row masses / candidates
-  uint32_t hcnt[kPfBins][kPfRows];                                // per-row counts
+  uint16_t hcnt[kPfBins][kPfRows];                                // per-row counts (saturating)
   uint64_t q_full;
   uint64_t k_full[kPfStages];
   uint64_t k_empty[kPfStages];
@@ -77,19 +77,25 @@ struct PfArgs {
   int* err;
 };
 
-RTP_DEVICE uint64_t pf_weight(float s, float m, float two_pow_frac) {
+// Fixed-point weight of a key at raw distance u = m - v from the row maximum:
+// round(2^(u * wmul) * 2^frac) with wmul = -log2(e) / 4, i.e. exp(s - max s).
+RTP_DEVICE uint64_t pf_weight_u(float u, float wmul, float two_pow_frac) {
   float e;
-  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(e) : "f"(__fmul_rn(__fsub_rn(s, m), 1.4426950408889634f)));
+  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(e) : "f"(__fmul_rn(u, wmul)));
   return __float2ull_rn(__fmul_rn(e, two_pow_frac));
 }
 
-__global__ void __launch_bounds__(kPfThreads, 3)
+__global__ void __launch_bounds__(kPfThreads, 2)
 topp_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap, PfArgs A) {
-  extern __shared__ __align__(1024) unsigned char smem_raw[];
-  PfSmem& S = *reinterpret_cast<PfSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(256) unsigned char smem_raw[];
+  PfSmem& S = *reinterpret_cast<PfSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 255) & ~uintptr_t(255));
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int t0 = (gridDim.x - 1 - blockIdx.x) * kPfRows;  // the longest prefixes start first
-  const int bh = blockIdx.y;
+  // 1-D grid ordered longest causal prefix first across all heads, so every SM
+  // receives a mix of long and short blocks
+  const int nb = (A.T + kPfRows - 1) / kPfRows;
+  const int heads = (int)(gridDim.x / nb);
+  const int t0 = (nb - 1 - (int)blockIdx.x / heads) * kPfRows;
+  const int bh = (int)blockIdx.x % heads;
   const int b = bh / A.Hq, h = bh % A.Hq, kvh = h / A.G;
   int n_b = A.N;
   if (A.lens) n_b = min(max(A.lens[b], 0), A.N);
@@ -130,13 +136,17 @@ topp_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
     A.tiepos[qrow] = -1;
     A.count[qrow] = 0;
   }
+  // Everything below works on raw accumulators v (the score is s = v / 4, an
+  // exact scaling): u = m - v with m the row's raw maximum.  Level-k bins are
+  // floor(u * 32^k) (level 0: floor(u), the tail folded into bin 31), so a
+  // level-k bin P is the interval [P / 32^k, (P + 1) / 32^k) of u, exactly.
   float m = -INFINITY;
-  uint64_t Z = 0, target = 0, mass_above = 0;
-  uint32_t cnt_above = 0;
+  uint64_t target = 0, mass_above = 0;
   int lin = 0, prefix = 0, tail = 0, shift = 0, n_tau = 0, ngt = 0, neq = 0, tiepos = -1, ncand = 0;
-  float lscale = 4.f;  // bins of level `lin`: floor(u * lscale)
+  float ulo = 0.f, uhi = 0.f, dscale = 1.f;  // current bracket of u, and 32^lin
   uint32_t kbase = 0, tau_key = 0;
   uint64_t kend = 0;
+  const float wmul = -0.25f * 1.4426950408889634f;  // weight 2^(u * wmul) = exp(-(m - v) / 4)
   uint32_t* mrow = (A.mask && is_row && t < A.T) ? A.mask + ((int64_t)bh * A.T + t) * A.mask_words : nullptr;
 
   uint32_t g = 0;  // global tile counter across sweeps (drives every ring phase)
@@ -144,12 +154,16 @@ topp_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
     const int more = __syncthreads_or(is_row && level != kLvDone);
     const int abort = __syncthreads_or(!alive);
     if (!more || abort || ntiles == 0) break;
+    if (is_row && level == kLvLin && lin == 0) dscale = 1.f;
     if (is_row && (level == kLvLin || level == kLvKey))
       for (int i = 0; i < kPfBins; ++i) {
         S.hist[i][row] = 0;
         S.hcnt[i][row] = 0;
       }
-    if (is_row) ncand = 0;
+    if (is_row) {
+      ncand = 0;
+      if (level == kLvCollect) ngt = 0;
+    }
 
     if (warp == 4) {
       // ---------------- TMA producer ----------------
@@ -192,7 +206,7 @@ topp_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
         const int key0 = i * kPfKeys;
         uint64_t mbits = 0ull;
 #pragma unroll 1
-        for (int half = 0; half < 2; ++half) {
+        for (int half = 0; half < 2; ++half) {  // two chunks of 32 columns
           uint32_t v[32];
           tmem_ld32(taddr + half * 32, v);
           tmem_ld_wait();
@@ -230,51 +244,57 @@ topp_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
                 mbits |= (uint64_t)sel << (half * 32 + j);
               }
             }
-          } else if (level == kLvLin) {
+          } else if (level == kLvLin && lin == 0) {
+            // every key lands in a bin; Z is the sum of the bins afterwards
             const int nvc = nv < 32 ? nv : 32;
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
               if (j < nvc) {
-                const float sv = __fadd_rn(__fmul_rn(__uint_as_float(v[j]), 0.25f), 0.0f);
-                const float t = __fmul_rn(__fsub_rn(mh, sv), lscale);
-                const int ti = lin == 0 ? (t >= 31.f ? 31 : (int)t) : (t >= 2.0e9f ? -1 : (int)t);
-                if ((ti >> 5) == prefix && ti >= 0) {
-                  const int d = ti & 31;
-                  const uint64_t w = pf_weight(sv, mh, A.two_pow_frac);
-                  Z += w;
-                  S.hist[d][row] += w;
-                  S.hcnt[d][row] += 1u;
+                const float u = __fsub_rn(mh, __uint_as_float(v[j]));
+                const int d = u >= 31.f ? 31 : (u > 0.f ? (int)u : 0);  // also 0 for a NaN input
+                S.hist[d][row] += pf_weight_u(u, wmul, A.two_pow_frac);
+              }
+            }
+          } else if (level == kLvLin || level == kLvCollect) {
+            // keys inside the bracket [ulo, uhi) of u (two compares each); most chunks have none
+            uint32_t in = 0u;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const float u = __fsub_rn(mh, __uint_as_float(v[j]));
+              const bool ok = j < nv;
+              in |= (uint32_t)(ok && u >= ulo && u < uhi) << j;
+              if (level == kLvCollect) ngt += ok && u < ulo;  // keys above the bracket
+            }
+            if (in) {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) {
+                if ((in >> j) & 1u) {
+                  const float u = __fsub_rn(mh, __uint_as_float(v[j]));
+                  if (level == kLvLin) {
+                    const int d = (int)__fmul_rn(u, dscale) - 32 * prefix;
+                    S.hist[d][row] += pf_weight_u(u, wmul, A.two_pow_frac);
+                    const uint16_t cc = S.hcnt[d][row];
+                    S.hcnt[d][row] = cc == 0xFFFFu ? cc : (uint16_t)(cc + 1u);
+                  } else if (ncand < kPfBins) {
+                    const float sv = __fadd_rn(__fmul_rn(__uint_as_float(v[j]), 0.25f), 0.0f);
+                    S.hist[ncand][row] = ((uint64_t)(uint32_t)(kb + j) << 32) | __float_as_uint(sv);
+                    ++ncand;
+                  }
                 }
               }
             }
-          } else if (level == kLvCollect) {
+          } else {  // KEY fallback: exact digits of the score key inside the bracket
             const int nvc = nv < 32 ? nv : 32;
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
               if (j < nvc) {
+                const float u = __fsub_rn(mh, __uint_as_float(v[j]));
+                const bool inb = tail ? u >= 31.f : (u >= ulo && u < uhi);
                 const float sv = __fadd_rn(__fmul_rn(__uint_as_float(v[j]), 0.25f), 0.0f);
-                const float t = __fmul_rn(__fsub_rn(mh, sv), lscale);
-                const int ti = lin == 0 ? (t >= 31.f ? 31 : (int)t) : (t >= 2.0e9f ? -1 : (int)t);
-                if (ti == prefix && ncand < kPfBins) {
-                  S.hist[ncand][row] = ((uint64_t)(uint32_t)(kb + j) << 32) | __float_as_uint(sv);
-                  ++ncand;
-                }
-              }
-            }
-          } else {  // KEY fallback
-            const int nvc = nv < 32 ? nv : 32;
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              if (j < nvc) {
-                const float sv = __fadd_rn(__fmul_rn(__uint_as_float(v[j]), 0.25f), 0.0f);
-                const float t = __fmul_rn(__fsub_rn(mh, sv), lscale);
-                const int ti = tail ? 31 : (t >= 2.0e9f ? -1 : (int)t);
-                const int tl = tail ? (__fmul_rn(__fsub_rn(mh, sv), 4.f) >= 31.f ? 31 : -1) : ti;
                 const uint32_t k = score_key(sv);
-                if (tl == prefix && k >= kbase && (uint64_t)k < kend) {
+                if (inb && k >= kbase && (uint64_t)k < kend) {
                   const int d = (int)((k - kbase) >> shift);
-                  S.hist[d][row] += pf_weight(sv, mh, A.two_pow_frac);
-                  S.hcnt[d][row] += 1u;
+                  S.hist[d][row] += pf_weight_u(u, wmul, A.two_pow_frac);
                 }
               }
             }
@@ -289,11 +309,9 @@ topp_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
       // ---- end of sweep: advance this row's bracket ----
       if (is_row && level != kLvDone && alive) {
         if (level == kLvMax) {
-          m = __fadd_rn(__fmul_rn(m, 0.25f), 0.0f);  // same rounding as every score
-          level = kLvLin;
+          level = kLvLin;  // m is the raw maximum
           lin = 0;
           prefix = 0;
-          lscale = 4.f;
         } else if (level == kLvTie) {
           if (mrow)  // words past the block's last tile
             for (int64_t w = 2 * (int64_t)ntiles; w < (A.N + 31) / 32; ++w) mrow[w] = 0u;
@@ -322,7 +340,8 @@ topp_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
           uint64_t cum = 0;
           int taken = ncand;
           for (int a = 0; a < ncand; ++a) {
-            cum += pf_weight(__uint_as_float((uint32_t)S.hist[a][row]), mh, A.two_pow_frac);
+            const float sa = __uint_as_float((uint32_t)S.hist[a][row]);
+            cum += pf_weight_u(__fsub_rn(mh, __fmul_rn(sa, 4.f)), wmul, A.two_pow_frac);
             if (cum >= need) {
               taken = a + 1;
               break;
@@ -333,7 +352,7 @@ topp_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
           tau_key = score_key(__uint_as_float((uint32_t)last));
           n_tau = 0;
           for (int a = 0; a < taken; ++a) n_tau += score_key(__uint_as_float((uint32_t)S.hist[a][row])) == tau_key;
-          const int cnt = (int)cnt_above + taken;
+          const int cnt = ngt + taken;
           if (mrow) {  // the selection mask needs one more sweep
             ngt = 0;
             neq = 0;
@@ -348,13 +367,14 @@ topp_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
           }
         } else {  // LIN or KEY: find the cut bin
           if (level == kLvLin && lin == 0) {
+            uint64_t Z = 0;
+            for (int i = 0; i < kPfBins; ++i) Z += S.hist[i][row];
             const double tt = ceil((double)A.p * (double)Z);
             uint64_t tg = tt >= (double)Z ? Z : (uint64_t)tt;
             target = tg < 1 ? 1 : tg;
           }
           const uint64_t need = target - mass_above;
           uint64_t cum = 0;
-          uint32_t cumc = 0;
           int cut = 0;
           for (int r = 0; r < kPfBins; ++r) {
             const int bin = level == kLvKey ? kPfBins - 1 - r : r;
@@ -364,35 +384,34 @@ topp_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
               break;
             }
             cum += hv;
-            cumc += S.hcnt[bin][row];
           }
           mass_above += cum;
-          cnt_above += cumc;
-          const uint32_t in_bin = S.hcnt[cut][row];
           if (level == kLvLin) {
             if (lin == 0 && cut == 31) {
-              // tail bin (u >= 7.75): exact digits over the keys up to m - 7.75
+              // tail bin (u >= 31, i.e. s <= max s - 7.75): exact digits over its keys
               tail = 1;
-              prefix = 31;
-              const float hi_s = mh - 7.75f;
-              const float mg = 1e-5f * (fabsf(mh) + 8.f) + 1e-30f;
+              const float hi_s = __fmul_rn(__fsub_rn(mh, 31.f), 0.25f);
+              const float mg = 1e-5f * (fabsf(hi_s) + 8.f) + 1e-30f;
               kbase = 0u;
               kend = (uint64_t)score_key(__fadd_rn(hi_s + mg, 0.0f)) + 1;
               shift = 0;
               while (((kend - kbase - 1) >> shift) >= (uint64_t)kPfBins) ++shift;
               level = kLvKey;
             } else {
-              prefix = (prefix << 5) | cut;
+              const uint32_t in_bin = lin == 0 ? 0xFFFFu : S.hcnt[cut][row];  // level 0 keeps no counts
+              prefix = lin == 0 ? cut : 32 * prefix + cut;  // full bin index at level `lin`
+              ulo = (float)prefix / dscale;                  // exact: dscale is a power of two
+              uhi = (float)(prefix + 1) / dscale;
               if (in_bin <= (uint32_t)kPfBins) {
-                level = kLvCollect;  // same scale: keys whose level-`lin` bin is `prefix`
+                level = kLvCollect;
               } else if (lin < 3) {
                 ++lin;
-                lscale *= 32.f;
+                dscale *= 32.f;
               } else {
-                // still too many keys: exact digits inside the bracket of this bin
-                const float hi_s = mh - (float)prefix / lscale;
-                const float lo_s = mh - (float)(prefix + 1) / lscale;
-                const float mg = 1e-5f * (fabsf(mh) + (float)(prefix + 1) / lscale) + 1e-30f;
+                // still too many keys: exact digits inside this bracket of u
+                const float hi_s = __fmul_rn(__fsub_rn(mh, ulo), 0.25f);
+                const float lo_s = __fmul_rn(__fsub_rn(mh, uhi), 0.25f);
+                const float mg = 1e-5f * (fabsf(hi_s) + fabsf(lo_s) + uhi) + 1e-30f;
                 kbase = score_key(__fadd_rn(lo_s - mg, 0.0f));
                 kend = (uint64_t)score_key(__fadd_rn(hi_s + mg, 0.0f)) + 1;
                 shift = 0;
@@ -406,7 +425,8 @@ topp_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
             kend = e < kend ? e : kend;
             if (shift == 0) {
               tau_key = kbase;
-              const uint64_t w_tau = pf_weight(key_score(tau_key), mh, A.two_pow_frac);
+              const float st = key_score(tau_key);
+              const uint64_t w_tau = pf_weight_u(__fsub_rn(mh, __fmul_rn(st, 4.f)), wmul, A.two_pow_frac);
               const uint64_t rem = target - mass_above;
               uint64_t nt = w_tau ? (rem + w_tau - 1) / w_tau : 1;
               n_tau = (int)(nt < 1 ? 1 : nt);
@@ -514,9 +534,9 @@ cudaError_t launch_topp_prefill(const LaunchToppPrefill& a, cudaStream_t stream)
   CUtensorMap qmap, kmap;
   if (!make_idx_map(&qmap, a.q_idx, a.B, a.Hq, a.T, kPfRows)) return cudaErrorInvalidValue;
   if (!make_idx_map(&kmap, a.k_idx, a.B, a.Hk, a.N, kPfKeys)) return cudaErrorInvalidValue;
-  const size_t smem = sizeof(PfSmem) + 1024;
+  const size_t smem = sizeof(PfSmem) + 256;
   cudaFuncSetAttribute(topp_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  const dim3 grid((unsigned)((a.T + kPfRows - 1) / kPfRows), (unsigned)(a.B * a.Hq));
+  const dim3 grid((unsigned)(((a.T + kPfRows - 1) / kPfRows) * a.B * a.Hq));
   topp_prefill_kernel<<<grid, kPfThreads, smem, stream>>>(qmap, kmap, A);
   return cudaGetLastError();
 }
