@@ -203,6 +203,8 @@ __device__ void finish_split(const AttnArgs& A, int grp, int split, const float*
 // ---- bf16 tensor-core variant ---------------------------------------------
 __global__ void __launch_bounds__(kAttnThreads)
 attn_decode_bf16_kernel(AttnArgs A) {
+  pdl_wait();
+  pdl_release();
   extern __shared__ __align__(128) unsigned char smem[];
   const int split = blockIdx.x, grp = blockIdx.y;
   const int b = grp / A.Hk, kvh = grp % A.Hk;
@@ -437,6 +439,8 @@ attn_decode_bf16_kernel(AttnArgs A) {
 // ---- fp32 CUDA-core variant -----------------------------------------------
 __global__ void __launch_bounds__(kAttnThreads)
 attn_decode_f32_kernel(AttnArgs A) {
+  pdl_wait();
+  pdl_release();
   __shared__ float wm[4][kMaxGroup], wl[4][kMaxGroup];
   __shared__ __align__(16) float wo[4][kMaxGroup][kHeadDim];
   __shared__ __align__(16) float part_o[kMaxGroup * kHeadDim];
@@ -611,11 +615,9 @@ cudaError_t launch_attn_decode(const LaunchAttnDecode& a, cudaStream_t stream) {
   if (a.bf16) {
     const size_t smem = (size_t)kStages * 2 * kTileBytes + (size_t)(kMaxGroup + 1) * kMaxChunkWords * 4;
     cudaFuncSetAttribute(attn_decode_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    attn_decode_bf16_kernel<<<grid, kAttnThreads, smem, stream>>>(A);
-  } else {
-    attn_decode_f32_kernel<<<grid, kAttnThreads, 0, stream>>>(A);
+    return launch_pdl(attn_decode_bf16_kernel, grid, dim3(kAttnThreads), smem, stream, 1, A);
   }
-  return cudaGetLastError();
+  return launch_pdl(attn_decode_f32_kernel, grid, dim3(kAttnThreads), 0, stream, 1, A);
 }
 
 }  // namespace rtp

@@ -35,6 +35,10 @@ constexpr int kApRowBytes = kHeadDim * 2;                 // 256 B
 constexpr int kApTileBytes = kApKeys * kApRowBytes;       // 16 KB per K or V tile
 constexpr int kApIdxTileBytes = kApKeys * kIdxDim * 2;    // 2 KB
 constexpr float kLog2eF = 1.4426950408889634f;
+// The MMA accumulators are folded into a round-to-nearest fp32 sum every
+// kApFlush tiles: tensor-core accumulation does not round to nearest, so one
+// accumulator carried over a million keys would drift by ~1e-3 relative.
+constexpr int kApFlush = 16;
 
 struct ApSmem {
   alignas(1024) uint8_t qidx[kApRows * kIdxDim * 2];      // 4 KB (sparse form)
@@ -42,6 +46,7 @@ struct ApSmem {
   alignas(128) uint8_t q[kApRows * kApRowBytes];          // 32 KB
   alignas(128) uint8_t kv[2][2][kApTileBytes];            // [stage][K,V] 64 KB
   uint32_t bits[2][kApRows][2];                           // admission bitmaps, double-buffered
+  float otot[kApMathWarps][64][32];                       // round-to-nearest running output sums
   uint64_t qidx_full;
   uint64_t kidx_full[2];
   uint64_t kidx_empty[2];
@@ -224,6 +229,21 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
 #pragma unroll
     for (int nt = 0; nt < 16; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
     float ma = -INFINITY, mb = -INFINITY, la = 0.f, lb = 0.f;
+    float* ot = &S.otot[warp][0][0];  // this thread's 64 sums at ot[e * 32 + lane]
+#pragma unroll
+    for (int e = 0; e < 64; ++e) ot[e * 32 + lane] = 0.f;
+    float ca = 1.f, cb = 1.f;  // rescale factors applied to o since the last fold
+    auto fold = [&]() {
+#pragma unroll
+      for (int nt = 0; nt < 16; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          float& acc = ot[(nt * 4 + e) * 32 + lane];
+          acc = __fmaf_rn(acc, e < 2 ? ca : cb, o[nt][e]);
+          o[nt][e] = 0.f;
+        }
+      ca = cb = 1.f;
+    };
 
     for (int i = 0; i < ntiles; ++i) {
       const int st = i & 1;
@@ -316,6 +336,8 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
         mb = mnb;
         la *= ala;
         lb *= alb;
+        ca *= ala;
+        cb *= alb;
 #pragma unroll
         for (int nt = 0; nt < 16; ++nt) {
           o[nt][0] *= ala;
@@ -356,9 +378,15 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
           }
         }
       }
+      if ((i % kApFlush) == kApFlush - 1) fold();
       named_sync(1, kApMathWarps * 32);  // the stage is free for the prefetch two tiles ahead
     }
     cp_wait_all();
+    fold();
+#pragma unroll
+    for (int nt = 0; nt < 16; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o[nt][e] = ot[(nt * 4 + e) * 32 + lane];
     // ---- normalise and store ----
     la += __shfl_xor_sync(0xffffffffu, la, 1);
     la += __shfl_xor_sync(0xffffffffu, la, 2);

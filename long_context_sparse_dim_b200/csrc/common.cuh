@@ -127,6 +127,14 @@ RTP_DEVICE uint64_t fixed_weight(float s, float m, float two_pow_frac) {
   return __float2ull_rn(__fmul_rn(e, two_pow_frac));
 }
 
+// ---- programmatic dependent launch -----------------------------------------
+// A kernel launched with programmatic stream serialization may start while the
+// previous kernel of its stream is still finishing; pdl_wait() blocks until that
+// kernel has completed and its writes are visible (a no-op otherwise), and
+// pdl_release() lets the next kernel of the stream be launched early.
+RTP_DEVICE void pdl_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+RTP_DEVICE void pdl_release() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
+
 // ---- warp helpers ----------------------------------------------------------
 RTP_DEVICE float warp_max(float v) {
 #pragma unroll

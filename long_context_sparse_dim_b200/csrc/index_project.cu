@@ -62,6 +62,8 @@ template <typename Tin, typename Tout>
 __global__ void __launch_bounds__(kProjThreads)
 index_project_kernel(View4 x, const float* __restrict__ P, int H, int heads_per_p, int N, int64_t rows,
                      MutView4 out) {
+  pdl_wait();
+  pdl_release();
   const int lane = threadIdx.x & 31;
   const int64_t warp0 = ((int64_t)blockIdx.x * kProjThreads + threadIdx.x) >> 5;
   const int64_t nwarps = ((int64_t)gridDim.x * kProjThreads) >> 5;
@@ -115,15 +117,17 @@ cudaError_t launch_index_project(const LaunchIndexProject& a, cudaStream_t strea
   const dim3 grid((unsigned)blocks);
   const int hpp = (int)(a.H / a.HP);
   const int H = (int)a.H, N = (int)a.N;
+  const dim3 block(kProjThreads);
   if (a.in_bf16 && a.out_bf16)
-    index_project_kernel<__nv_bfloat16, __nv_bfloat16><<<grid, kProjThreads, 0, stream>>>(a.x, a.P, H, hpp, N, rows, a.out);
-  else if (a.in_bf16)
-    index_project_kernel<__nv_bfloat16, float><<<grid, kProjThreads, 0, stream>>>(a.x, a.P, H, hpp, N, rows, a.out);
-  else if (a.out_bf16)
-    index_project_kernel<float, __nv_bfloat16><<<grid, kProjThreads, 0, stream>>>(a.x, a.P, H, hpp, N, rows, a.out);
-  else
-    index_project_kernel<float, float><<<grid, kProjThreads, 0, stream>>>(a.x, a.P, H, hpp, N, rows, a.out);
-  return cudaGetLastError();
+    return launch_pdl(index_project_kernel<__nv_bfloat16, __nv_bfloat16>, grid, block, 0, stream, 1, a.x, a.P, H, hpp,
+                      N, rows, a.out);
+  if (a.in_bf16)
+    return launch_pdl(index_project_kernel<__nv_bfloat16, float>, grid, block, 0, stream, 1, a.x, a.P, H, hpp, N, rows,
+                      a.out);
+  if (a.out_bf16)
+    return launch_pdl(index_project_kernel<float, __nv_bfloat16>, grid, block, 0, stream, 1, a.x, a.P, H, hpp, N, rows,
+                      a.out);
+  return launch_pdl(index_project_kernel<float, float>, grid, block, 0, stream, 1, a.x, a.P, H, hpp, N, rows, a.out);
 }
 
 }  // namespace rtp

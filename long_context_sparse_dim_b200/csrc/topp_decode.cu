@@ -97,6 +97,8 @@ topp_query_kernel(View4 qv, View4 kv, const int32_t* __restrict__ lens, int Hq, 
                    int n_chunk, float p, float two_pow_frac, uint32_t* __restrict__ tau_bits,
                    int32_t* __restrict__ tiepos, int32_t* __restrict__ count,
                    uint32_t* __restrict__ mask, int64_t mask_words) {
+  pdl_wait();
+  pdl_release();
   cg::cluster_group cluster = cg::this_cluster();
   const int C = (int)cluster.num_blocks();
   const int rank = (int)cluster.block_rank();
@@ -377,23 +379,9 @@ static int sm_count() {
 
 template <typename K, typename... Args>
 static cudaError_t launch_cluster(K kern, int grid, int C, size_t smem, cudaStream_t stream, Args... args) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)grid);
-  cfg.blockDim = dim3(kSelThreads);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = (unsigned)C;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (C > 8) cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, args...);
-  if (e != cudaSuccess) return e;
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3((unsigned)grid), dim3(kSelThreads), smem, stream, (unsigned)C, args...);
 }
 
 cudaError_t launch_topp_decode(const LaunchToppDecode& a, cudaStream_t stream) {

@@ -1,0 +1,77 @@
+"""GPU parity at the full workload sizes, in the launch configuration bench.py
+times: decode of 4 sequences of 131072 keys (three top-p masses), causal
+prefill of 32768 tokens, and the last 8192 tokens against a 1,048,576-token
+cache.  Prefill checks a seeded sample of query tokens (always the first and
+the last) over every head; decode checks every query."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from long_context_sparse_dim_b200 import rtp
+from long_context_sparse_dim_b200 import workloads as wl
+
+from gpu_check import compare_outputs, compare_selection, make_oracle, upload
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("p", [0.9, 0.95, 0.99])
+def test_decode_b4_n131072_top_p_sweep(p):
+    from long_context_sparse_dim_b200.layer import DecodeLayer
+    w = wl.DECODE_B4_N128K.replace(p=p)
+    inst = wl.generate(w)
+    q, k, v, P, lens = upload(inst)
+    layer = DecodeLayer(q, k, v, P, R=w.R, W=w.W, p=p)
+    layer.build_index()
+    o = layer.step().float().cpu().numpy()
+    torch.cuda.synchronize()
+    L = make_oracle(inst, p=p)
+    res = L.run()
+    compare_outputs(o, res, w.name)
+    mask = layer.sel.mask.cpu().numpy().view(np.uint32)
+    count = layer.sel.count.cpu().numpy()
+    Hr = w.R * w.G
+    for b in range(w.B):
+        for h in range(Hr):
+            compare_selection(res[(b, h, 0)], mask[b * Hr + h], w.N, int(count[b * Hr + h]), f"b{b} h{h}")
+    hit, tot = oracle.needle_recall(res, inst.needles)
+    assert hit / tot >= 0.9
+
+
+def _prefill_full(w, n_sample, seed):
+    from long_context_sparse_dim_b200.layer import PrefillLayer
+    inst = wl.generate(w)
+    q, k, v, P, lens = upload(inst)
+    layer = PrefillLayer(q, k, v, P, R=w.R, W=w.W, p=w.p, with_mask=True)
+    o = layer.step()
+    torch.cuda.synchronize()
+    assert rtp.poll_device_error() == 0
+    rng = np.random.default_rng(seed)
+    toks = sorted(set([0, w.T - 1] + rng.choice(w.T, size=n_sample, replace=False).tolist()))
+    Hr = w.R * w.G
+    o_s = o[:, :, toks].float().cpu().numpy()
+    rows = [(h * w.T + t) for h in range(Hr) for t in toks]
+    mask = layer.sel.mask[rows].cpu().numpy().view(np.uint32)
+    count = layer.sel.count[rows].cpu().numpy()
+    del layer, o
+    torch.cuda.empty_cache()
+    L = make_oracle(inst)
+    res = L.run([(0, h, t) for h in range(w.Hq) for t in toks])
+    res_s = {(0, h, i): res[(0, h, t)] for h in range(w.Hq) for i, t in enumerate(toks)}
+    compare_outputs(o_s, res_s, w.name)
+    for r_i, (h, t) in enumerate((h, t) for h in range(Hr) for t in toks):
+        n = L.pos(0, t) + 1
+        compare_selection(res[(0, h, t)], mask[r_i], n, int(count[r_i]), f"{w.name} h{h} t{t}")
+    needles = [n for n in inst.needles if n[3] in set(toks)]
+    if needles:
+        hit, tot = oracle.needle_recall(res, needles)
+        assert hit / tot >= 0.9
+
+
+def test_prefill_t32768_causal_sampled():
+    _prefill_full(wl.PREFILL_N32K, 30, 0)
+
+
+def test_prefill_chunk_t8192_n1048576_sampled():
+    _prefill_full(wl.PREFILL_CHUNK_1M, 6, 1)
