@@ -41,6 +41,8 @@ constexpr int kBins = 256;
 constexpr int kMaxCluster = 16;
 constexpr int kMaxKeysPerCta = 32768;  // scores of one CTA held in shared memory (128 KB)
 constexpr float kLinBinsPerNat = 16.f; // pass 0 bin width 1/16 nat
+constexpr int kListCap = kSelWarps * kBins;  // members of the cut bin one CTA can list
+constexpr int kCandCap = kSelThreads;        // candidates rank 0 orders (one per thread)
 static_assert(kSelThreads == kBins, "one thread per histogram bin");
 
 struct SelSmem {
@@ -57,6 +59,22 @@ struct SelSmem {
   uint32_t wcnt2[kSelWarps];
   int cut_bin;
   uint64_t cut_above;
+  // candidate path (pass-0 cut bin -> 256 sub-bins -> candidates at rank 0)
+  uint32_t l1lo[kBins];              // sub-bin masses of this CTA (lo/hi words)
+  uint32_t l1hi[kBins];
+  uint32_t l1cnt[kBins];             // sub-bin key counts of this CTA
+  uint64_t h1[kBins];                // sub-bin masses of this CTA as 64-bit values
+  uint32_t nlist, nabove, novf;      // members listed, keys above the cut bin, list overflow
+  uint32_t tot_above, tot_ovf, cut_cnt, cut_cnt_above;
+  uint32_t ncand;                    // rank 0: candidates received
+  float cand_s[kCandCap];            // rank 0: candidates (score, position) in arrival order
+  int32_t cand_p[kCandCap];
+  float sort_s[kCandCap];            // rank 0: candidates in (score desc, position asc) order
+  int32_t sort_p[kCandCap];
+  int bc_t;
+  float bc_tau;                      // the cut, written into every CTA by rank 0
+  int32_t bc_tiepos;
+  uint32_t bc_count;
 };
 
 // Exact 64-bit add into a (lo, hi) pair of 32-bit shared-memory words: native
@@ -91,6 +109,180 @@ RTP_DEVICE int lin_bin(float s, float m) {
   return t >= (float)(kBins - 1) ? kBins - 1 : (int)t;
 }
 
+// Sub-bin of a score inside pass-0 bin `lin` (lin < 255): floor((m - s) * 4096)
+// - 256 lin.  (m - s) is the same rounded value lin_bin scales by 16, and both
+// scalings are exact, so the sub-bins of bin lin are exactly its members.
+RTP_DEVICE int sub_bin(float s, float m, int lin) {
+  const float t = __fmul_rn(__fsub_rn(m, s), kLinBinsPerNat * (float)kBins);
+  const int d = (int)t - lin * kBins;
+  return d < 0 ? 0 : (d > kBins - 1 ? kBins - 1 : d);
+}
+
+RTP_DEVICE uint32_t warp_sum_u32(uint32_t v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Inclusive prefix sum over the block's threads in thread order; `wsum` holds
+// one word per warp.  Ends with a barrier, so `wsum` may be reused at once.
+RTP_DEVICE uint64_t block_scan_u64(uint64_t v, uint64_t* wsum, uint64_t& excl) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint64_t incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint64_t t = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  if (lane == 31) wsum[warp] = incl;
+  __syncthreads();
+  uint64_t off = 0;
+  for (int w = 0; w < warp; ++w) off += wsum[w];
+  __syncthreads();
+  incl += off;
+  excl = incl - v;
+  return incl;
+}
+
+// Candidate path for a cut inside pass-0 bin `lin` (not the tail bin), `need`
+// = the mass still to take inside that bin.  Each CTA lists the members of bin
+// lin (and counts its keys in higher bins), histograms them into 256 sub-bins
+// 1/4096 nat wide (mass and count), and every CTA finds the same cut sub-bin
+// from the cluster-wide sums.  If it holds at most kCandCap keys, they go to
+// rank 0, which orders them by (score desc, position asc), walks their weights
+// to the cut and writes (tau, tiepos, count) into every CTA.  Returns the same
+// value in every CTA of the cluster; false (a CTA's list overflowed, or the cut
+// sub-bin is too full) leaves the key-window refinement to find the cut.
+RTP_DEVICE bool collect_cut(SelSmem& S, cg::cluster_group& cluster, const float* scores, int nloc, int c0,
+                            float m, float two_pow_frac, int lin, uint64_t need) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int C = (int)cluster.num_blocks();
+  const int rank = (int)cluster.block_rank();
+  float* list_s = reinterpret_cast<float*>(&S.whlo[0][0]);
+  int32_t* list_i = reinterpret_cast<int32_t*>(&S.whhi[0][0]);
+  static_assert(sizeof(S.whlo) >= kListCap * sizeof(float), "list fits in the per-warp histograms");
+
+  // members of bin lin -> local list (warp-aggregated appends)
+  uint32_t nab = 0;
+  for (int base = 0; base < nloc; base += kSelThreads) {
+    const int i = base + tid;
+    const bool valid = i < nloc;
+    const float sc = valid ? scores[i] : 0.f;
+    const int d = valid ? lin_bin(sc, m) : kBins;
+    nab += d < lin;
+    const bool mem = d == lin;
+    const uint32_t bal = __ballot_sync(0xffffffffu, mem);
+    if (bal) {
+      uint32_t b0 = 0;
+      if (lane == 0) b0 = atomicAdd(&S.nlist, (uint32_t)__popc(bal));
+      b0 = __shfl_sync(0xffffffffu, b0, 0);
+      if (mem) {
+        const uint32_t slot = b0 + (uint32_t)__popc(bal & ((1u << lane) - 1u));
+        if (slot < (uint32_t)kListCap) {
+          list_s[slot] = sc;
+          list_i[slot] = i;
+        }
+      }
+    }
+  }
+  nab = warp_sum_u32(nab);
+  if (lane == 0) atomicAdd(&S.nabove, nab);
+  __syncthreads();
+  const int nl = min((int)S.nlist, kListCap);
+  for (int j = tid; j < nl; j += kSelThreads) {
+    const float sc = list_s[j];
+    const int sb = sub_bin(sc, m, lin);
+    add_u64_pair(&S.l1lo[sb], &S.l1hi[sb], sel_weight(sc, m, two_pow_frac));
+    atomicAdd(&S.l1cnt[sb], 1u);
+  }
+  __syncthreads();
+  S.h1[tid] = pair_value(S.l1lo[tid], S.l1hi[tid]);
+  if (tid == 0) S.novf = S.nlist > (uint32_t)kListCap ? 1u : 0u;
+  cluster.sync();  // every CTA's sub-bin histogram is complete
+
+  // cluster-wide sub-bin masses and counts, identical in every CTA
+  uint64_t a = 0, c = 0;
+#pragma unroll
+  for (int r = 0; r < kMaxCluster; ++r)
+    if (r < C) {
+      a += cluster.map_shared_rank(S.h1, r)[tid];
+      c += cluster.map_shared_rank(S.l1cnt, r)[tid];
+    }
+  if (warp == 0) {
+    uint32_t na = 0, ov = 0;
+    if (lane < C) {
+      na = *cluster.map_shared_rank(&S.nabove, lane);
+      ov = *cluster.map_shared_rank(&S.novf, lane);
+    }
+    na = warp_sum_u32(na);
+    ov = warp_sum_u32(ov);
+    if (lane == 0) {
+      S.tot_above = na;
+      S.tot_ovf = ov;
+      S.cut_bin = -1;
+    }
+  }
+  uint64_t em, ec;
+  const uint64_t im = block_scan_u64(a, S.wsum, em);  // sub-bin 0 holds the highest scores
+  block_scan_u64(c, S.wsum, ec);
+  if (em < need && need <= im) {
+    S.cut_bin = tid;
+    S.cut_above = em;
+    S.cut_cnt_above = (uint32_t)ec;
+    S.cut_cnt = (uint32_t)c;
+  }
+  __syncthreads();
+  const int sb = S.cut_bin;
+  if (S.tot_ovf != 0 || sb < 0 || S.cut_cnt > (uint32_t)kCandCap) return false;
+
+  // the cut sub-bin's keys -> rank 0
+  {
+    uint32_t* nc = cluster.map_shared_rank(&S.ncand, 0);
+    float* cs = cluster.map_shared_rank(S.cand_s, 0);
+    int32_t* cp = cluster.map_shared_rank(S.cand_p, 0);
+    for (int j = tid; j < nl; j += kSelThreads) {
+      const float sc = list_s[j];
+      if (sub_bin(sc, m, lin) == sb) {
+        const uint32_t slot = atomicAdd(nc, 1u);
+        cs[slot] = sc;
+        cp[slot] = c0 + list_i[j];
+      }
+    }
+  }
+  cluster.sync();  // rank 0 holds all candidates
+
+  if (rank == 0) {
+    const int n = (int)S.ncand;  // == S.cut_cnt <= kCandCap
+    if (tid < n) {
+      const uint32_t kt = score_key(S.cand_s[tid]);
+      const int pt = S.cand_p[tid];
+      int rk = 0;
+      for (int j = 0; j < n; ++j) {
+        const uint32_t kj = score_key(S.cand_s[j]);
+        rk += (kj > kt || (kj == kt && S.cand_p[j] < pt)) ? 1 : 0;
+      }
+      S.sort_s[rk] = S.cand_s[tid];
+      S.sort_p[rk] = pt;
+    }
+    if (tid == 0) S.bc_t = n - 1;
+    __syncthreads();
+    const uint64_t w = tid < n ? sel_weight(S.sort_s[tid], m, two_pow_frac) : 0;
+    uint64_t ew;
+    const uint64_t iw = block_scan_u64(w, S.wsum, ew);
+    const uint64_t need1 = need - S.cut_above;  // >= 1, <= the sub-bin's mass
+    if (tid < n && ew < need1 && need1 <= iw) S.bc_t = tid;
+    __syncthreads();
+    if (tid < C) {
+      const int t = S.bc_t;
+      *cluster.map_shared_rank(&S.bc_tau, tid) = S.sort_s[t];
+      *cluster.map_shared_rank(&S.bc_tiepos, tid) = S.sort_p[t];
+      *cluster.map_shared_rank(&S.bc_count, tid) = S.tot_above + S.cut_cnt_above + (uint32_t)t + 1u;
+    }
+  }
+  cluster.sync();  // every CTA holds the cut; no distributed access after this
+  return true;
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kSelThreads)
 topp_query_kernel(View4 qv, View4 kv, const int32_t* __restrict__ lens, int Hq, int G, int N,
@@ -109,6 +301,14 @@ topp_query_kernel(View4 qv, View4 kv, const int32_t* __restrict__ lens, int Hq, 
   extern __shared__ __align__(16) unsigned char smem_raw[];
   SelSmem& S = *reinterpret_cast<SelSmem*>(smem_raw);
   float* scores = reinterpret_cast<float*>(smem_raw + sizeof(SelSmem));
+  S.l1lo[tid] = 0;
+  S.l1hi[tid] = 0;
+  S.l1cnt[tid] = 0;
+  if (tid == 0) {
+    S.nlist = 0;
+    S.nabove = 0;
+    S.ncand = 0;
+  }
 
   int n_b = N;
   if (lens) n_b = min(max(lens[b], 0), N);
@@ -180,13 +380,14 @@ topp_query_kernel(View4 qv, View4 kv, const int32_t* __restrict__ lens, int Hq, 
   for (int r = 0; r < kMaxCluster; ++r)
     if (r < C) m = fmaxf(m, *cluster.map_shared_rank(&S.cmax_self, r));
 
-  // ---- bracket narrowing --------------------------------------------------------
-  // pass 0: linear bins; then key-window bins [base, base + 256 << shift).
+  // ---- pass 0: 256 linear bins of (max - s), 1/16 nat wide ---------------------
+  // (then either the candidate path below or key-window refinement passes)
   uint64_t target = 0, mass_above = 0;
   int lin = -1;               // cut bin of pass 0
   uint32_t kbase = 0;         // key window [kbase, kend) of the refinement passes
   uint64_t kend = 0;
   int shift = 0;
+  bool fast = false;
   for (int pass = 0;; ++pass) {
     uint32_t* wlo = S.whlo[warp];
     uint32_t* whi = S.whhi[warp];
@@ -195,16 +396,34 @@ topp_query_kernel(View4 qv, View4 kv, const int32_t* __restrict__ lens, int Hq, 
       whi[i] = 0;
     }
     __syncwarp();
-    for (int i = tid; i < nloc; i += kSelThreads) {
-      const float sc = scores[i];
-      int d = -1;
-      if (pass == 0) {
-        d = lin_bin(sc, m);
-      } else if (lin_bin(sc, m) == lin) {
-        const uint32_t k = score_key(sc);
-        if (k >= kbase && (uint64_t)k < kend) d = (int)((uint64_t)(k - kbase) >> shift);
+    if (pass == 0) {
+      for (int base = 0; base < nloc; base += 4 * kSelThreads) {
+        float sc[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int i = base + u * kSelThreads + tid;
+          sc[u] = i < nloc ? scores[i] : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int i = base + u * kSelThreads + tid;
+          if (i < nloc) {
+            const int d = lin_bin(sc[u], m);
+            add_u64_pair(&wlo[d], &whi[d], sel_weight(sc[u], m, two_pow_frac));
+          }
+        }
       }
-      if (d >= 0) add_u64_pair(&wlo[d], &whi[d], sel_weight(sc, m, two_pow_frac));
+    } else {
+      for (int i = tid; i < nloc; i += kSelThreads) {
+        const float sc = scores[i];
+        if (lin_bin(sc, m) == lin) {
+          const uint32_t k = score_key(sc);
+          if (k >= kbase && (uint64_t)k < kend) {
+            const int d = (int)((uint64_t)(k - kbase) >> shift);
+            add_u64_pair(&wlo[d], &whi[d], sel_weight(sc, m, two_pow_frac));
+          }
+        }
+      }
     }
     __syncthreads();
     uint64_t* hb = S.hist[pass & 1];
@@ -243,19 +462,8 @@ topp_query_kernel(View4 qv, View4 kv, const int32_t* __restrict__ lens, int Hq, 
     // refinement bin 255 is the highest key.  Position r in that order:
     const int bin_of_r = pass == 0 ? tid : (kBins - 1 - tid);
     const uint64_t mine = S.red[bin_of_r];
-    // inclusive prefix of the mass over the descending order (block scan)
-    uint64_t incl = mine;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint64_t v = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += v;
-    }
-    if (lane == 31) S.wsum[warp] = incl;
-    __syncthreads();
-    uint64_t off = 0;
-    for (int w = 0; w < warp; ++w) off += S.wsum[w];
-    incl += off;
-    const uint64_t excl = incl - mine;
+    uint64_t excl;
+    const uint64_t incl = block_scan_u64(mine, S.wsum, excl);
     if (excl < need && need <= incl) {  // exactly one position holds the cut
       S.cut_bin = bin_of_r;
       S.cut_above = excl;
@@ -266,6 +474,10 @@ topp_query_kernel(View4 qv, View4 kv, const int32_t* __restrict__ lens, int Hq, 
     __syncthreads();
     if (pass == 0) {
       lin = cb;
+      if (lin < kBins - 1) {
+        fast = collect_cut(S, cluster, scores, nloc, c0, m, two_pow_frac, lin, target - mass_above);
+        if (fast) break;
+      }
       // key window holding every score of linear bin `lin` (with a margin)
       const float hi_s = m - (float)lin / kLinBinsPerNat;
       const float lo_s = m - (float)(lin + 1) / kLinBinsPerNat;
@@ -284,6 +496,32 @@ topp_query_kernel(View4 qv, View4 kv, const int32_t* __restrict__ lens, int Hq, 
       if (shift == 0) break;            // the bracket is one score value
       shift = shift >= 8 ? shift - 8 : 0;
     }
+  }
+
+  if (fast) {
+    // ---- candidate path: (tau, tiepos) came from rank 0; one mask pass -------
+    const float tau = S.bc_tau;
+    const uint32_t tau_key = score_key(tau);
+    const int tpos = S.bc_tiepos;
+    for (int base = 0; base < n_chunk; base += 4 * kSelThreads) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = base + u * kSelThreads + tid;
+        const bool valid = i < nloc;
+        const uint32_t k = valid ? score_key(scores[i]) : 0u;
+        const bool sel = valid && (k > tau_key || (k == tau_key && c0 + i <= tpos));
+        const uint32_t word = __ballot_sync(0xffffffffu, sel);
+        const int wpos = base + u * kSelThreads + warp * 32;
+        const int w = (c0 + wpos) >> 5;
+        if (lane == 0 && mrow && wpos < n_chunk && w < n_words_total) mrow[w] = word;
+      }
+    }
+    if (rank == 0 && tid == 0) {
+      tau_bits[qrow] = __float_as_uint(tau);
+      tiepos[qrow] = tpos;
+      count[qrow] = (int)S.bc_count;
+    }
+    return;
   }
 
   // ---- counts at tau: keys above and equal, per CTA, then over the cluster ----
