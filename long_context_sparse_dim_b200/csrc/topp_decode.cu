@@ -9,21 +9,27 @@
 // Design (B200): one thread-block CLUSTER per query.  Each CTA of the cluster
 // owns a contiguous slice of the keys, computes their scores once from the
 // projected-key cache (32-byte rows, 16-byte vector loads) and keeps them in
-// shared memory.  The cut is found without sorting, by narrowing a bracket:
-//   pass 0   256 bins linear in (max - s) (1/16 nat wide; the last bin holds
-//            the tail) -- scores spread over many bins, so the per-warp
-//            shared-memory histograms see few same-bin collisions;
-//   pass 1.. 256 bins over the order-preserving uint32 image of the fp32
-//            score (8-bit digits of the offset inside the bracket), only for
-//            keys still inside the bracket, until the bracket is one score
-//            value tau.
-// Every pass accumulates 64-bit fixed-point masses (integer sums, so the
-// result does not depend on thread order).  After each pass every CTA reads
-// all CTAs' 256 bins through distributed shared memory and finds the same cut
-// bin by itself, so a pass costs one cluster barrier.  Ties at tau are
-// resolved by position with a prefix count over the cluster; then every CTA
-// writes its bits of the selection mask.  No global-memory atomics and no spin
-// waits: all synchronisation is the hardware cluster barrier.
+// shared memory.  The cut is found without sorting all keys:
+//   pass 0   a 4096-bin histogram of the weights, bins linear in (max - s),
+//            1/256 nat wide (the last bin holds the tail).  Summing 16 fine
+//            bins gives 256 coarse bins (1/16 nat); every CTA reads all CTAs'
+//            coarse bins through distributed shared memory and finds the same
+//            coarse cut bin, then the fine cut bin from the 16 fine bins
+//            under it;
+//   scan     one pass over the scores writes the mask words (keys above the
+//            fine cut bin) and sends the keys inside it -- the candidates --
+//            to cluster rank 0, with the count of keys above it;
+//   rank 0   splits the candidates into 256 sub-bins (1/65536 nat), orders
+//            the keys of the cut sub-bin by (score desc, position asc), walks
+//            their weights to the cut and sets the candidates' mask bits.
+// If the cut lies in the tail bin or the fine cut bin holds more than 1024
+// keys (heavy ties), narrowing continues in key space instead: 256 bins over
+// the order-preserving uint32 image of the fp32 score (8-bit digits of the
+// offset inside the coarse cut bin) until the bracket is one score value tau;
+// ties at tau are resolved by position with a prefix count over the cluster.
+// Every mass is a 64-bit fixed-point integer sum, so the result does not depend
+// on thread order.  No spin waits: all synchronisation is the hardware cluster
+// barrier.
 #include <cooperative_groups.h>
 
 #include <math.h>
@@ -37,18 +43,37 @@ namespace rtp {
 
 constexpr int kSelThreads = 256;
 constexpr int kSelWarps = kSelThreads / 32;
-constexpr int kBins = 256;
+constexpr int kBins = 256;                  // coarse bins, key-space digits, rank 0's sub-bins
+constexpr int kFinePerBin = 16;
+constexpr int kFineBins = kBins * kFinePerBin;
 constexpr int kMaxCluster = 16;
-constexpr int kMaxKeysPerCta = 32768;  // scores of one CTA held in shared memory (128 KB)
-constexpr float kLinBinsPerNat = 16.f; // pass 0 bin width 1/16 nat
-constexpr int kListCap = kSelWarps * kBins;  // members of the cut bin one CTA can list
-constexpr int kCandCap = kSelThreads;        // candidates rank 0 orders (one per thread)
+constexpr int kMaxKeysPerCta = 32768;       // scores of one CTA held in shared memory (128 KB)
+constexpr float kCoarsePerNat = 16.f;       // coarse bin width 1/16 nat
+constexpr float kFinePerNat = 256.f;        // fine bin width 1/256 nat
+constexpr float kSubPerNat = 65536.f;       // rank 0's sub-bin width 1/65536 nat
+constexpr int kCandCap = 1024;              // candidates rank 0 resolves
 static_assert(kSelThreads == kBins, "one thread per histogram bin");
+static_assert(kCandCap == 4 * kSelThreads, "four candidates per thread in the walk");
 
 struct SelSmem {
-  uint32_t whlo[kSelWarps][kBins];   // per-warp private histograms (64-bit masses as lo/hi words)
-  uint32_t whhi[kSelWarps][kBins];
-  uint64_t hist[2][kBins];           // this CTA's histogram, double-buffered by pass parity
+  union {
+    struct {                                  // pass 0, CTA-wide (64-bit masses as lo/hi words)
+      uint32_t lo[kFineBins];
+      uint32_t hi[kFineBins];
+    } f;
+    struct {                                  // key-space passes, one histogram per warp
+      uint32_t lo[kSelWarps][kBins];
+      uint32_t hi[kSelWarps][kBins];
+    } w;
+    struct {                                  // rank 0, once every candidate has arrived
+      uint32_t lo[kBins], hi[kBins], cnt[kBins];
+      float s[kCandCap];                      // keys of the cut sub-bin, arrival order
+      int32_t p[kCandCap];
+      float ss[kCandCap];                     // the same keys in (score desc, position asc) order
+      int32_t sp[kCandCap];
+    } r;
+  } u;
+  uint64_t hist[2][kBins];           // this CTA's coarse / key-space histogram, double-buffered
   uint64_t red[kBins];               // cluster-wide histogram (each CTA holds a copy)
   uint64_t wsum[kSelWarps];
   uint32_t tcount[kMaxCluster];      // keys equal to tau, per CTA
@@ -59,22 +84,18 @@ struct SelSmem {
   uint32_t wcnt2[kSelWarps];
   int cut_bin;
   uint64_t cut_above;
-  // candidate path (pass-0 cut bin -> 256 sub-bins -> candidates at rank 0)
-  uint32_t l1lo[kBins];              // sub-bin masses of this CTA (lo/hi words)
-  uint32_t l1hi[kBins];
-  uint32_t l1cnt[kBins];             // sub-bin key counts of this CTA
-  uint64_t h1[kBins];                // sub-bin masses of this CTA as 64-bit values
-  uint32_t nlist, nabove, novf;      // members listed, keys above the cut bin, list overflow
-  uint32_t tot_above, tot_ovf, cut_cnt, cut_cnt_above;
-  uint32_t ncand;                    // rank 0: candidates received
-  float cand_s[kCandCap];            // rank 0: candidates (score, position) in arrival order
+  int fine_cut;                      // fine bin holding the cut
+  uint64_t fine_above;               // mass of the fine bins above it
+  // rank 0: filled by every CTA between the fine cut and the candidate barrier
+  uint32_t ncand;                    // candidates sent (may exceed kCandCap)
+  uint32_t nabove;                   // keys above the fine cut bin
+  float cand_s[kCandCap];
   int32_t cand_p[kCandCap];
-  float sort_s[kCandCap];            // rank 0: candidates in (score desc, position asc) order
-  int32_t sort_p[kCandCap];
-  int bc_t;
-  float bc_tau;                      // the cut, written into every CTA by rank 0
-  int32_t bc_tiepos;
-  uint32_t bc_count;
+  // rank 0 scratch
+  int sub_cut;
+  uint64_t sub_above;
+  uint32_t sub_cnt_above, nsort;
+  int t_cut;
 };
 
 // Exact 64-bit add into a (lo, hi) pair of 32-bit shared-memory words: native
@@ -103,18 +124,20 @@ RTP_DEVICE uint64_t sel_weight(float s, float m, float two_pow_frac) {
   return __float2ull_rn(__fmul_rn(e, two_pow_frac));
 }
 
-// pass-0 bin of a score: floor((m - s) * 16), the tail folded into the last bin
-RTP_DEVICE int lin_bin(float s, float m) {
-  const float t = __fmul_rn(__fsub_rn(m, s), kLinBinsPerNat);
+// Bins of u = m - s (u rounded once, by __fsub_rn).  The three scalings by
+// powers of two are exact, so floor(u * 256) >> 4 == floor(u * 16) and
+// floor(u * 65536) >> 8 == floor(u * 256): the bins nest exactly.
+RTP_DEVICE int coarse_bin(float s, float m) {  // tail folded into bin 255
+  const float t = __fmul_rn(__fsub_rn(m, s), kCoarsePerNat);
   return t >= (float)(kBins - 1) ? kBins - 1 : (int)t;
 }
-
-// Sub-bin of a score inside pass-0 bin `lin` (lin < 255): floor((m - s) * 4096)
-// - 256 lin.  (m - s) is the same rounded value lin_bin scales by 16, and both
-// scalings are exact, so the sub-bins of bin lin are exactly its members.
-RTP_DEVICE int sub_bin(float s, float m, int lin) {
-  const float t = __fmul_rn(__fsub_rn(m, s), kLinBinsPerNat * (float)kBins);
-  const int d = (int)t - lin * kBins;
+RTP_DEVICE int fine_bin(float s, float m) {  // tail folded into bin 4095 (coarse 255)
+  const float t = __fmul_rn(__fsub_rn(m, s), kFinePerNat);
+  return t >= (float)(kFineBins - 1) ? kFineBins - 1 : (int)t;
+}
+RTP_DEVICE int sub_bin(float s, float m, int fine) {  // fine < 4080: u < 15.94, t < 2^20
+  const float t = __fmul_rn(__fsub_rn(m, s), kSubPerNat);
+  const int d = (int)t - fine * kBins;
   return d < 0 ? 0 : (d > kBins - 1 ? kBins - 1 : d);
 }
 
@@ -144,143 +167,154 @@ RTP_DEVICE uint64_t block_scan_u64(uint64_t v, uint64_t* wsum, uint64_t& excl) {
   return incl;
 }
 
-// Candidate path for a cut inside pass-0 bin `lin` (not the tail bin), `need`
-// = the mass still to take inside that bin.  Each CTA lists the members of bin
-// lin (and counts its keys in higher bins), histograms them into 256 sub-bins
-// 1/4096 nat wide (mass and count), and every CTA finds the same cut sub-bin
-// from the cluster-wide sums.  If it holds at most kCandCap keys, they go to
-// rank 0, which orders them by (score desc, position asc), walks their weights
-// to the cut and writes (tau, tiepos, count) into every CTA.  Returns the same
-// value in every CTA of the cluster; false (a CTA's list overflowed, or the cut
-// sub-bin is too full) leaves the key-window refinement to find the cut.
-RTP_DEVICE bool collect_cut(SelSmem& S, cg::cluster_group& cluster, const float* scores, int nloc, int c0,
-                            float m, float two_pow_frac, int lin, uint64_t need) {
+// Split cluster barrier: arrive (release) after this CTA's last access to
+// another CTA's shared memory; wait (acquire) before touching shared memory
+// that others may still read.
+RTP_DEVICE void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.aligned;\n" ::: "memory"); }
+RTP_DEVICE void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;\n" ::: "memory"); }
+
+// Cluster-wide histogram of `hb` (256 bins) and the bin holding the cut:
+// with `first`, Z = total mass and target = ceil(p Z) are set first.  Bins are
+// taken in descending score order (`ascending_bins`: bin 0 holds the highest
+// scores).  Returns the cut bin; mass_above grows by the mass before it.
+RTP_DEVICE int cluster_cut(SelSmem& S, cg::cluster_group& cluster, const uint64_t* hb, bool first,
+                           bool ascending_bins, float p, uint64_t& target, uint64_t& mass_above) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int C = (int)cluster.num_blocks();
-  const int rank = (int)cluster.block_rank();
-  float* list_s = reinterpret_cast<float*>(&S.whlo[0][0]);
-  int32_t* list_i = reinterpret_cast<int32_t*>(&S.whhi[0][0]);
-  static_assert(sizeof(S.whlo) >= kListCap * sizeof(float), "list fits in the per-warp histograms");
-
-  // members of bin lin -> local list (warp-aggregated appends)
-  uint32_t nab = 0;
-  for (int base = 0; base < nloc; base += kSelThreads) {
-    const int i = base + tid;
-    const bool valid = i < nloc;
-    const float sc = valid ? scores[i] : 0.f;
-    const int d = valid ? lin_bin(sc, m) : kBins;
-    nab += d < lin;
-    const bool mem = d == lin;
-    const uint32_t bal = __ballot_sync(0xffffffffu, mem);
-    if (bal) {
-      uint32_t b0 = 0;
-      if (lane == 0) b0 = atomicAdd(&S.nlist, (uint32_t)__popc(bal));
-      b0 = __shfl_sync(0xffffffffu, b0, 0);
-      if (mem) {
-        const uint32_t slot = b0 + (uint32_t)__popc(bal & ((1u << lane) - 1u));
-        if (slot < (uint32_t)kListCap) {
-          list_s[slot] = sc;
-          list_i[slot] = i;
-        }
-      }
-    }
-  }
-  nab = warp_sum_u32(nab);
-  if (lane == 0) atomicAdd(&S.nabove, nab);
-  __syncthreads();
-  const int nl = min((int)S.nlist, kListCap);
-  for (int j = tid; j < nl; j += kSelThreads) {
-    const float sc = list_s[j];
-    const int sb = sub_bin(sc, m, lin);
-    add_u64_pair(&S.l1lo[sb], &S.l1hi[sb], sel_weight(sc, m, two_pow_frac));
-    atomicAdd(&S.l1cnt[sb], 1u);
-  }
-  __syncthreads();
-  S.h1[tid] = pair_value(S.l1lo[tid], S.l1hi[tid]);
-  if (tid == 0) S.novf = S.nlist > (uint32_t)kListCap ? 1u : 0u;
-  cluster.sync();  // every CTA's sub-bin histogram is complete
-
-  // cluster-wide sub-bin masses and counts, identical in every CTA
-  uint64_t a = 0, c = 0;
-#pragma unroll
-  for (int r = 0; r < kMaxCluster; ++r)
-    if (r < C) {
-      a += cluster.map_shared_rank(S.h1, r)[tid];
-      c += cluster.map_shared_rank(S.l1cnt, r)[tid];
-    }
-  if (warp == 0) {
-    uint32_t na = 0, ov = 0;
-    if (lane < C) {
-      na = *cluster.map_shared_rank(&S.nabove, lane);
-      ov = *cluster.map_shared_rank(&S.novf, lane);
-    }
-    na = warp_sum_u32(na);
-    ov = warp_sum_u32(ov);
-    if (lane == 0) {
-      S.tot_above = na;
-      S.tot_ovf = ov;
-      S.cut_bin = -1;
-    }
-  }
-  uint64_t em, ec;
-  const uint64_t im = block_scan_u64(a, S.wsum, em);  // sub-bin 0 holds the highest scores
-  block_scan_u64(c, S.wsum, ec);
-  if (em < need && need <= im) {
-    S.cut_bin = tid;
-    S.cut_above = em;
-    S.cut_cnt_above = (uint32_t)ec;
-    S.cut_cnt = (uint32_t)c;
-  }
-  __syncthreads();
-  const int sb = S.cut_bin;
-  if (S.tot_ovf != 0 || sb < 0 || S.cut_cnt > (uint32_t)kCandCap) return false;
-
-  // the cut sub-bin's keys -> rank 0
+  cluster.sync();  // every CTA's histogram of this pass is complete
   {
-    uint32_t* nc = cluster.map_shared_rank(&S.ncand, 0);
-    float* cs = cluster.map_shared_rank(S.cand_s, 0);
-    int32_t* cp = cluster.map_shared_rank(S.cand_p, 0);
-    for (int j = tid; j < nl; j += kSelThreads) {
-      const float sc = list_s[j];
-      if (sub_bin(sc, m, lin) == sb) {
-        const uint32_t slot = atomicAdd(nc, 1u);
-        cs[slot] = sc;
-        cp[slot] = c0 + list_i[j];
-      }
-    }
+    uint64_t a = 0;
+#pragma unroll
+    for (int r = 0; r < kMaxCluster; ++r)
+      if (r < C) a += cluster.map_shared_rank(hb, r)[tid];
+    S.red[tid] = a;
   }
-  cluster.sync();  // rank 0 holds all candidates
+  __syncthreads();
+  if (first) {
+    uint64_t a = S.red[tid];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+    if (lane == 0) S.wsum[warp] = a;
+    __syncthreads();
+    uint64_t Z = 0;
+    for (int w = 0; w < kSelWarps; ++w) Z += S.wsum[w];
+    const double t = ceil((double)p * (double)Z);
+    const uint64_t tt = t >= (double)Z ? Z : (uint64_t)t;
+    target = tt < 1 ? 1 : tt;
+    __syncthreads();  // S.wsum is reused by the scan below
+  }
+  const uint64_t need = target - mass_above;  // >= 1
+  const int bin_of_r = ascending_bins ? tid : (kBins - 1 - tid);
+  const uint64_t mine = S.red[bin_of_r];
+  uint64_t excl;
+  const uint64_t incl = block_scan_u64(mine, S.wsum, excl);
+  if (excl < need && need <= incl) {  // exactly one position holds the cut
+    S.cut_bin = bin_of_r;
+    S.cut_above = excl;
+  }
+  __syncthreads();
+  mass_above += S.cut_above;
+  const int cb = S.cut_bin;
+  __syncthreads();
+  return cb;
+}
 
-  if (rank == 0) {
-    const int n = (int)S.ncand;  // == S.cut_cnt <= kCandCap
-    if (tid < n) {
-      const uint32_t kt = score_key(S.cand_s[tid]);
-      const int pt = S.cand_p[tid];
-      int rk = 0;
-      for (int j = 0; j < n; ++j) {
-        const uint32_t kj = score_key(S.cand_s[j]);
-        rk += (kj > kt || (kj == kt && S.cand_p[j] < pt)) ? 1 : 0;
-      }
-      S.sort_s[rk] = S.cand_s[tid];
-      S.sort_p[rk] = pt;
-    }
-    if (tid == 0) S.bc_t = n - 1;
-    __syncthreads();
-    const uint64_t w = tid < n ? sel_weight(S.sort_s[tid], m, two_pow_frac) : 0;
-    uint64_t ew;
-    const uint64_t iw = block_scan_u64(w, S.wsum, ew);
-    const uint64_t need1 = need - S.cut_above;  // >= 1, <= the sub-bin's mass
-    if (tid < n && ew < need1 && need1 <= iw) S.bc_t = tid;
-    __syncthreads();
-    if (tid < C) {
-      const int t = S.bc_t;
-      *cluster.map_shared_rank(&S.bc_tau, tid) = S.sort_s[t];
-      *cluster.map_shared_rank(&S.bc_tiepos, tid) = S.sort_p[t];
-      *cluster.map_shared_rank(&S.bc_count, tid) = S.tot_above + S.cut_cnt_above + (uint32_t)t + 1u;
+// Rank 0, once all n (<= kCandCap) keys of fine bin `fb` are in cand_s/cand_p:
+// split them into 256 sub-bins (mass and count), order the keys of the cut
+// sub-bin by (score desc, position asc), walk their weights to the cut, write
+// the result and set the selected candidates' mask bits (the other CTAs wrote
+// the words of the keys above bin fb before the candidate barrier).  `need` is
+// the mass still to take inside bin fb: >= 1 and <= the bin's mass, which the
+// candidates' weights add up to exactly.
+RTP_DEVICE void resolve_candidates(SelSmem& S, int n, int fb, float m, float two_pow_frac, uint64_t need,
+                                   uint32_t* mrow, int qrow, uint32_t* tau_bits, int32_t* tiepos,
+                                   int32_t* count) {
+  const int tid = threadIdx.x;
+  S.u.r.lo[tid] = 0;
+  S.u.r.hi[tid] = 0;
+  S.u.r.cnt[tid] = 0;
+  if (tid == 0) {
+    S.nsort = 0;
+    S.sub_cut = 0;
+    S.sub_above = 0;
+    S.sub_cnt_above = 0;
+    S.t_cut = -1;
+  }
+  __syncthreads();
+  for (int j = tid; j < n; j += kSelThreads) {
+    const float sc = S.cand_s[j];
+    const int d = sub_bin(sc, m, fb);
+    add_u64_pair(&S.u.r.lo[d], &S.u.r.hi[d], sel_weight(sc, m, two_pow_frac));
+    atomicAdd(&S.u.r.cnt[d], 1u);
+  }
+  __syncthreads();
+  uint64_t em, ec;
+  const uint64_t im = block_scan_u64(pair_value(S.u.r.lo[tid], S.u.r.hi[tid]), S.wsum, em);  // sub-bin 0 = highest
+  block_scan_u64((uint64_t)S.u.r.cnt[tid], S.wsum, ec);
+  if (em < need && need <= im) {
+    S.sub_cut = tid;
+    S.sub_above = em;
+    S.sub_cnt_above = (uint32_t)ec;
+  }
+  __syncthreads();
+  const int sb = S.sub_cut;
+  const uint64_t need2 = need - S.sub_above;
+  for (int j = tid; j < n; j += kSelThreads) {
+    const float sc = S.cand_s[j];
+    if (sub_bin(sc, m, fb) == sb) {
+      const uint32_t k = atomicAdd(&S.nsort, 1u);
+      S.u.r.s[k] = sc;
+      S.u.r.p[k] = S.cand_p[j];
     }
   }
-  cluster.sync();  // every CTA holds the cut; no distributed access after this
-  return true;
+  __syncthreads();
+  const int ns = (int)S.nsort;
+  for (int j = tid; j < ns; j += kSelThreads) {
+    const uint32_t kt = score_key(S.u.r.s[j]);
+    const int pt = S.u.r.p[j];
+    int rk = 0;
+    for (int i = 0; i < ns; ++i) {
+      const uint32_t ki = score_key(S.u.r.s[i]);
+      rk += (ki > kt || (ki == kt && S.u.r.p[i] < pt)) ? 1 : 0;
+    }
+    S.u.r.ss[rk] = S.u.r.s[j];
+    S.u.r.sp[rk] = pt;
+  }
+  __syncthreads();
+  // walk the ordered keys; thread t holds positions 4t .. 4t+3
+  uint64_t wv[4], tot = 0;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int idx = 4 * tid + k;
+    wv[k] = idx < ns ? sel_weight(S.u.r.ss[idx], m, two_pow_frac) : 0;
+    tot += wv[k];
+  }
+  uint64_t run;
+  block_scan_u64(tot, S.wsum, run);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int idx = 4 * tid + k;
+    if (idx < ns && run < need2 && need2 <= run + wv[k]) S.t_cut = idx;
+    run += wv[k];
+  }
+  __syncthreads();
+  int t = S.t_cut;
+  if (t < 0) t = ns > 0 ? ns - 1 : 0;  // not reached: the sub-bin's mass covers need2
+  const float tau = S.u.r.ss[t];
+  const int tp = S.u.r.sp[t];
+  const uint32_t tk = score_key(tau);
+  if (mrow) {
+    for (int j = tid; j < n; j += kSelThreads) {
+      const uint32_t k = score_key(S.cand_s[j]);
+      const int pos = S.cand_p[j];
+      if (k > tk || (k == tk && pos <= tp)) atomicOr(&mrow[pos >> 5], 1u << (pos & 31));
+    }
+  }
+  if (tid == 0) {
+    tau_bits[qrow] = __float_as_uint(tau);
+    tiepos[qrow] = tp;
+    count[qrow] = (int)(S.nabove + S.sub_cnt_above + (uint32_t)t + 1u);
+  }
 }
 
 template <typename T>
@@ -301,14 +335,6 @@ topp_query_kernel(View4 qv, View4 kv, const int32_t* __restrict__ lens, int Hq, 
   extern __shared__ __align__(16) unsigned char smem_raw[];
   SelSmem& S = *reinterpret_cast<SelSmem*>(smem_raw);
   float* scores = reinterpret_cast<float*>(smem_raw + sizeof(SelSmem));
-  S.l1lo[tid] = 0;
-  S.l1hi[tid] = 0;
-  S.l1cnt[tid] = 0;
-  if (tid == 0) {
-    S.nlist = 0;
-    S.nabove = 0;
-    S.ncand = 0;
-  }
 
   int n_b = N;
   if (lens) n_b = min(max(lens[b], 0), N);
@@ -339,6 +365,17 @@ topp_query_kernel(View4 qv, View4 kv, const int32_t* __restrict__ lens, int Hq, 
       count[qrow] = n_b;
     }
     return;
+  }
+
+  for (int i = tid; i < kFineBins; i += kSelThreads) {
+    S.u.f.lo[i] = 0;
+    S.u.f.hi[i] = 0;
+  }
+  if (tid == 0) {
+    S.ncand = 0;
+    S.nabove = 0;
+    S.fine_cut = 0;
+    S.fine_above = 0;
   }
 
   // ---- scores of this CTA's keys (eight independent row loads in flight per thread)
@@ -380,48 +417,145 @@ topp_query_kernel(View4 qv, View4 kv, const int32_t* __restrict__ lens, int Hq, 
   for (int r = 0; r < kMaxCluster; ++r)
     if (r < C) m = fmaxf(m, *cluster.map_shared_rank(&S.cmax_self, r));
 
-  // ---- pass 0: 256 linear bins of (max - s), 1/16 nat wide ---------------------
-  // (then either the candidate path below or key-window refinement passes)
+  // ---- pass 0: fine histogram of the weights (CTA-wide), then coarse bins ----
+  for (int base = 0; base < nloc; base += 4 * kSelThreads) {
+    float sc[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = base + u * kSelThreads + tid;
+      sc[u] = i < nloc ? scores[i] : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = base + u * kSelThreads + tid;
+      if (i < nloc) {
+        const int f = fine_bin(sc[u], m);
+        add_u64_pair(&S.u.f.lo[f], &S.u.f.hi[f], sel_weight(sc[u], m, two_pow_frac));
+      }
+    }
+  }
+  __syncthreads();
+  {
+    // coarse bin tid = fine bins 16 tid .. 16 tid + 15 (rotated start: no bank conflicts)
+    uint64_t a = 0;
+#pragma unroll
+    for (int j = 0; j < kFinePerBin; ++j) {
+      const int f = tid * kFinePerBin + ((j + tid) & (kFinePerBin - 1));
+      a += pair_value(S.u.f.lo[f], S.u.f.hi[f]);
+    }
+    S.hist[0][tid] = a;
+  }
   uint64_t target = 0, mass_above = 0;
-  int lin = -1;               // cut bin of pass 0
-  uint32_t kbase = 0;         // key window [kbase, kend) of the refinement passes
-  uint64_t kend = 0;
+  const int lin = cluster_cut(S, cluster, S.hist[0], true, true, p, target, mass_above);
+
+  if (lin < kBins - 1) {
+    // ---- the fine bin of the cut, from the 16 fine bins under coarse bin lin --
+    if (warp == 0) {
+      uint64_t a = 0;
+      if (lane < kFinePerBin) {
+        const int f = lin * kFinePerBin + lane;
+#pragma unroll
+        for (int r = 0; r < kMaxCluster; ++r)
+          if (r < C) a += pair_value(cluster.map_shared_rank(S.u.f.lo, r)[f], cluster.map_shared_rank(S.u.f.hi, r)[f]);
+      }
+      uint64_t incl = a;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint64_t t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+      }
+      const uint64_t need = target - mass_above;
+      if (lane < kFinePerBin && incl - a < need && need <= incl) {
+        S.fine_cut = lin * kFinePerBin + lane;
+        S.fine_above = mass_above + (incl - a);
+      }
+    }
+    __syncthreads();
+    const int fb = S.fine_cut;
+
+    // ---- one scan: mask words of the keys above the fine cut bin; its keys
+    //      (the candidates) and the count of keys above it go to rank 0 ------
+    {
+      uint32_t* r_ncand = cluster.map_shared_rank(&S.ncand, 0);
+      float* r_cs = cluster.map_shared_rank(S.cand_s, 0);
+      int32_t* r_cp = cluster.map_shared_rank(S.cand_p, 0);
+      uint32_t nab = 0;
+      for (int base = 0; base < n_chunk; base += 4 * kSelThreads) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int i = base + u * kSelThreads + tid;
+          const bool valid = i < nloc;
+          const float sc = valid ? scores[i] : 0.f;
+          const int f = valid ? fine_bin(sc, m) : kFineBins;
+          const uint32_t word = __ballot_sync(0xffffffffu, f < fb);
+          const int wpos = base + u * kSelThreads + warp * 32;
+          const int w = (c0 + wpos) >> 5;
+          if (lane == 0 && wpos < n_chunk && w < n_words_total) {
+            if (mrow) mrow[w] = word;
+            nab += (uint32_t)__popc(word);
+          }
+          const bool cand = f == fb;
+          const uint32_t cb = __ballot_sync(0xffffffffu, cand);
+          if (cb) {
+            uint32_t s0 = 0;
+            if (lane == 0) s0 = atomicAdd(r_ncand, (uint32_t)__popc(cb));
+            s0 = __shfl_sync(0xffffffffu, s0, 0);
+            if (cand) {
+              const uint32_t slot = s0 + (uint32_t)__popc(cb & ((1u << lane) - 1u));
+              if (slot < (uint32_t)kCandCap) {
+                r_cs[slot] = sc;
+                r_cp[slot] = c0 + i;
+              }
+            }
+          }
+        }
+      }
+      if (lane == 0 && nab) atomicAdd(cluster.map_shared_rank(&S.nabove, 0), nab);
+    }
+    cluster.sync();  // every candidate and count is at rank 0
+    const uint32_t ntot = *cluster.map_shared_rank(&S.ncand, 0);
+    cluster_arrive();  // this CTA's last distributed access
+    if (ntot <= (uint32_t)kCandCap) {
+      if (rank == 0) resolve_candidates(S, (int)ntot, fb, m, two_pow_frac, target - S.fine_above, mrow, qrow,
+                                        tau_bits, tiepos, count);
+      // rank 0 keeps its shared memory until every CTA has read the candidate total
+      if (rank == 0) cluster_wait();
+      return;
+    }
+    cluster_wait();  // more candidates than rank 0 takes: narrow in key space below
+  }
+
+  // ---- key-space narrowing inside coarse bin lin -----------------------------
+  // key window holding every score of coarse bin `lin` (with a margin)
+  uint32_t kbase;
+  uint64_t kend;
   int shift = 0;
-  bool fast = false;
-  for (int pass = 0;; ++pass) {
-    uint32_t* wlo = S.whlo[warp];
-    uint32_t* whi = S.whhi[warp];
+  {
+    const float hi_s = m - (float)lin / kCoarsePerNat;
+    const float lo_s = m - (float)(lin + 1) / kCoarsePerNat;
+    const float mg = 1e-5f * (fabsf(m) + (float)(lin + 1) / kCoarsePerNat) + 1e-30f;
+    const uint32_t khi = score_key(__fadd_rn(hi_s + mg, 0.0f));
+    const uint32_t klo = lin == kBins - 1 ? 0u : score_key(__fadd_rn(lo_s - mg, 0.0f));
+    kbase = klo;
+    kend = (uint64_t)khi + 1;
+    const uint64_t range = kend - klo;
+    while (((range - 1) >> shift) >= (uint64_t)kBins) ++shift;
+  }
+  for (int pass = 1;; ++pass) {
+    uint32_t* wlo = S.u.w.lo[warp];
+    uint32_t* whi = S.u.w.hi[warp];
     for (int i = lane; i < kBins; i += 32) {
       wlo[i] = 0;
       whi[i] = 0;
     }
     __syncwarp();
-    if (pass == 0) {
-      for (int base = 0; base < nloc; base += 4 * kSelThreads) {
-        float sc[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int i = base + u * kSelThreads + tid;
-          sc[u] = i < nloc ? scores[i] : 0.f;
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int i = base + u * kSelThreads + tid;
-          if (i < nloc) {
-            const int d = lin_bin(sc[u], m);
-            add_u64_pair(&wlo[d], &whi[d], sel_weight(sc[u], m, two_pow_frac));
-          }
-        }
-      }
-    } else {
-      for (int i = tid; i < nloc; i += kSelThreads) {
-        const float sc = scores[i];
-        if (lin_bin(sc, m) == lin) {
-          const uint32_t k = score_key(sc);
-          if (k >= kbase && (uint64_t)k < kend) {
-            const int d = (int)((uint64_t)(k - kbase) >> shift);
-            add_u64_pair(&wlo[d], &whi[d], sel_weight(sc, m, two_pow_frac));
-          }
+    for (int i = tid; i < nloc; i += kSelThreads) {
+      const float sc = scores[i];
+      if (coarse_bin(sc, m) == lin) {
+        const uint32_t k = score_key(sc);
+        if (k >= kbase && (uint64_t)k < kend) {
+          const int d = (int)((uint64_t)(k - kbase) >> shift);
+          add_u64_pair(&wlo[d], &whi[d], sel_weight(sc, m, two_pow_frac));
         }
       }
     }
@@ -430,98 +564,16 @@ topp_query_kernel(View4 qv, View4 kv, const int32_t* __restrict__ lens, int Hq, 
     {
       uint64_t a = 0;
 #pragma unroll
-      for (int w = 0; w < kSelWarps; ++w) a += pair_value(S.whlo[w][tid], S.whhi[w][tid]);
+      for (int w = 0; w < kSelWarps; ++w) a += pair_value(S.u.w.lo[w][tid], S.u.w.hi[w][tid]);
       hb[tid] = a;
     }
-    cluster.sync();  // every CTA's histogram of this pass is complete
-    // cluster-wide histogram, computed identically by every CTA
-    {
-      uint64_t a = 0;
-#pragma unroll
-      for (int r = 0; r < kMaxCluster; ++r)
-        if (r < C) a += cluster.map_shared_rank(hb, r)[tid];
-      S.red[tid] = a;
-    }
-    __syncthreads();
-    if (pass == 0) {
-      // Z = total mass; target = ceil(p Z)
-      uint64_t a = S.red[tid];
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-      if (lane == 0) S.wsum[warp] = a;
-      __syncthreads();
-      uint64_t Z = 0;
-      for (int w = 0; w < kSelWarps; ++w) Z += S.wsum[w];
-      const double t = ceil((double)p * (double)Z);
-      const uint64_t tt = t >= (double)Z ? Z : (uint64_t)t;
-      target = tt < 1 ? 1 : tt;
-      __syncthreads();  // S.wsum is reused by the scan below
-    }
-    const uint64_t need = target - mass_above;  // >= 1
-    // Bins in descending score order: pass 0 bin 0 is the highest scores;
-    // refinement bin 255 is the highest key.  Position r in that order:
-    const int bin_of_r = pass == 0 ? tid : (kBins - 1 - tid);
-    const uint64_t mine = S.red[bin_of_r];
-    uint64_t excl;
-    const uint64_t incl = block_scan_u64(mine, S.wsum, excl);
-    if (excl < need && need <= incl) {  // exactly one position holds the cut
-      S.cut_bin = bin_of_r;
-      S.cut_above = excl;
-    }
-    __syncthreads();
-    mass_above += S.cut_above;
-    const int cb = S.cut_bin;
-    __syncthreads();
-    if (pass == 0) {
-      lin = cb;
-      if (lin < kBins - 1) {
-        fast = collect_cut(S, cluster, scores, nloc, c0, m, two_pow_frac, lin, target - mass_above);
-        if (fast) break;
-      }
-      // key window holding every score of linear bin `lin` (with a margin)
-      const float hi_s = m - (float)lin / kLinBinsPerNat;
-      const float lo_s = m - (float)(lin + 1) / kLinBinsPerNat;
-      const float mg = 1e-5f * (fabsf(m) + (float)(lin + 1) / kLinBinsPerNat) + 1e-30f;
-      const uint32_t khi = score_key(__fadd_rn(hi_s + mg, 0.0f));
-      const uint32_t klo = lin == kBins - 1 ? 0u : score_key(__fadd_rn(lo_s - mg, 0.0f));
-      kbase = klo;
-      kend = (uint64_t)khi + 1;
-      const uint64_t range = kend - klo;
-      shift = 0;
-      while (((range - 1) >> shift) >= (uint64_t)kBins) ++shift;
-    } else {
-      kbase += (uint32_t)cb << shift;
-      const uint64_t e = (uint64_t)kbase + (uint64_t(1) << shift);
-      kend = e < kend ? e : kend;
-      if (shift == 0) break;            // the bracket is one score value
-      shift = shift >= 8 ? shift - 8 : 0;
-    }
-  }
-
-  if (fast) {
-    // ---- candidate path: (tau, tiepos) came from rank 0; one mask pass -------
-    const float tau = S.bc_tau;
-    const uint32_t tau_key = score_key(tau);
-    const int tpos = S.bc_tiepos;
-    for (int base = 0; base < n_chunk; base += 4 * kSelThreads) {
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int i = base + u * kSelThreads + tid;
-        const bool valid = i < nloc;
-        const uint32_t k = valid ? score_key(scores[i]) : 0u;
-        const bool sel = valid && (k > tau_key || (k == tau_key && c0 + i <= tpos));
-        const uint32_t word = __ballot_sync(0xffffffffu, sel);
-        const int wpos = base + u * kSelThreads + warp * 32;
-        const int w = (c0 + wpos) >> 5;
-        if (lane == 0 && mrow && wpos < n_chunk && w < n_words_total) mrow[w] = word;
-      }
-    }
-    if (rank == 0 && tid == 0) {
-      tau_bits[qrow] = __float_as_uint(tau);
-      tiepos[qrow] = tpos;
-      count[qrow] = (int)S.bc_count;
-    }
-    return;
+    // digit bins: bin 255 holds the highest keys
+    const int cb = cluster_cut(S, cluster, hb, false, false, p, target, mass_above);
+    kbase += (uint32_t)cb << shift;
+    const uint64_t e = (uint64_t)kbase + (uint64_t(1) << shift);
+    kend = e < kend ? e : kend;
+    if (shift == 0) break;            // the bracket is one score value
+    shift = shift >= 8 ? shift - 8 : 0;
   }
 
   // ---- counts at tau: keys above and equal, per CTA, then over the cluster ----
