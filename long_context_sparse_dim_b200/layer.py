@@ -51,44 +51,68 @@ class DecodeLayer:
         self.ws_ret = rtp.workspace(rtp.sparse_attn_decode_workspace_size(B, R * G, R, N), dev) if R else None
         self.ws_loc = (rtp.workspace(rtp.window_attn_workspace_size(B, Hq - R * G, 1, Hkv - R, N, W), dev)
                        if Hkv > R else None)
+        self._plans = {}
 
     def build_index(self, stream=None) -> None:
         """Project every cached key of the retrieval heads (done once, before decoding)."""
         if self.R:
             rtp.index_project(self.k_ret, self.P, self.k_idx, stream)
 
+    def _plan(self, main: torch.cuda.Stream, side: Optional[torch.cuda.Stream]):
+        """The step's C-ABI calls with their arguments marshalled once, for
+        this pair of streams: projections, window attention, and the chain
+        selection -> sparse attention."""
+        pre, win, chain = [], [], []
+        if self.R:
+            if self.lens_host is None:
+                n = self.N
+                pre.append(rtp.bind_index_project(self.k_ret[:, :, n - 1: n], self.P, self.k_idx[:, :, n - 1: n],
+                                                  main))
+            else:
+                for b, n in enumerate(self.lens_host):
+                    if n > 0:
+                        pre.append(rtp.bind_index_project(self.k_ret[b: b + 1, :, n - 1: n], self.P,
+                                                          self.k_idx[b: b + 1, :, n - 1: n], main))
+            pre.append(rtp.bind_index_project(self.q_ret, self.P, self.q_idx, main))
+            chain.append(rtp.bind_topp_select(self.q_idx, self.k_idx, self.lens, self.p, self.sel, self.ws_sel, main))
+            chain.append(rtp.bind_sparse_attn_decode(self.q_ret, self.k_ret, self.v_ret, self.lens, self.sel,
+                                                     self.scale, self.o_ret, self.ws_ret, main))
+        if self.Hkv > self.R:
+            win.append(rtp.bind_window_attn(self.q_loc, self.k_loc, self.v_loc, self.lens, self.W, self.scale,
+                                            self.o_loc, self.ws_loc, main if side is None else side))
+        return pre, win, chain
+
     def step(self, stream=None, side_stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
         """One decode step over the resident cache; returns o [B, Hq, 1, D].
 
         With ``side_stream`` the local heads' window attention (which does not
-        depend on the selection) runs there, forked from and joined back into
-        the main stream, so it overlaps the retrieval heads' chain."""
+        depend on the selection) runs there, forked from the main stream once
+        the selection is done and joined back at the end: the two attention
+        launches then stream their K/V rows from HBM concurrently.  The calls'
+        arguments are marshalled on the first step with a given pair of
+        streams and reused afterwards (the layer's buffers are fixed)."""
         main = torch.cuda.current_stream() if stream is None else stream
-        local = self.Hkv > self.R
-        if side_stream is not None and local:
+        key = (main.cuda_stream, None if side_stream is None else side_stream.cuda_stream)
+        plan = self._plans.get(key)
+        if plan is None:
+            plan = self._plans[key] = self._plan(main, side_stream)
+        pre, win, chain = plan
+        for call in pre:
+            call()
+        if chain:
+            chain[0]()                       # selection
+        if win and side_stream is not None:
             side_stream.wait_stream(main)
-            with torch.cuda.stream(side_stream):
-                rtp.window_attn(self.q_loc, self.k_loc, self.v_loc, self.lens, self.W, self.scale, self.o_loc,
-                                self.ws_loc, side_stream)
-            local = False
-        if self.R:
-            if self.lens_host is None:
-                n = self.N
-                rtp.index_project(self.k_ret[:, :, n - 1: n], self.P, self.k_idx[:, :, n - 1: n], stream)
-            else:
-                for b, n in enumerate(self.lens_host):
-                    if n > 0:
-                        rtp.index_project(self.k_ret[b: b + 1, :, n - 1: n], self.P,
-                                          self.k_idx[b: b + 1, :, n - 1: n], stream)
-            rtp.index_project(self.q_ret, self.P, self.q_idx, stream)
-            rtp.topp_select(self.q_idx, self.k_idx, self.lens, self.p, self.sel, self.ws_sel, stream)
-            rtp.sparse_attn_decode(self.q_ret, self.k_ret, self.v_ret, self.lens, self.sel, self.scale,
-                                   self.o_ret, self.ws_ret, stream)
-        if local:
-            rtp.window_attn(self.q_loc, self.k_loc, self.v_loc, self.lens, self.W, self.scale, self.o_loc,
-                            self.ws_loc, stream)
-        if side_stream is not None and self.Hkv > self.R:
+            for call in win:
+                call()
+            for call in chain[1:]:           # sparse attention
+                call()
             main.wait_stream(side_stream)
+        else:
+            for call in chain[1:]:
+                call()
+            for call in win:
+                call()
         return self.o
 
 

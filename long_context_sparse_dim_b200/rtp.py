@@ -239,6 +239,66 @@ def window_attn(q, k, v, lens, W: int, scale: float, o, ws=None, stream=None) ->
                                 ctypes.byref(tensor_desc(o)), w, nb, _stream(stream)), "rtp_window_attn")
 
 
+# --------------------------------------------------------------------------
+# bound calls: arguments marshalled once for buffers that do not change
+# --------------------------------------------------------------------------
+
+class Bound:
+    """One C-ABI call whose arguments (descriptors, pointers, scalars, stream)
+    were marshalled once; calling it re-issues the call with them.  Valid while
+    the tensors it was built from keep their storage and shapes."""
+
+    __slots__ = ("_fn", "_args", "_name", "_keep")
+
+    def __init__(self, name: str, args, keep):
+        self._fn = getattr(_lib, name)
+        self._args = tuple(args)
+        self._name = name
+        self._keep = keep
+
+    def __call__(self) -> None:
+        status = self._fn(*self._args)
+        if status != RTP_OK:
+            raise RtpError(status, self._name)
+
+
+def _ref(struct, keep):
+    keep.append(struct)
+    return ctypes.byref(struct)
+
+
+def bind_index_project(x, P, x_idx, stream=None) -> Bound:
+    keep = [x, P, x_idx]
+    return Bound("rtp_index_project", [_ref(tensor_desc(x), keep), _ref(tensor_desc(P, 3), keep),
+                                       _ref(tensor_desc(x_idx), keep), _stream(stream)], keep)
+
+
+def bind_topp_select(q_idx, k_idx, lens, p: float, sel: Selection, ws=None, stream=None) -> Bound:
+    keep = [q_idx, k_idx, lens, sel, ws]
+    w, nb = _ws(ws)
+    return Bound("rtp_topp_select", [_ref(tensor_desc(q_idx), keep), _ref(tensor_desc(k_idx), keep), _ptr(lens),
+                                     ctypes.c_float(p), _ref(sel.desc(), keep), w, ctypes.c_size_t(nb),
+                                     _stream(stream)], keep)
+
+
+def bind_sparse_attn_decode(q, k, v, lens, sel: Selection, scale: float, o, ws=None, stream=None) -> Bound:
+    keep = [q, k, v, lens, sel, o, ws]
+    w, nb = _ws(ws)
+    return Bound("rtp_sparse_attn_decode",
+                 [_ref(tensor_desc(q), keep), _ref(tensor_desc(k), keep), _ref(tensor_desc(v), keep), _ptr(lens),
+                  _ref(sel.desc(), keep), ctypes.c_float(scale), _ref(tensor_desc(o), keep), w,
+                  ctypes.c_size_t(nb), _stream(stream)], keep)
+
+
+def bind_window_attn(q, k, v, lens, W: int, scale: float, o, ws=None, stream=None) -> Bound:
+    keep = [q, k, v, lens, o, ws]
+    w, nb = _ws(ws)
+    return Bound("rtp_window_attn",
+                 [_ref(tensor_desc(q), keep), _ref(tensor_desc(k), keep), _ref(tensor_desc(v), keep), _ptr(lens),
+                  ctypes.c_int32(W), ctypes.c_float(scale), _ref(tensor_desc(o), keep), w, ctypes.c_size_t(nb),
+                  _stream(stream)], keep)
+
+
 def poll_device_error() -> int:
     """Synchronise, return and clear the device error word (0 = no error)."""
     code = ctypes.c_int32(0)
