@@ -35,7 +35,8 @@ def _selected(inst):
     rtp.index_project(k_ret, P, k_idx)
     rtp.index_project(q_ret, P, q_idx)
     sel = rtp.Selection.empty(w.B * R * G, w.N, dev)
-    rtp.topp_select(q_idx, k_idx, None, w.p, sel)
+    ws = rtp.workspace(rtp.topp_select_workspace_size(w.B, R * G, 1, R, w.N), dev)
+    rtp.topp_select(q_idx, k_idx, None, w.p, sel, ws)
     return q_ret, k_ret, v_ret, sel
 
 
