@@ -13,8 +13,10 @@
 //     heads is served from one read of every K/V row that ANY head of the group
 //     selected (the union of the group's masks); rows nobody selected are never
 //     loaded and 64-key tiles nobody selected are skipped;
-//   * rows are gathered with 16-byte cp.async into a 3-stage shared-memory
-//     ring (XOR-swizzled 256-byte rows so ldmatrix is conflict-free);
+//   * rows are gathered with 16-byte cp.async into a shared-memory ring of 3
+//     stages (2 for the window, so that its CTAs fit beside the selection's on
+//     an SM; both kernels ask for the largest shared-memory carveout)
+//     (XOR-swizzled 256-byte rows so ldmatrix is conflict-free);
 //   * bf16 tensor-core math (mma.sync m16n8k16) with the KEYS on the M side and
 //     the query heads of the group on N (8 columns; G <= 8), so a GQA group of
 //     4 wastes half a column tile instead of 3/4 of a row tile; the score
@@ -34,7 +36,9 @@ namespace rtp {
 
 constexpr int kAttnThreads = 128;  // 4 warps
 constexpr int kTileKeys = 64;      // keys per pipeline stage (16 per warp)
-constexpr int kStages = 3;
+constexpr int kStagesSparse = 3;  // pipeline depth of the gather (retrieval heads)
+constexpr int kStagesWindow = 2;  // and of the window (local heads): a smaller footprint lets its CTAs share
+                                  // SMs with the selection kernel, which runs concurrently
 constexpr int kRowBytes = kHeadDim * 2;  // 256 B per bf16 row
 constexpr int kTileBytes = kTileKeys * kRowBytes;
 constexpr int kMaxGroup = 8;
@@ -201,6 +205,7 @@ __device__ void finish_split(const AttnArgs& A, int grp, int split, const float*
 }
 
 // ---- bf16 tensor-core variant ---------------------------------------------
+template <int kStages>
 __global__ void __launch_bounds__(kAttnThreads)
 attn_decode_bf16_kernel(AttnArgs A) {
   pdl_wait();
@@ -613,9 +618,19 @@ cudaError_t launch_attn_decode(const LaunchAttnDecode& a, cudaStream_t stream) {
   A.tickets = reinterpret_cast<uint32_t*>(ws + (o_bytes + 255) / 256 * 256 + (ml_bytes + 255) / 256 * 256);
   dim3 grid((unsigned)splits, (unsigned)groups);
   if (a.bf16) {
-    const size_t smem = (size_t)kStages * 2 * kTileBytes + (size_t)(kMaxGroup + 1) * kMaxChunkWords * 4;
-    cudaFuncSetAttribute(attn_decode_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    return launch_pdl(attn_decode_bf16_kernel, grid, dim3(kAttnThreads), smem, stream, 1, A);
+    if (a.W > 0) {  // window: no mask staging
+      const size_t smem = (size_t)kStagesWindow * 2 * kTileBytes;
+      cudaFuncSetAttribute(attn_decode_bf16_kernel<kStagesWindow>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem);
+      cudaFuncSetAttribute(attn_decode_bf16_kernel<kStagesWindow>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           100);
+      return launch_pdl(attn_decode_bf16_kernel<kStagesWindow>, grid, dim3(kAttnThreads), smem, stream, 1, A);
+    }
+    const size_t smem = (size_t)kStagesSparse * 2 * kTileBytes + (size_t)(kMaxGroup + 1) * kMaxChunkWords * 4;
+    cudaFuncSetAttribute(attn_decode_bf16_kernel<kStagesSparse>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)smem);
+    cudaFuncSetAttribute(attn_decode_bf16_kernel<kStagesSparse>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    return launch_pdl(attn_decode_bf16_kernel<kStagesSparse>, grid, dim3(kAttnThreads), smem, stream, 1, A);
   }
   return launch_pdl(attn_decode_f32_kernel, grid, dim3(kAttnThreads), 0, stream, 1, A);
 }

@@ -22,7 +22,7 @@
 //   rank 0   splits the candidates into 256 sub-bins (1/65536 nat), orders
 //            the keys of the cut sub-bin by (score desc, position asc), walks
 //            their weights to the cut and sets the candidates' mask bits.
-// If the cut lies in the tail bin or the fine cut bin holds more than 1024
+// If the cut lies in the tail bin or the fine cut bin holds more than 512
 // keys (heavy ties), narrowing continues in key space instead: 256 bins over
 // the order-preserving uint32 image of the fp32 score (8-bit digits of the
 // offset inside the coarse cut bin) until the bracket is one score value tau;
@@ -51,9 +51,9 @@ constexpr int kMaxKeysPerCta = 32768;       // scores of one CTA held in shared 
 constexpr float kCoarsePerNat = 16.f;       // coarse bin width 1/16 nat
 constexpr float kFinePerNat = 256.f;        // fine bin width 1/256 nat
 constexpr float kSubPerNat = 65536.f;       // rank 0's sub-bin width 1/65536 nat
-constexpr int kCandCap = 1024;              // candidates rank 0 resolves
+constexpr int kCandCap = 512;               // candidates rank 0 resolves
 static_assert(kSelThreads == kBins, "one thread per histogram bin");
-static_assert(kCandCap == 4 * kSelThreads, "four candidates per thread in the walk");
+static_assert(kCandCap <= 4 * kSelThreads, "at most four candidates per thread in the walk");
 
 struct SelSmem {
   union {
@@ -317,8 +317,10 @@ RTP_DEVICE void resolve_candidates(SelSmem& S, int n, int fb, float m, float two
   }
 }
 
+// At most 96 registers a thread, so that two of these CTAs leave room on an SM
+// for a CTA of the window attention that runs concurrently.
 template <typename T>
-__global__ void __launch_bounds__(kSelThreads)
+__global__ void __maxnreg__(96)
 topp_query_kernel(View4 qv, View4 kv, const int32_t* __restrict__ lens, int Hq, int G, int N,
                    int n_chunk, float p, float two_pow_frac, uint32_t* __restrict__ tau_bits,
                    int32_t* __restrict__ tiepos, int32_t* __restrict__ count,
@@ -378,12 +380,12 @@ topp_query_kernel(View4 qv, View4 kv, const int32_t* __restrict__ lens, int Hq, 
     S.fine_above = 0;
   }
 
-  // ---- scores of this CTA's keys (eight independent row loads in flight per thread)
+  // ---- scores of this CTA's keys (four independent row loads in flight per thread)
   float qf[kIdxDim];
   load_idx_row<T>(static_cast<const T*>(qv.data) + b * qv.sb + h * qv.sh, qf);
   const T* kb = static_cast<const T*>(kv.data) + b * kv.sb + kvh * kv.sh;
   float lmax = -INFINITY;
-  constexpr int U = sizeof(T) == 2 ? 8 : 4;
+  constexpr int U = sizeof(T) == 2 ? 4 : 2;
   for (int base = 0; base < nloc; base += U * kSelThreads) {
     IdxRaw<T> raw[U];
 #pragma unroll
@@ -670,6 +672,7 @@ static int sm_count() {
 template <typename K, typename... Args>
 static cudaError_t launch_cluster(K kern, int grid, int C, size_t smem, cudaStream_t stream, Args... args) {
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
   if (C > 8) cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
   return launch_pdl(kern, dim3((unsigned)grid), dim3(kSelThreads), smem, stream, (unsigned)C, args...);
 }

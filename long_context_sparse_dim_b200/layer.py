@@ -86,11 +86,11 @@ class DecodeLayer:
         """One decode step over the resident cache; returns o [B, Hq, 1, D].
 
         With ``side_stream`` the local heads' window attention (which does not
-        depend on the selection) runs there, forked from the main stream once
-        the selection is done and joined back at the end: the two attention
-        launches then stream their K/V rows from HBM concurrently.  The calls'
-        arguments are marshalled on the first step with a given pair of
-        streams and reused afterwards (the layer's buffers are fixed)."""
+        depend on the selection) runs there, forked from the main stream after
+        the projections and joined back at the end: its CTAs share the SMs with
+        the selection, which is bound by latency rather than by HBM traffic.
+        The calls' arguments are marshalled on the first step with a given pair
+        of streams and reused afterwards (the layer's buffers are fixed)."""
         main = torch.cuda.current_stream() if stream is None else stream
         key = (main.cuda_stream, None if side_stream is None else side_stream.cuda_stream)
         plan = self._plans.get(key)
@@ -99,17 +99,15 @@ class DecodeLayer:
         pre, win, chain = plan
         for call in pre:
             call()
-        if chain:
-            chain[0]()                       # selection
         if win and side_stream is not None:
             side_stream.wait_stream(main)
             for call in win:
                 call()
-            for call in chain[1:]:           # sparse attention
+            for call in chain:
                 call()
             main.wait_stream(side_stream)
         else:
-            for call in chain[1:]:
+            for call in chain:
                 call()
             for call in win:
                 call()
