@@ -186,26 +186,68 @@ def cpu_baseline(inst, wl, budget_s=10.0):
                       f"projected-key cache prebuilt, {dt:.1f} s"}
 
 
+REFERENCE_BUDGET_S = 120.0  # the oracle arm's whole warm-up + timed run, on the host's cores
+
+
 def run_reference(args, wl, rank):
+    """The oracle arm: the CPU oracle on this workload.  A step is a bounded
+    sample of it -- a number of (sequence, head[, token]) queries sized so that
+    warm-up plus timed steps take about REFERENCE_BUDGET_S -- and the rate is
+    reported in the same unit as our arm (tokens or query tokens per second,
+    a token counting all of its heads)."""
     if rank != 0:
         return 0
+    import oracle
     inst = wls.generate(wl)
-    run = oracle_step_runner(inst, wl)
-    for i in range(args.warmup):
-        run(i % wl.B)
+    L = oracle.LayerOracle(inst.q, inst.k, inst.v, inst.P, inst.lens, R=wl.R, W=wl.W,
+                           p=float(np.float32(wl.p)), storage=wl.dtype)
+    T = inst.q.shape[2]
+    for b in range(wl.B):            # the projected-key cache exists before the step starts
+        for kvh in range(wl.R):
+            L.k_idx(b, kvh)
+    rng = np.random.default_rng(12345)
+    order = [(b, h) for b in range(wl.B) for h in range(wl.Hq)]
+    cursor = [0]
+
+    def one_query():
+        b, h = order[cursor[0] % len(order)]
+        cursor[0] += 1
+        t = 0 if T == 1 else int(rng.integers(T))
+        L.query(b, h, t)
+
+    # calibrate the cost of one query (untimed), then size the step
     t0 = time.perf_counter()
-    for i in range(args.steps):
-        run(i % wl.B)
+    for _ in range(min(wl.Hq, 8)):
+        one_query()
+    per_query = (time.perf_counter() - t0) / min(wl.Hq, 8)
+    per_step = REFERENCE_BUDGET_S / max(args.steps + args.warmup, 1)
+    q_per_step = int(min(max(per_step / max(per_query, 1e-9), 1), wl.Hq))
+    for _ in range(args.warmup):
+        for _ in range(q_per_step):
+            one_query()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        for _ in range(q_per_step):
+            one_query()
     dt = time.perf_counter() - t0
-    v = args.steps / dt
-    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
+    tokens = args.steps * q_per_step / wl.Hq
+    v = tokens / dt
+    decode = wl.mode != "prefill"
+    metric, unit = (METRIC, "tokens/s") if decode else (METRIC_PREFILL, "queries/s")
+    sample = (f"each step = {q_per_step} of the {wl.Hq} head queries of one "
+              f"{'decode token' if decode else 'uniformly drawn query token'} of {wl.name} "
+              f"(cycling over sequences and heads), projected-key cache prebuilt; a token counts all {wl.Hq} heads")
+    config = {"workload": wl.name, "B": wl.B, "N": wl.N, "Hq": wl.Hq, "Hkv": wl.Hkv,
+              "retrieval_kv_heads": wl.R, "W": wl.W, "p": wl.p}
+    if not decode:
+        config["T"] = T
+    line = {"impl": "reference", "metric": metric, "value": v, "unit": unit, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": wl.name, "B": wl.B, "N": wl.N, "Hq": wl.Hq, "Hkv": wl.Hkv,
-                                             "retrieval_kv_heads": wl.R, "W": wl.W, "p": wl.p},
-            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": _oracle_cores(), "kind": "oracle",
-                             "sample": f"each step = all {wl.Hq} heads of one sequence of {wl.name}"},
-            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+            "data": "synthetic", "config": config,
+            "cpu_baseline": {"value": v, "unit": unit, "cores": _oracle_cores(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": v, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
 
