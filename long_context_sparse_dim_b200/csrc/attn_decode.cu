@@ -551,8 +551,9 @@ static void attn_layout(int64_t B, int64_t Hk, int64_t N, int32_t W, int sms, in
   if (c < 256) c = 256;
   if (c > kMaxChunk) c = kMaxChunk;
   int64_t s = (range + c - 1) / c;
-  while (s > kMaxSplits) {  // very long ranges: grow the chunk beyond the one-wave target
-    c *= 2;
+  if (s > kMaxSplits) {  // very long ranges: the smallest tile-multiple chunk that needs at most kMaxSplits
+    c = (range + kMaxSplits - 1) / kMaxSplits;
+    c = (c + kTileKeys - 1) / kTileKeys * kTileKeys;
     s = (range + c - 1) / c;
   }
   *chunk = (int)c;

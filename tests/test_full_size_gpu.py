@@ -75,3 +75,26 @@ def test_prefill_t32768_causal_sampled():
 
 def test_prefill_chunk_t8192_n1048576_sampled():
     _prefill_full(wl.PREFILL_CHUNK_1M, 6, 1)
+
+
+def test_decode_b1_n524288_longest_supported():
+    # the longest decode context: one retrieval KV head (4 query heads, one
+    # 16-CTA cluster each in the selection) and one local KV head; the sparse
+    # attention needs its largest chunk (8192 keys x 64 splits)
+    from long_context_sparse_dim_b200.layer import DecodeLayer
+    w = wl.DECODE_B4_N128K.replace(name="decode_b1_n524288", B=1, N=524288, Hq=8, Hkv=2, R=1, needles=64,
+                                   p=0.95, seed=21)
+    inst = wl.generate(w)
+    q, k, v, P, lens = upload(inst)
+    layer = DecodeLayer(q, k, v, P, R=w.R, W=w.W, p=w.p)
+    layer.build_index()
+    o = layer.step().float().cpu().numpy()
+    torch.cuda.synchronize()
+    assert rtp.poll_device_error() == 0
+    L = make_oracle(inst)
+    res = L.run()
+    compare_outputs(o, res, w.name)
+    mask = layer.sel.mask.cpu().numpy().view(np.uint32)
+    count = layer.sel.count.cpu().numpy()
+    for h in range(w.R * w.G):
+        compare_selection(res[(0, h, 0)], mask[h], w.N, int(count[h]), f"h{h}")
