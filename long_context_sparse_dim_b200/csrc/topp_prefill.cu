@@ -10,7 +10,7 @@
 // token r of the block is TMEM lane r.  The score tile of 128 tokens x 64 keys
 // is ONE tcgen05.mma (kind::f16, M=128, N=64, K=16): the projected queries
 // (A) stay in shared memory, 64-key tiles of the projected-key cache (B) are
-// streamed by TMA (32-byte swizzle, no multicast) through a 4-stage ring, and
+// streamed by TMA (32-byte swizzle, each CTA loading its own) through a 2-stage ring, and
 // the fp32 accumulators alternate between two TMEM buffers so the next MMA
 // runs while four epilogue warps read the previous tile.  Warp roles:
 //   warps 0-3  epilogue: thread r owns query row r (its TMEM lane)
