@@ -256,15 +256,21 @@ def run_reference(args, wl, rank):
 # our arm
 # --------------------------------------------------------------------------
 
+HOST_SIDE_MARKER = "// ---- host side"
+
+
 def _traffic_record(kernel: str):
-    """DRAM bytes per launch from a committed ncu summary, if the kernel source is unchanged."""
+    """DRAM bytes per launch from a committed ncu summary, if the kernel's device
+    code (the source file up to its host-side section) is unchanged since."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             rec = json.load(f)[kernel]
-        with open(os.path.join(ROOT, rec["source"]), "rb") as f:
-            sha = hashlib.sha1(f.read()).hexdigest()
-        if sha != rec["source_sha1"]:
+        with open(os.path.join(ROOT, rec["source"]), encoding="utf-8") as f:
+            text = f.read()
+        if HOST_SIDE_MARKER in text:
+            text = text[:text.index(HOST_SIDE_MARKER)]
+        if hashlib.sha1(text.encode("utf-8")).hexdigest() != rec["device_code_sha1"]:
             return None
         return rec
     except Exception:
