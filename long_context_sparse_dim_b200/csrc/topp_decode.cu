@@ -149,7 +149,7 @@ RTP_DEVICE uint32_t warp_sum_u32(uint32_t v) {
 
 // Inclusive prefix sum over the block's threads in thread order; `wsum` holds
 // one word per warp.  Ends with a barrier, so `wsum` may be reused at once.
-RTP_DEVICE uint64_t block_scan_u64(uint64_t v, uint64_t* wsum, uint64_t& excl) {
+RTP_DEVICE uint64_t block_scan_u64(uint64_t v, uint64_t* wsum, uint64_t& excl, uint64_t* total = nullptr) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   uint64_t incl = v;
 #pragma unroll
@@ -159,9 +159,15 @@ RTP_DEVICE uint64_t block_scan_u64(uint64_t v, uint64_t* wsum, uint64_t& excl) {
   }
   if (lane == 31) wsum[warp] = incl;
   __syncthreads();
-  uint64_t off = 0;
-  for (int w = 0; w < warp; ++w) off += wsum[w];
+  uint64_t off = 0, all = 0;
+#pragma unroll
+  for (int w = 0; w < kSelWarps; ++w) {
+    const uint64_t x = wsum[w];
+    off += w < warp ? x : 0;
+    all += x;
+  }
   __syncthreads();
+  if (total) *total = all;
   incl += off;
   excl = incl - v;
   return incl;
@@ -179,44 +185,36 @@ RTP_DEVICE void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.alig
 // scores).  Returns the cut bin; mass_above grows by the mass before it.
 RTP_DEVICE int cluster_cut(SelSmem& S, cg::cluster_group& cluster, const uint64_t* hb, bool first,
                            bool ascending_bins, float p, uint64_t& target, uint64_t& mass_above) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tid = threadIdx.x;
   const int C = (int)cluster.num_blocks();
   cluster.sync();  // every CTA's histogram of this pass is complete
-  {
-    uint64_t a = 0;
+  uint64_t a = 0;
 #pragma unroll
-    for (int r = 0; r < kMaxCluster; ++r)
-      if (r < C) a += cluster.map_shared_rank(hb, r)[tid];
+  for (int r = 0; r < kMaxCluster; ++r)
+    if (r < C) a += cluster.map_shared_rank(hb, r)[tid];
+  // position r of the descending score order holds bin r (ascending bins) or bin 255 - r
+  uint64_t mine = a;
+  if (!ascending_bins) {
     S.red[tid] = a;
-  }
-  __syncthreads();
-  if (first) {
-    uint64_t a = S.red[tid];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-    if (lane == 0) S.wsum[warp] = a;
     __syncthreads();
-    uint64_t Z = 0;
-    for (int w = 0; w < kSelWarps; ++w) Z += S.wsum[w];
+    mine = S.red[kBins - 1 - tid];
+  }
+  uint64_t excl, Z;
+  const uint64_t incl = block_scan_u64(mine, S.wsum, excl, &Z);
+  if (first) {  // Z = total mass; target = ceil(p Z)
     const double t = ceil((double)p * (double)Z);
     const uint64_t tt = t >= (double)Z ? Z : (uint64_t)t;
     target = tt < 1 ? 1 : tt;
-    __syncthreads();  // S.wsum is reused by the scan below
   }
   const uint64_t need = target - mass_above;  // >= 1
-  const int bin_of_r = ascending_bins ? tid : (kBins - 1 - tid);
-  const uint64_t mine = S.red[bin_of_r];
-  uint64_t excl;
-  const uint64_t incl = block_scan_u64(mine, S.wsum, excl);
   if (excl < need && need <= incl) {  // exactly one position holds the cut
-    S.cut_bin = bin_of_r;
+    S.cut_bin = ascending_bins ? tid : (kBins - 1 - tid);
     S.cut_above = excl;
   }
   __syncthreads();
+  // (S.cut_bin and S.cut_above are written again only after the next cluster barrier)
   mass_above += S.cut_above;
-  const int cb = S.cut_bin;
-  __syncthreads();
-  return cb;
+  return S.cut_bin;
 }
 
 // Rank 0, once all n (<= kCandCap) keys of fine bin `fb` are in cand_s/cand_p:
