@@ -160,3 +160,26 @@ def test_workspace_sizes_are_monotone():
     assert 0 < a <= b
     assert rtp.window_attn_workspace_size(8, 24, 1, 6, 32768, 4096) > 0
     assert rtp.topp_select_workspace_size(8, 8, 1, 2, 32768) == 0
+
+
+def test_bench_traffic_record_follows_the_kernels_device_code(tmp_path, monkeypatch):
+    # the DRAM-traffic figure is reported while the kernel's device code (the
+    # source up to its host-side section) is the one the counters were taken on
+    import hashlib
+    import json
+    import bench
+    src = tmp_path / "k.cu"
+    device = "__global__ void k() {}\n"
+    src.write_text(device + bench.HOST_SIDE_MARKER + " ----\nint host() { return 1; }\n")
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    rec = {"kern": {"dram_bytes_retrieval_launch": 123, "source": "k.cu",
+                    "device_code_sha1": hashlib.sha1(device.encode()).hexdigest()}}
+    (prof / "traffic.json").write_text(json.dumps(rec))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench._traffic_record("kern")["dram_bytes_retrieval_launch"] == 123
+    src.write_text(device + bench.HOST_SIDE_MARKER + " ----\nint host() { return 2; }\n")  # host side only
+    assert bench._traffic_record("kern") is not None
+    src.write_text("__global__ void k() { int x; }\n" + bench.HOST_SIDE_MARKER + "\n")   # device code changed
+    assert bench._traffic_record("kern") is None
+    assert bench._traffic_record("other") is None
