@@ -183,3 +183,62 @@ def test_bench_traffic_record_follows_the_kernels_device_code(tmp_path, monkeypa
     src.write_text("__global__ void k() { int x; }\n" + bench.HOST_SIDE_MARKER + "\n")   # device code changed
     assert bench._traffic_record("kern") is None
     assert bench._traffic_record("other") is None
+
+
+class _FakeStream:
+    """Stands in for a CUDA stream handle when only the marshalling is checked."""
+
+    def __init__(self, handle):
+        self.cuda_stream = handle
+
+    def __int__(self):
+        return self.cuda_stream
+
+
+def _descs(bound, rtp):
+    return [x for x in bound._keep if isinstance(x, rtp.RtpTensor)]
+
+
+def test_decode_layer_marshals_each_call_of_the_step():
+    # the calls of one decode step, marshalled once: which calls, in which
+    # order, on which stream, and the exact views they are given
+    import torch
+    rtp = _lib()
+    from long_context_sparse_dim_b200.layer import DecodeLayer
+    B, Hq, Hkv, N, D, R, W = 2, 8, 2, 300, 128, 1, 64
+    G = Hq // Hkv
+    q = torch.zeros(B, Hq, 1, D, dtype=torch.bfloat16)
+    k = torch.zeros(B, Hkv, N, D, dtype=torch.bfloat16)
+    v = torch.zeros(B, Hkv, N, D, dtype=torch.bfloat16)
+    P = torch.zeros(R, 16, D)
+    layer = DecodeLayer(q, k, v, P, R=R, W=W, p=0.9)
+    main, side = _FakeStream(11), _FakeStream(22)
+    pre, win, chain = layer._plan(main, side)
+    assert [c._name for c in pre] == ["rtp_index_project", "rtp_index_project"]
+    assert [c._name for c in win] == ["rtp_window_attn"]
+    assert [c._name for c in chain] == ["rtp_topp_select", "rtp_sparse_attn_decode"]
+    for c in pre + chain:
+        assert c._args[-1].value == 11
+    assert win[0]._args[-1].value == 22
+    # the newest key row of the retrieval heads, a strided view of the cache
+    kx, kp, ko = _descs(pre[0], rtp)
+    assert list(kx.shape) == [B, R, 1, D] and list(kx.stride) == [Hkv * N * D, N * D, D, 1]
+    assert kx.data == k.data_ptr() + (N - 1) * D * 2
+    assert list(kp.shape)[:3] == [R, 16, D] and kp.ndim == 3
+    assert list(ko.shape) == [B, R, 1, 16] and ko.data == layer.k_idx.data_ptr() + (N - 1) * 16 * 2
+    # queries of the retrieval heads -> q_idx
+    qx, _, qo = _descs(pre[1], rtp)
+    assert list(qx.shape) == [B, R * G, 1, D] and qx.data == q.data_ptr()
+    assert list(qo.shape) == [B, R * G, 1, 16]
+    # window attention over the local heads: views starting at KV head R
+    wq, wk, wv, wo = _descs(win[0], rtp)
+    assert list(wq.shape) == [B, Hq - R * G, 1, D] and wq.data == q.data_ptr() + R * G * D * 2
+    assert list(wk.shape) == [B, Hkv - R, N, D] and wk.data == k.data_ptr() + R * N * D * 2
+    assert wv.data == v.data_ptr() + R * N * D * 2
+    assert list(wo.shape) == [B, Hq - R * G, 1, D]
+    # the selection's descriptors, then the sparse attention's
+    sq, sk = _descs(chain[0], rtp)[:2]
+    assert sq.data == layer.q_idx.data_ptr() and sk.data == layer.k_idx.data_ptr()
+    aq, ak, av, ao = _descs(chain[1], rtp)
+    assert list(ak.shape) == [B, R, N, D] and ak.data == k.data_ptr()
+    assert list(ao.shape) == [B, R * G, 1, D] and ao.data == layer.o.data_ptr()
