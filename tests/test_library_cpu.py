@@ -242,3 +242,29 @@ def test_decode_layer_marshals_each_call_of_the_step():
     aq, ak, av, ao = _descs(chain[1], rtp)
     assert list(ak.shape) == [B, R, N, D] and ak.data == k.data_ptr()
     assert list(ao.shape) == [B, R * G, 1, D] and ao.data == layer.o.data_ptr()
+
+
+def test_header_is_plain_c_and_links_against_the_library(tmp_path):
+    # include/rtp.h is a C header (C99, no C++), and a C program links
+    # against librtp.so by the names it declares
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    rtp = _lib()
+    src = tmp_path / "use.c"
+    src.write_text(
+        '#include "rtp.h"\n'
+        "int main(void) {\n"
+        "  size_t ws = rtp_topp_select_workspace_size(1, 8, 1, 2, 4096)\n"
+        "            + rtp_sparse_attn_decode_workspace_size(1, 8, 2, 4096)\n"
+        "            + rtp_window_attn_workspace_size(1, 24, 1, 6, 4096, 512);\n"
+        "  return (rtp_version() > 0 && ws > 0 && rtp_status_string(RTP_OK) != 0) ? 0 : 1;\n"
+        "}\n")
+    inc = os.path.join(ROOT, "include")
+    libdir = os.path.dirname(rtp.LIB_PATH)
+    exe = tmp_path / "use"
+    r = subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic", str(src), "-I", inc,
+                        "-L", libdir, "-lrtp", "-Wl,-rpath," + libdir, "-o", str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    assert subprocess.run([str(exe)]).returncode == 0
