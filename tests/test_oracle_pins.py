@@ -354,3 +354,34 @@ def test_mutants_are_caught(mutant, monkeypatch):
         except AssertionError:
             failures += 1
     assert failures >= 1
+
+
+# --------------------------------------------------------------------------
+# head layout: grouped-query mapping and which heads are retrieval heads
+# --------------------------------------------------------------------------
+
+def test_gqa_mapping_and_head_roles():
+    # V carries (position, KV head) in its first two coordinates.  Every query
+    # head must read KV head h // G; local heads (KV head >= R) with W = 1 see
+    # only their own position, retrieval heads with p = 1 see every key.
+    rng = np.random.default_rng(7)
+    B, Hq, Hkv, N, D, R = 2, 8, 4, 50, 16, 2
+    G = Hq // Hkv
+    q = rng.standard_normal((B, Hq, 1, D))
+    k = rng.standard_normal((B, Hkv, N, D))
+    v = np.zeros((B, Hkv, N, D))
+    v[:, :, :, 0] = np.arange(N)[None, None, :]
+    v[:, :, :, 1] = np.arange(Hkv)[None, :, None]
+    lens = np.array([N, 37])
+    P = np.zeros((R, 16, D))
+    P[:, np.arange(16), np.arange(16)] = 1.0
+    L = oracle.LayerOracle(q, k, v, P, lens, R=R, W=1, p=1.0, storage="f64")
+    for b in range(B):
+        pos = int(lens[b]) - 1
+        for h in range(Hq):
+            o = L.query(b, h, 0).o
+            assert o[1] == pytest.approx(h // G)          # the KV head of the group
+            if h // G >= R:
+                assert o[0] == pytest.approx(pos)         # window of one key: the token itself
+            else:
+                assert 0.0 < o[0] < pos                   # an average over keys 0 .. pos
