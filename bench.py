@@ -44,6 +44,8 @@ METRIC = "decode sparse-attn tokens/s"
 METRIC_PREFILL = "prefill queries/s"
 ROW_BYTES = {"bf16": 2 * 128 * 2, "f32": 2 * 128 * 4}  # one K row + one V row
 L2_BYTES = 126 * 2 ** 20
+E2E_MIN_STEPS = 200  # end-to-end decode steps timed, whatever --steps is
+PREFILL_STEPS = 10   # timed steps of the prefill object on the default decode line
 
 
 def _peaks():
@@ -147,13 +149,21 @@ class ClockSampler:
 # reference arm: the CPU oracle
 # --------------------------------------------------------------------------
 
-def _oracle_cores():
-    try:
-        from threadpoolctl import threadpool_info
-        n = max([d.get("num_threads", 1) for d in threadpool_info()] or [1])
-        return int(n)
-    except Exception:
-        return 1
+class _OneThread:
+    """The oracle evaluates one query at a time in NumPy; its BLAS calls are
+    pinned to one thread so that the reported core count is the parallelism used."""
+
+    def __enter__(self):
+        from threadpoolctl import threadpool_limits
+        self._lim = threadpool_limits(limits=1)
+        return self
+
+    def __exit__(self, *exc):
+        self._lim.unregister()
+        return False
+
+
+ORACLE_CORES = 1
 
 
 def oracle_step_runner(inst, wl):
@@ -172,6 +182,11 @@ def oracle_step_runner(inst, wl):
 
 
 def cpu_baseline(inst, wl, budget_s=10.0):
+    with _OneThread():
+        return _cpu_baseline(inst, wl, budget_s)
+
+
+def _cpu_baseline(inst, wl, budget_s):
     run = oracle_step_runner(inst, wl)
     t0 = time.perf_counter()
     done = 0
@@ -181,7 +196,7 @@ def cpu_baseline(inst, wl, budget_s=10.0):
         if time.perf_counter() - t0 >= budget_s or done >= 4 * wl.B:
             break
     dt = time.perf_counter() - t0
-    return {"value": done / dt, "unit": "tokens/s", "cores": _oracle_cores(), "kind": "oracle",
+    return {"value": done / dt, "unit": "tokens/s", "cores": ORACLE_CORES, "kind": "oracle",
             "sample": f"{done} sequences x all {wl.Hq} heads of {wl.name} (one token each), "
                       f"projected-key cache prebuilt, {dt:.1f} s"}
 
@@ -197,6 +212,11 @@ def run_reference(args, wl, rank):
     a token counting all of its heads)."""
     if rank != 0:
         return 0
+    with _OneThread():
+        return _run_reference(args, wl)
+
+
+def _run_reference(args, wl):
     import oracle
     inst = wls.generate(wl)
     L = oracle.LayerOracle(inst.q, inst.k, inst.v, inst.P, inst.lens, R=wl.R, W=wl.W,
@@ -245,7 +265,7 @@ def run_reference(args, wl, rank):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": config,
-            "cpu_baseline": {"value": v, "unit": unit, "cores": _oracle_cores(), "kind": "oracle",
+            "cpu_baseline": {"value": v, "unit": unit, "cores": ORACLE_CORES, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": v, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -367,7 +387,7 @@ def run_ours(args, wl, rank, world, local_rank):
     tr = _traffic_record("attn_decode_bf16_kernel" if wl.dtype == "bf16" else "attn_decode_f32_kernel")
 
     # end to end through the public API with host buffers
-    e2e = _e2e(layer, inst, wl, dev, max(min(args.steps, 200), 20))
+    e2e = _e2e(layer, inst, wl, dev, max(args.steps, E2E_MIN_STEPS))
 
     line = {
         "metric": METRIC, "value": world * wl.B / (step_ms * 1e-3), "unit": "tokens/s", "n_gpus": world,
@@ -398,9 +418,15 @@ def run_ours(args, wl, rank, world, local_rank):
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(inst, wl, args.cpu_budget)
+    del graphs, layer, q, k, v
+    torch.cuda.empty_cache()
+    if not args.no_prefill and wl.name == DEFAULT_WORKLOAD:
+        # the metric's second half: the 32768-token causal prefill of the same layer shape
+        line["prefill"] = measure_prefill(args, wls.PREFILL_N32K, dev, world, PREFILL_STEPS, 3,
+                                          rank == 0 and world == 1 and not args.no_cpu_baseline)
+        line["gpu_launches"] += line["prefill"]["gpu_launches"]
     if rank == 0:
         print(json.dumps(line), flush=True)
-    del graphs
     return 0
 
 
@@ -447,11 +473,12 @@ def _e2e(layer, inst, wl, dev, steps):
     h_o = torch.empty(layer.o.shape, dtype=layer.o.dtype).pin_memory()
     h2d = h_q.numel() * h_q.element_size() + 2 * h_k.numel() * h_k.element_size()
     d2h = h_o.numel() * h_o.element_size()
+    side = torch.cuda.Stream(dev)
+    layer.step(side_stream=side)       # marshals the step's calls for this stream pair (untimed)
     torch.cuda.synchronize()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record()
-    side = torch.cuda.Stream(dev)
     for _ in range(steps):
         layer.q.copy_(h_q, non_blocking=True)
         layer.k[:, :, n - 1: n].copy_(h_k, non_blocking=True)
@@ -488,6 +515,11 @@ def _prefill_calls(layer, side):
 
 
 def cpu_baseline_prefill(inst, wl, budget_s=10.0):
+    with _OneThread():
+        return _cpu_baseline_prefill(inst, wl, budget_s)
+
+
+def _cpu_baseline_prefill(inst, wl, budget_s):
     import oracle
     L = oracle.LayerOracle(inst.q, inst.k, inst.v, inst.P, inst.lens, R=wl.R, W=wl.W,
                            p=float(np.float32(wl.p)), storage=wl.dtype)
@@ -502,18 +534,17 @@ def cpu_baseline_prefill(inst, wl, budget_s=10.0):
             L.query(0, h, t)
         done += 1
     dt = time.perf_counter() - t0
-    return {"value": done / dt, "unit": "queries/s", "cores": _oracle_cores(), "kind": "oracle",
+    return {"value": done / dt, "unit": "queries/s", "cores": ORACLE_CORES, "kind": "oracle",
             "sample": f"{done} uniformly drawn query tokens x all {wl.Hq} heads of {wl.name}, "
                       f"projected-key cache prebuilt, {dt:.1f} s"}
 
 
-def run_prefill(args, wl, rank, world, local_rank):
+def measure_prefill(args, wl, dev, world, steps, warmup, with_cpu):
+    """One prefill workload measured on this rank: the JSON fields of its line."""
     import torch
     from long_context_sparse_dim_b200 import rtp  # noqa: F401
     from long_context_sparse_dim_b200.layer import PrefillLayer
 
-    torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
     inst = wls.generate(wl)
     q = torch.from_numpy(inst.q).to(dev, torch.bfloat16)
     k = torch.from_numpy(inst.k).to(dev, torch.bfloat16)
@@ -521,13 +552,13 @@ def run_prefill(args, wl, rank, world, local_rank):
     P = torch.from_numpy(inst.P).to(dev, torch.float32)
     layer = PrefillLayer(q, k, v, P, R=wl.R, W=wl.W, p=wl.p)
     side = torch.cuda.Stream(dev)
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         layer.step(side_stream=side)
     torch.cuda.synchronize()
 
     # per-kernel times, serialised on one stream (events on the launching stream)
     calls = _prefill_calls(layer, side)
-    reps = max(1, min(args.steps, 3))
+    reps = max(1, min(steps, 3))
     times = {n: [] for n, _ in calls}
     for _ in range(reps):
         for n, fn in calls:
@@ -540,7 +571,7 @@ def run_prefill(args, wl, rank, world, local_rank):
             times[n].append(a.elapsed_time(b))
     kernels_ms = {n: statistics.mean(v) for n, v in times.items()}
 
-    clocks = ClockSampler(local_rank)
+    clocks = ClockSampler(dev.index)
     clocks.start()
     time.sleep(0.2)
     barrier(world, dev)
@@ -548,14 +579,14 @@ def run_prefill(args, wl, rank, world, local_rank):
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     t_start.record()
-    for _ in range(args.steps):
+    for _ in range(steps):
         layer.step(side_stream=side)
     t_end.record()
     torch.cuda.synchronize()
     barrier(world, dev)
     clock_info = clocks.stop()
     assert rtp.poll_device_error() == 0, "a device wait timed out"
-    step_ms = max_over_ranks(t_start.elapsed_time(t_end) / args.steps, world, dev)
+    step_ms = max_over_ranks(t_start.elapsed_time(t_end) / steps, world, dev)
 
     G, R = wl.G, wl.R
     T, N = wl.T, wl.N
@@ -568,31 +599,55 @@ def run_prefill(args, wl, rank, world, local_rank):
     attn_flop = 4.0 * 128 * admitted                   # QK^T + PV, 2 FLOP per MAC
     win_flop = 4.0 * 128 * win
     gemm_flop = 2.0 * 16 * causal                      # one pass of the depth-16 score GEMM
-    dom = max(("sparse_attn_prefill", attn_flop), ("window_attn", win_flop), key=lambda x: kernels_ms.get(x[0], 0))
-    dom_ach = dom[1] / (kernels_ms[dom[0]] * 1e-3) / 1e12
-    line = {
+    flop = {"sparse_attn_prefill": attn_flop, "window_attn": win_flop, "topp_select": gemm_flop}
+    dom = max((n for n in flop if n in kernels_ms), key=lambda n: kernels_ms[n])
+    dom_ach = flop[dom] / (kernels_ms[dom] * 1e-3) / 1e12
+    out = {
         "metric": METRIC_PREFILL, "value": world * wl.B * T / (step_ms * 1e-3), "unit": "queries/s",
-        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "ms_per_step": step_ms, "steps": steps, "warmup": warmup, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": wl.name, "B": wl.B, "T": T, "N": N, "Hq": wl.Hq, "Hkv": wl.Hkv,
                    "retrieval_kv_heads": R, "W": wl.W, "p": wl.p,
                    "l2": "inputs larger than L2 (K/V cache and score sweeps), no flush",
                    "parallelism": f"replicas x{world}"},
-        "roofline": {"kernel": dom[0], "bound": "tensor", "achieved": dom_ach, "peak": sustained,
+        "roofline": {"kernel": dom, "bound": "tensor", "achieved": dom_ach, "peak": sustained,
                      "unit": "TFLOP/s", "frac": dom_ach / sustained, "peak_kind": pk + " sustained",
-                     "traffic": None, "algorithmic_flop": dom[1], "ms_per_launch": kernels_ms[dom[0]]},
+                     "traffic": None, "algorithmic_flop": flop[dom], "ms_per_launch": kernels_ms[dom],
+                     "flop_per_unit": {"sparse_attn_prefill": "512 per admitted (query, key) pair",
+                                       "window_attn": "512 per (query, key) pair in the band",
+                                       "topp_select": "32 per causal (query, key) pair, one pass of the "
+                                                      "score GEMM"}[dom]},
         "score_gemm": {"kernel": "topp_select", "algorithmic_flop_one_pass": gemm_flop,
+                       "causal_pairs": causal,
                        "achieved_tflops_one_pass": gemm_flop / (kernels_ms["topp_select"] * 1e-3) / 1e12,
-                       "frac_of_burst": gemm_flop / (kernels_ms["topp_select"] * 1e-3) / 1e12 / burst},
+                       "frac_of_burst": gemm_flop / (kernels_ms["topp_select"] * 1e-3) / 1e12 / burst,
+                       "pairs_per_s": causal / (kernels_ms["topp_select"] * 1e-3)},
         "kernels_ms": kernels_ms,
+        "kernels_tflops": {n: flop[n] / (kernels_ms[n] * 1e-3) / 1e12 for n in flop if n in kernels_ms},
         "selection": {"mean_selected_fraction": admitted / max(causal, 1)},
-        "gpu_launches": len(calls) * args.steps,
+        "gpu_launches": len(calls) * steps,
         "streams": "window attention (local heads) forked onto a second stream inside each step",
         "clocks": clock_info,
     }
-    line["e2e"] = _e2e_prefill(layer, inst, dev, side, max(1, min(args.steps, 3)))
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline_prefill(inst, wl, args.cpu_budget)
+    out["e2e"] = _e2e_prefill(layer, inst, dev, side, max(1, min(steps, 3)))
+    if with_cpu:
+        out["cpu_baseline"] = cpu_baseline_prefill(inst, wl, args.cpu_budget)
+    del layer, q, k, v
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_prefill(args, wl, rank, world, local_rank):
+    import torch
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    m = measure_prefill(args, wl, dev, world, args.steps, args.warmup,
+                        rank == 0 and world == 1 and not args.no_cpu_baseline)
+    line = {"metric": m.pop("metric"), "value": m.pop("value"), "unit": m.pop("unit"), "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": m.pop("ms_per_step"),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None}
+    m.pop("steps")
+    m.pop("warmup")
+    line.update(m)
     if rank == 0:
         print(json.dumps(line), flush=True)
     return 0
@@ -633,6 +688,7 @@ def main(argv=None):
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(ALL_WORKLOADS))
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true", help="leave the prefill object out of the decode line")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3

@@ -165,8 +165,12 @@ RTP_API size_t rtp_sparse_attn_decode_workspace_size(int64_t B, int64_t Hq, int6
  *     keeps until the process exits.  Shapes whose scratch would exceed it
  *     (rtp_sparse_attn_decode_workspace_size() > RTP_NOALLOC_SCRATCH_BYTES)
  *     return RTP_ERR_UNSUPPORTED.
- *   - The first call on a device (with that device current) looks up the
- *     array's device address; make that first call before any stream capture.
+ *   - The first call in a CUDA context (on a device, with that context
+ *     current) looks up the array's device address; make that first call
+ *     before any stream capture.  After a device reset, or in another context
+ *     on the same device, the next call looks it up again.
+ *   - Every argument is checked first: an error status means nothing was
+ *     enqueued and the array was not touched.
  *   - All calls on a device share the array: calls that overlap on the GPU
  *     race.  Order them on one stream.  Each call clears the part of the array
  *     that must start at zero; the rest keeps the previous call's contents.
@@ -216,6 +220,15 @@ RTP_API size_t rtp_window_attn_workspace_size(int64_t B, int64_t Hq, int64_t T, 
  */
 #define RTP_DEVICE_ERR_TIMEOUT 1
 RTP_API rtp_status rtp_poll_device_error(int32_t* code);
+/* Budget, in GPU clock cycles, of each bounded device wait in the prefill
+ * kernels launched after this call (process-wide).  0 restores the default
+ * (4e9 cycles, about two seconds); a negative value is RTP_ERR_INVALID_ARG.
+ * A diagnostic knob: a tiny budget makes waits give up on purpose, which is
+ * how the give-up path is tested; the results of such a launch are invalid,
+ * the error word reports RTP_DEVICE_ERR_TIMEOUT, and the next launch with the
+ * default budget is unaffected (a kernel that gives up still waits for the
+ * copies and tensor-core operations it issued before it exits). */
+RTP_API rtp_status rtp_set_wait_budget_cycles(int64_t cycles);
 
 /* ---- utilities ---------------------------------------------------------- */
 RTP_API const char* rtp_status_string(rtp_status s);   /* static string, never NULL */

@@ -16,15 +16,15 @@
 //   * all calls on a device share the one array, so calls that overlap on the
 //     GPU (different streams without ordering between them) race and give
 //     wrong results; order them on one stream;
-//   * the array's device address is looked up once per device, on the first
-//     call made with that device current (cudaGetSymbolAddress); make that
-//     first call before any stream capture.
-// The array keeps whatever the previous call left in it; the only part that
-// must start at zero (the per-group completion tickets) is cleared on the
-// stream by every call.  No cudaMalloc, cudaFree or allocating library routine
+//   * the array's device address is looked up once per CUDA context, on the
+//     first call made with that context current (cudaGetSymbolAddress); make
+//     that first call before any stream capture.  A device reset or a second
+//     context on the same device gets its own lookup.
+// Every argument is checked before anything is enqueued, so a call that returns
+// an error status has launched nothing and written nothing.  The array keeps
+// whatever the previous call left in it; the only part that must start at zero
+// (the per-group completion tickets) is cleared on the stream by every call.  No cudaMalloc, cudaFree or allocating library routine
 // is called.
-#include <mutex>
-
 #include <cuda_runtime.h>
 
 #include "launch.h"
@@ -32,29 +32,7 @@
 
 namespace {
 
-constexpr int kMaxDevices = 64;
-
 static __device__ __align__(256) unsigned char g_noalloc_scratch[RTP_NOALLOC_SCRATCH_BYTES];
-
-std::mutex g_setup_mu;
-void* g_scratch_ptr[kMaxDevices] = {};
-
-// Device address of the scratch array on the current device (looked up once).
-cudaError_t scratch_address(void** out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> lock(g_setup_mu);
-  if (!g_scratch_ptr[dev]) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess) return e;
-    g_scratch_ptr[dev] = p;
-  }
-  *out = g_scratch_ptr[dev];
-  return cudaSuccess;
-}
 
 }  // namespace
 
@@ -62,17 +40,20 @@ extern "C" rtp_status rtp_sparse_attn_decode_noalloc(const rtp_tensor* q, const 
                                                      const rtp_tensor* v, const int32_t* lens,
                                                      const rtp_selection* sel, float scale,
                                                      const rtp_tensor* o, rtp_stream_t stream) {
-  if (!q || !k || q->ndim != 4 || k->ndim != 4) return RTP_ERR_INVALID_ARG;
-  const size_t need = rtp_sparse_attn_decode_workspace_size(q->shape[0], q->shape[1], k->shape[1], k->shape[2]);
+  // every argument check first: an invalid call launches and writes nothing
+  rtp::LaunchAttnDecode a;
+  const rtp_status s = rtp::check_sparse_attn_decode(q, k, v, lens, sel, scale, o, &a);
+  if (s != RTP_OK) return s;
+  const size_t need = rtp_sparse_attn_decode_workspace_size(a.B, a.Hq, a.Hk, a.N);
   if (need > (size_t)RTP_NOALLOC_SCRATCH_BYTES) return RTP_ERR_UNSUPPORTED;
   void* scratch = nullptr;
-  cudaError_t e = scratch_address(&scratch);
+  cudaError_t e = rtp::symbol_address(reinterpret_cast<const void*>(&g_noalloc_scratch), &scratch);
   if (e != cudaSuccess) {
     rtp::set_last_cuda_error((int32_t)e);
     return RTP_ERR_CUDA;
   }
   size_t t_off = 0, t_bytes = 0;
-  rtp::attn_decode_ticket_range(q->shape[0], k->shape[1], k->shape[2], 0, &t_off, &t_bytes);
+  rtp::attn_decode_ticket_range(a.B, a.Hk, a.N, 0, &t_off, &t_bytes);
   if (t_bytes) {
     e = cudaMemsetAsync(static_cast<unsigned char*>(scratch) + t_off, 0, t_bytes, (cudaStream_t)stream);
     if (e != cudaSuccess) {
@@ -80,5 +61,11 @@ extern "C" rtp_status rtp_sparse_attn_decode_noalloc(const rtp_tensor* q, const 
       return RTP_ERR_CUDA;
     }
   }
-  return rtp_sparse_attn_decode(q, k, v, lens, sel, scale, o, scratch, (size_t)RTP_NOALLOC_SCRATCH_BYTES, stream);
+  a.ws = scratch;
+  e = rtp::launch_attn_decode(a, (cudaStream_t)stream);
+  if (e != cudaSuccess) {
+    rtp::set_last_cuda_error((int32_t)e);
+    return RTP_ERR_CUDA;
+  }
+  return RTP_OK;
 }

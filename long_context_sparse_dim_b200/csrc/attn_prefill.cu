@@ -65,6 +65,7 @@ struct ApArgs {
   MutView4 o;
   int o_bf16;
   int* err;
+  long long budget;
 };
 
 RTP_DEVICE uint32_t ap_swz(int r, int c) { return (uint32_t)(r * kApRowBytes + ((c ^ (r & 7)) << 4)); }
@@ -147,29 +148,40 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
     if (lane == 0 && ntiles > 0) {
       mbar_expect_tx(&S.qidx_full, kApRows * kIdxDim * 2);
       tma_load_4d(S.qidx, &qmap, &S.qidx_full, 0, t0, h, b);
+      int loads = 0, mma_issued = 0;
       for (int i = 0; i < ntiles && i < 2; ++i) {
         mbar_expect_tx(&S.kidx_full[i], kApIdxTileBytes);
         tma_load_4d(S.kidx[i], &kmap, &S.kidx_full[i], 0, (tile0 + i) * kApKeys, kvh, b);
+        loads = i + 1;
       }
-      mbar_wait(&S.qidx_full, 0, alive, A.err);
+      mbar_wait(&S.qidx_full, 0, alive, A.err, A.budget);
       const uint64_t adesc = umma_desc_k_sw32(S.qidx);
       constexpr uint32_t idesc = umma_idesc_bf16_f32(kApRows, kApKeys);
       for (int i = 0; i < ntiles; ++i) {
         const int st = i & 1;
         const uint32_t ph = (i >> 1) & 1;
-        if (!mbar_wait(&S.kidx_full[st], ph, alive, A.err)) break;
-        if (!mbar_wait(&S.t_empty[st], ph ^ 1, alive, A.err)) break;
+        if (!mbar_wait(&S.kidx_full[st], ph, alive, A.err, A.budget)) break;
+        if (!mbar_wait(&S.t_empty[st], ph ^ 1, alive, A.err, A.budget)) break;
         tc_fence_after();
         umma_f16(tmem + st * kApKeys, adesc, umma_desc_k_sw32(S.kidx[st]), idesc, 0);
         umma_commit(&S.kidx_empty[st]);
         umma_commit(&S.t_full[st]);
+        mma_issued = i + 1;
         if (i + 2 < ntiles) {  // refill this stage once the MMA has read it
-          if (!mbar_wait(&S.kidx_empty[st], ph, alive, A.err)) break;
+          if (!mbar_wait(&S.kidx_empty[st], ph, alive, A.err, A.budget)) break;
           mbar_expect_tx(&S.kidx_full[st], kApIdxTileBytes);
           tma_load_4d(S.kidx[st], &kmap, &S.kidx_full[st], 0, (tile0 + i + 2) * kApKeys, kvh, b);
+          loads = i + 3;
         }
       }
-      if (ntiles > 0) mbar_wait(&S.t_full[(ntiles - 1) & 1], ((ntiles - 1) >> 1) & 1, alive, A.err);
+      // wind down: the last MMA and every TMA load issued land before TMEM is freed
+      if (ntiles > 0) {
+        mbar_drain(&S.qidx_full, 0, A.err);
+        for (int i = loads > 2 ? loads - 2 : 0; i < loads; ++i)
+          mbar_drain(&S.kidx_full[i & 1], (i >> 1) & 1, A.err);
+        if (mma_issued > 0)
+          mbar_drain(&S.t_full[(mma_issued - 1) & 1], ((mma_issued - 1) >> 1) & 1, A.err);
+      }
     }
   } else {
     // ---------------- math warps 0-7 ----------------
@@ -253,7 +265,7 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
       if (SPARSE && warp < 4) {
         // admission bitmap of row `tid` for this tile
         uint32_t w0 = 0u, w1 = 0u;
-        if (mbar_wait(&S.t_full[st], (i >> 1) & 1, alive, A.err)) {
+        if (mbar_wait(&S.t_full[st], (i >> 1) & 1, alive, A.err, A.budget)) {
           tc_fence_after();
           uint32_t v0[32], v1[32];
           const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16) + st * kApKeys;
@@ -418,8 +430,6 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
 }
 
 // ---- host ---------------------------------------------------------------------
-bool make_idx_map(CUtensorMap* map, const View4& v, int64_t B, int64_t H, int64_t R, int box_rows);
-
 cudaError_t launch_attn_prefill(const LaunchAttnPrefill& a, cudaStream_t stream) {
   if (a.B * a.Hq * a.T == 0) return cudaSuccess;
   ApArgs A;
@@ -439,6 +449,7 @@ cudaError_t launch_attn_prefill(const LaunchAttnPrefill& a, cudaStream_t stream)
   A.o = a.o;
   A.o_bf16 = a.o_bf16 ? 1 : 0;
   A.err = a.err;
+  A.budget = wait_budget_cycles();
   const size_t smem = sizeof(ApSmem) + 1024;
   const dim3 grid((unsigned)((a.T + kApRows - 1) / kApRows), (unsigned)(a.B * a.Hq));
   if (a.W > 0) {

@@ -2,6 +2,7 @@
 // Arguments arrive here already validated.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -98,8 +99,15 @@ struct LaunchAttnPrefill {
 };
 cudaError_t launch_attn_prefill(const LaunchAttnPrefill& a, cudaStream_t stream);
 
-// Device address of the library's error word on the current device.
+// Device address of the library's error word in the current CUDA context.
 cudaError_t device_error_word(int** out);
+// Device address of a file-scope __device__ variable (given by its host-side
+// name) in the current CUDA context, looked up once per context: a device
+// reset or another context on the same device gets its own lookup.
+cudaError_t symbol_address(const void* symbol, void** out);
+// Cycles a device wait may take before it gives up (rtp_set_wait_budget_cycles).
+constexpr long long kDefaultWaitBudgetCycles = 4000000000LL;  // ~2 s at 1.9 GHz
+long long wait_budget_cycles();
 
 // Decode attention: sparse (mask given) or sliding window (W > 0).
 struct LaunchAttnDecode {
@@ -119,8 +127,19 @@ struct LaunchAttnDecode {
 bool attn_decode_supported(int64_t B, int64_t Hk, int64_t N, int32_t W);
 size_t attn_decode_workspace_bytes(int64_t B, int64_t Hq, int64_t Hk, int64_t N, int32_t W);
 cudaError_t launch_attn_decode(const LaunchAttnDecode& a, cudaStream_t stream);
+// Every check rtp_sparse_attn_decode makes except the workspace's; on RTP_OK
+// *a holds the launch arguments (a->ws still to be set).  Nothing is launched.
+rtp_status check_sparse_attn_decode(const rtp_tensor* q, const rtp_tensor* k, const rtp_tensor* v,
+                                    const int32_t* lens, const rtp_selection* sel, float scale,
+                                    const rtp_tensor* o, LaunchAttnDecode* a);
 // Byte range of the completion tickets inside a decode-attention workspace.
 void attn_decode_ticket_range(int64_t B, int64_t Hk, int64_t N, int32_t W, size_t* offset, size_t* bytes);
+
+// TMA descriptors: [B, H, R, 16] bf16 projected rows (box of box_rows rows,
+// 32-byte swizzle), and [B, H, R, 128] bf16 K/V rows (box of box_rows rows x
+// 64 columns, 128-byte swizzle).
+bool make_idx_map(CUtensorMap* map, const View4& v, int64_t B, int64_t H, int64_t R, int box_rows);
+bool make_row_map(CUtensorMap* map, const View4& v, int64_t B, int64_t H, int64_t R, int box_rows);
 
 // Records a CUDA error for rtp_last_cuda_error() on this thread.
 void set_last_cuda_error(int32_t e);

@@ -203,35 +203,50 @@ static rtp_status check_decode_common(const rtp_tensor* q, const rtp_tensor* k, 
   return RTP_OK;
 }
 
-rtp_status rtp_sparse_attn_decode(const rtp_tensor* q, const rtp_tensor* k, const rtp_tensor* v,
-                                  const int32_t* lens, const rtp_selection* sel, float scale,
-                                  const rtp_tensor* o, void* workspace, size_t workspace_bytes,
-                                  rtp_stream_t stream) {
+}  // extern "C"
+
+namespace rtp {
+rtp_status check_sparse_attn_decode(const rtp_tensor* q, const rtp_tensor* k, const rtp_tensor* v,
+                                    const int32_t* lens, const rtp_selection* sel, float scale,
+                                    const rtp_tensor* o, LaunchAttnDecode* a) {
   rtp_status s;
   if ((s = check_decode_common(q, k, v, o, scale)) != RTP_OK) return s;
   if (q->shape[2] != 1) return RTP_ERR_SHAPE;
   if (!sel || !sel->mask) return RTP_ERR_INVALID_ARG;
   const int64_t N = k->shape[2];
   if (sel->mask_words < (N + 31) / 32) return RTP_ERR_SHAPE;
-  const size_t need = rtp_sparse_attn_decode_workspace_size(q->shape[0], q->shape[1], k->shape[1], N);
-  if ((s = check_workspace(workspace, workspace_bytes, need)) != RTP_OK) return s;
-  if (!rtp::attn_decode_supported(q->shape[0], k->shape[1], N, 0)) return RTP_ERR_UNSUPPORTED;
+  if (!attn_decode_supported(q->shape[0], k->shape[1], N, 0)) return RTP_ERR_UNSUPPORTED;
+  a->q = view(q);
+  a->k = view(k);
+  a->v = view(v);
+  a->lens = lens;
+  a->mask = sel->mask;
+  a->mask_words = sel->mask_words;
+  a->B = q->shape[0];
+  a->Hq = q->shape[1];
+  a->Hk = k->shape[1];
+  a->N = N;
+  a->W = 0;
+  a->scale = scale;
+  a->bf16 = q->dtype == RTP_BF16;
+  a->o = mview(o);
+  a->o_bf16 = o->dtype == RTP_BF16;
+  a->ws = nullptr;
+  return RTP_OK;
+}
+}  // namespace rtp
+
+extern "C" {
+
+rtp_status rtp_sparse_attn_decode(const rtp_tensor* q, const rtp_tensor* k, const rtp_tensor* v,
+                                  const int32_t* lens, const rtp_selection* sel, float scale,
+                                  const rtp_tensor* o, void* workspace, size_t workspace_bytes,
+                                  rtp_stream_t stream) {
   rtp::LaunchAttnDecode a;
-  a.q = view(q);
-  a.k = view(k);
-  a.v = view(v);
-  a.lens = lens;
-  a.mask = sel->mask;
-  a.mask_words = sel->mask_words;
-  a.B = q->shape[0];
-  a.Hq = q->shape[1];
-  a.Hk = k->shape[1];
-  a.N = N;
-  a.W = 0;
-  a.scale = scale;
-  a.bf16 = q->dtype == RTP_BF16;
-  a.o = mview(o);
-  a.o_bf16 = o->dtype == RTP_BF16;
+  rtp_status s;
+  if ((s = rtp::check_sparse_attn_decode(q, k, v, lens, sel, scale, o, &a)) != RTP_OK) return s;
+  const size_t need = rtp_sparse_attn_decode_workspace_size(a.B, a.Hq, a.Hk, a.N);
+  if ((s = check_workspace(workspace, workspace_bytes, need)) != RTP_OK) return s;
   a.ws = workspace;
   return cuda_status(rtp::launch_attn_decode(a, (cudaStream_t)stream));
 }

@@ -1,10 +1,12 @@
 // sm_100a building blocks: mbarriers with time-bounded waits, TMA tile loads,
 // tcgen05 (5th-generation tensor core) MMA with accumulators in tensor memory.
 //
-// Every wait here gives up after kWaitBudgetCycles, records a code in the
-// library's device error word (its address is passed to each kernel; the host
-// reads and clears it with rtp_poll_device_error) and lets the kernel wind
-// down, so a protocol mistake can never hang the GPU.
+// Every wait here gives up after a cycle budget (kWaitBudgetCycles, about two
+// seconds, unless the host set another one), records a code in the library's
+// device error word (its address is passed to each kernel; the host reads and
+// clears it with rtp_poll_device_error) and lets the kernel wind down, so a
+// protocol mistake can never hang the GPU.  Winding down still waits (bounded)
+// for the asynchronous copies and tensor-core operations already issued.
 #pragma once
 
 #include <cuda.h>
@@ -16,7 +18,7 @@
 namespace rtp {
 
 constexpr int kDevErrTimeout = 1;  // value written to the device error word
-constexpr long long kWaitBudgetCycles = 4000000000LL;  // ~2 s at 1.9 GHz
+constexpr long long kWaitBudgetCycles = 4000000000LL;  // ~2 s at 1.9 GHz; the default wait budget
 
 RTP_DEVICE uint32_t smem_addr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
@@ -57,20 +59,37 @@ RTP_DEVICE bool mbar_try(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 // Wait for the phase with the given parity to complete; false on timeout
-// (the error word is set).  Once any wait of the kernel timed out, `alive`
-// is false and later waits return at once.
-RTP_DEVICE bool mbar_wait(uint64_t* bar, uint32_t parity, bool& alive, int* err) {
+// (the error word is set).  `budget` is the number of clock cycles the wait
+// may take (kWaitBudgetCycles unless the host set another budget).  Once any
+// wait of the kernel timed out, `alive` is false and later waits return at
+// once.
+RTP_DEVICE bool mbar_wait(uint64_t* bar, uint32_t parity, bool& alive, int* err, long long budget) {
   if (!alive) return false;
   if (mbar_try(bar, parity)) return true;
   const long long t0 = clock64();
   while (!mbar_try(bar, parity)) {
-    if (clock64() - t0 > kWaitBudgetCycles) {
+    if (clock64() - t0 > budget) {
       atomicExch(err, kDevErrTimeout);
       alive = false;
       return false;
     }
   }
   return true;
+}
+
+// Wind-down wait for an asynchronous operation this CTA already issued (a TMA
+// load or a tensor-core commit): it ignores `alive`, because such an operation
+// completes on its own and must land before the CTA frees its tensor memory or
+// exits.  Bounded by kWaitBudgetCycles all the same; a give-up is recorded.
+RTP_DEVICE void mbar_drain(uint64_t* bar, uint32_t parity, int* err) {
+  if (mbar_try(bar, parity)) return;
+  const long long t0 = clock64();
+  while (!mbar_try(bar, parity)) {
+    if (clock64() - t0 > kWaitBudgetCycles) {
+      atomicExch(err, kDevErrTimeout);
+      return;
+    }
+  }
 }
 
 // ---- TMA -------------------------------------------------------------------

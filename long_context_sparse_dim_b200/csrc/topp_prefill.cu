@@ -1,39 +1,48 @@
 // a2 + a3 (prefill): indexer scores of every (query, earlier key) pair on the
 // tcgen05 tensor cores, and the dynamic top-p cut of every query over its
-// causal prefix, in threshold form (tau, tiepos, count).
+// causal prefix, in threshold form (tau, tiepos, count) and optionally as a
+// selection mask.
 //
 // "RTPurbo: Turning Dense LLMs into Sparse Attention Models with Just a Few
 // Hundred Training Steps", "Three Key Insights" 2-3: a 16-dim indexer ranks the
 // tokens and each query keeps the cumulative top-p of that ranking.
 //
 // Design (B200): a CTA takes one query head and 128 consecutive query tokens;
-// token r of the block is TMEM lane r.  The score tile of 128 tokens x 64 keys
-// is ONE tcgen05.mma (kind::f16, M=128, N=64, K=16): the projected queries
-// (A) stay in shared memory, 64-key tiles of the projected-key cache (B) are
-// streamed by TMA (32-byte swizzle, each CTA loading its own) through a 2-stage ring, and
+// token r of the block is TMEM lane r.  A score tile of 128 tokens x 128 keys
+// is ONE tcgen05.mma (kind::f16, M=128, N=128, K=16): the projected queries
+// (A) stay in shared memory, 128-key tiles of the projected-key cache (B) are
+// streamed by TMA (32-byte swizzle, no multicast) through a 4-stage ring, and
 // the fp32 accumulators alternate between two TMEM buffers so the next MMA
-// runs while four epilogue warps read the previous tile.  Warp roles:
-//   warps 0-3  epilogue: thread r owns query row r (its TMEM lane)
-//   warp 4     TMA producer (one elected lane)
-//   warp 5     MMA issuer (one elected lane)
+// runs while the epilogue reads the previous tile.  Warp roles (two CTAs per
+// SM):
+//   warps 0-7  epilogue: warp w reads TMEM lane quadrant w % 4; warps 0-3
+//              take columns 0-63 of every tile, warps 4-7 columns 64-127, so
+//              each query row is served by two threads ("halves"); the half-0
+//              thread owns the row's decisions
+//   warp 8     TMA producer (one elected lane)
+//   warp 9     MMA issuer (one elected lane)
 // The cut of every row is found by sweeps over its causal prefix; each sweep
 // recomputes the score tiles (depth-16 MMAs are cheap) and narrows a bracket
-// around the cut score, every row on the same schedule:
-//   MAX      row maximum m
-//   LIN 0-3  32 bins of u = m - s, 1/4, 1/128, 1/4096, 1/131072 nat wide (each
-//            level splits the previous cut bin; power-of-two rescaling of u is
-//            exact), with 64-bit fixed-point masses (Z on level 0) and counts
-//   COLLECT  once the cut bin holds <= 32 keys, their (score, position) pairs
-//            are kept and an in-thread sort by (score desc, position asc)
-//            finishes the cut: tau, the number taken, tiepos, count
-// Fallbacks: the tail bin of level 0, or a bin still too full after level 3,
+// around the cut score.  All arithmetic is on the raw accumulator v = 4 s (the
+// score scaling is exact), with u = m - v for the row maximum m:
+//   MAX      row maximum m (3-input max, two independent halves)
+//   LIN0     32 bins of u (1/4 nat each, the last one the tail u >= 31), with
+//            64-bit fixed-point masses; Z is their sum
+//   LIN 1-3  32 sub-bins of the previous cut bin (widths 1/128, 1/4096,
+//            1/131072 nat; power-of-two rescaling of u is exact), masses and
+//            counts
+//   COLLECT  once the cut bin holds <= 32 keys, their (v, position) pairs are
+//            kept and sorted by (score desc, position asc) to finish the cut
+//   MASK     (only when a mask is requested) one more sweep writes it
+// Fallbacks: a cut in the tail bin, or a bin still too full after LIN 3,
 // continue with 5-bit digits of the order-preserving uint32 image of the score
-// (KEY) until one value is left, then a TIE sweep counts and locates the ties;
-// the TIE sweep also writes the optional selection mask.
-// A row owns its 32-bin histogram columns in shared memory (no atomics); the
-// candidate list reuses the row's mass column.
-#include <cudaTypedefs.h>
-
+// (KEY) until one value is left; a TIE sweep then counts the keys above it and
+// locates the ties in position order.
+// Every bracket is an interval (vlo, vhi] of raw accumulators, precomputed
+// once per row and sweep, so testing a key costs two compares; keys inside a
+// bracket (rare after LIN 1) are handled per column with a warp-uniform
+// ballot.  Masses are integers, so the cut does not depend on the order in
+// which threads add them.
 #include <math.h>
 
 #include "launch.h"
@@ -41,21 +50,46 @@
 
 namespace rtp {
 
-constexpr int kPfRows = 128;      // query rows per CTA (TMEM lanes)
-constexpr int kPfKeys = 64;       // keys per score tile (MMA N)
-constexpr int kPfStages = 2;      // K_idx tile ring
-constexpr int kPfBins = 32;       // histogram bins per row (also the candidate capacity)
-constexpr int kPfThreads = 192;   // 4 epilogue warps + producer + MMA
-constexpr int kPfTileBytes = kPfKeys * kIdxDim * 2;  // 2 KB
-constexpr int kPfTmemCols = 2 * kPfKeys;             // two accumulator buffers
+namespace {
 
-enum PfLevel : int { kLvMax = 0, kLvLin = 1, kLvCollect = 2, kLvKey = 3, kLvTie = 4, kLvDone = 5 };
+constexpr int kPfRows = 128;      // query rows per CTA (TMEM lanes)
+constexpr int kPfKeys = 128;      // keys per score tile (MMA N)
+constexpr int kPfStages = 4;      // K_idx tile ring
+constexpr int kPfBins = 32;       // histogram bins per row (also the candidate capacity)
+constexpr int kPfEpiWarps = 8;    // two per TMEM lane quadrant (column halves)
+constexpr int kPfProducerWarp = kPfEpiWarps;
+constexpr int kPfMmaWarp = kPfEpiWarps + 1;
+constexpr int kPfThreads = (kPfEpiWarps + 2) * 32;
+constexpr int kPfTileBytes = kPfKeys * kIdxDim * 2;  // 4 KB
+constexpr int kPfTmemCols = 2 * kPfKeys;             // two accumulator buffers
+constexpr int kPfMaxSweeps = 24;
+
+enum PfLevel : int { kLvMax, kLvLin0, kLvLin, kLvKey, kLvCollect, kLvTie, kLvMask, kLvDone };
+
+// The part of a row's state that its half-1 thread needs in the next sweep
+// (written by the row's half-0 thread after every sweep).
+struct PfRowState {
+  int level;
+  float m;         // raw row maximum
+  float vlo, vhi;  // bracket: raw accumulators v with vlo < v <= vhi
+  float dscale;    // LIN: 32^lin
+  int prefix;      // LIN: full bin index of the bracket at the previous level
+  uint32_t kbase;  // KEY: lowest score key of the digit range
+  int shift;       // KEY: digit shift
+  uint64_t kend;   // KEY: one past the highest score key
+  float vtau;      // MASK: raw accumulator of the cut score
+  int tiepos;      // MASK: last selected position among keys equal to the cut score
+};
 
 struct PfSmem {
-  alignas(256) uint8_t qtile[kPfRows * kIdxDim * 2];             // A operand, 4 KB
-  alignas(256) uint8_t ktile[kPfStages][kPfTileBytes];            // B operand ring
-  uint64_t hist[kPfBins][kPfRows];                                // per-row masses / candidates
-  uint16_t hcnt[kPfBins][kPfRows];                                // per-row counts (saturating)
+  alignas(1024) uint8_t qtile[kPfRows * kIdxDim * 2];  // A operand, 4 KB
+  alignas(1024) uint8_t ktile[kPfStages][kPfTileBytes];  // B operand ring
+  uint64_t hist[2][kPfBins][kPfRows];  // per half: bin masses, or candidates (COLLECT)
+  uint8_t hcnt[2][kPfBins][kPfRows];   // per half: bin counts (saturating at 255)
+  PfRowState rs[kPfRows];
+  float pmax[kPfRows];  // half 1's partial maximum
+  int pn[kPfRows];      // half 1's candidate count
+  int pgt[kPfRows];     // half 1's count of keys above the bracket
   uint64_t q_full;
   uint64_t k_full[kPfStages];
   uint64_t k_empty[kPfStages];
@@ -75,6 +109,7 @@ struct PfArgs {
   uint32_t* mask;
   int64_t mask_words;
   int* err;
+  long long budget;
 };
 
 // Fixed-point weight of a key at raw distance u = m - v from the row maximum:
@@ -85,10 +120,44 @@ RTP_DEVICE uint64_t pf_weight_u(float u, float wmul, float two_pow_frac) {
   return __float2ull_rn(__fmul_rn(e, two_pow_frac));
 }
 
+RTP_DEVICE float canon_score(float v) { return __fadd_rn(__fmul_rn(v, 0.25f), 0.0f); }
+
+RTP_DEVICE float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;\n" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// Level-0 bin of u: floor(u) clamped to [0, 31] (31 is the tail; NaN -> 0),
+// by rounding u + 2^23 down, which leaves floor(u) in the low mantissa bits.
+RTP_DEVICE int lin0_bin(float u) {
+  const float x = __fadd_rd(fminf(fmaxf(u, 0.f), 31.f), 8388608.f);
+  return __float_as_int(x) - 0x4B000000;
+}
+
+// The largest v with fsub_rn(m, v) >= u.  fsub_rn(m, v) does not increase
+// with v, so {v : lo <= fsub_rn(m, v) < hi} = (vmax(hi), vmax(lo)]; binary
+// search over the order-preserving integer image of the floats.
+RTP_DEVICE float vmax_u_ge(float m, float u) {
+  uint32_t lo = score_key(-INFINITY), hi = score_key(INFINITY);  // predicate true at lo, false at hi
+  while (hi - lo > 1u) {
+    const uint32_t mid = lo + ((hi - lo) >> 1);
+    if (__fsub_rn(m, key_score(mid)) >= u)
+      lo = mid;
+    else
+      hi = mid;
+  }
+  return key_score(lo);
+}
+
+RTP_DEVICE void hist_add(uint64_t* h, uint64_t w) { *h += w; }
+
+}  // namespace
+
 __global__ void __launch_bounds__(kPfThreads, 2)
 topp_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap, PfArgs A) {
-  extern __shared__ __align__(256) unsigned char smem_raw[];
-  PfSmem& S = *reinterpret_cast<PfSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 255) & ~uintptr_t(255));
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  PfSmem& S = *reinterpret_cast<PfSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   // 1-D grid ordered longest causal prefix first across all heads, so every SM
   // receives a mix of long and short blocks
@@ -103,7 +172,8 @@ topp_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
   // keys needed by the block: 0 .. position of its last token
   const int t_last = min(t0 + kPfRows, A.T) - 1;
   const int kmax = min(qbase + t_last, n_b - 1);
-  const int ntiles = kmax >= 0 ? (kmax + kPfKeys) / kPfKeys : 0;
+  const int ntiles = kmax >= 0 ? kmax / kPfKeys + 1 : 0;
+  const int64_t words = (A.N + 31) / 32;
 
   if (tid == 0) {
     mbar_init(&S.q_full, 1);
@@ -113,7 +183,7 @@ topp_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&S.t_full[i], 1);
-      mbar_init(&S.t_empty[i], kPfRows);
+      mbar_init(&S.t_empty[i], kPfEpiWarps);
     }
     mbar_fence_init();
   }
@@ -124,330 +194,431 @@ topp_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
   const uint32_t tmem = S.tmem_base;
   bool alive = true;
 
-  // ---- per-row state (epilogue threads) -------------------------------------
-  const int row = tid;  // valid for tid < 128
+  // ---- per-row state (epilogue threads) ---------------------------------------
+  const bool epi = warp < kPfEpiWarps;
+  const int quad = warp & 3, half = (warp >> 2) & 1;
+  const int row = quad * 32 + lane;
   const int t = t0 + row;
   const int pos = qbase + t;
-  const bool is_row = tid < kPfRows;
-  int level = (is_row && t < A.T && pos >= 0) ? kLvMax : kLvDone;
-  if (is_row && t < A.T && pos < 0) {  // a token before the sequence: no keys
-    const int64_t qrow = (int64_t)bh * A.T + t;
+  const bool owner = epi && half == 0;
+  const int64_t qrow = (int64_t)bh * A.T + t;
+  int level = (epi && t < A.T && pos >= 0) ? kLvMax : kLvDone;
+  uint32_t* mrow = (A.mask && epi && t < A.T) ? A.mask + qrow * A.mask_words : nullptr;
+  if (owner && t < A.T && pos < 0) {  // a token before the sequence: no keys
     A.tau_bits[qrow] = 0x7f800000u;
     A.tiepos[qrow] = -1;
     A.count[qrow] = 0;
+    if (mrow)
+      for (int64_t w = 0; w < words; ++w) mrow[w] = 0u;
   }
-  // Everything below works on raw accumulators v (the score is s = v / 4, an
-  // exact scaling): u = m - v with m the row's raw maximum.  Level-k bins are
-  // floor(u * 32^k) (level 0: floor(u), the tail folded into bin 31), so a
-  // level-k bin P is the interval [P / 32^k, (P + 1) / 32^k) of u, exactly.
-  float m = -INFINITY;
-  uint64_t target = 0, mass_above = 0;
-  int lin = 0, prefix = 0, tail = 0, shift = 0, n_tau = 0, ngt = 0, neq = 0, tiepos = -1, ncand = 0;
-  float ulo = 0.f, uhi = 0.f, dscale = 1.f;  // current bracket of u, and 32^lin
-  uint32_t kbase = 0, tau_key = 0;
+  float m = -INFINITY, vlo = 0.f, vhi = 0.f, dscale = 1.f, vtau = 0.f;
+  int prefix = 0, shift = 0, tiepos = -1, ngt = 0, neq = 0, ncand = 0;
+  uint32_t kbase = 0;
   uint64_t kend = 0;
+  // owner-only state
+  uint64_t target = 0, mass_above = 0;
+  int lin = 0, n_tau = 0;
+  uint32_t tau_key = 0;
   const float wmul = -0.25f * 1.4426950408889634f;  // weight 2^(u * wmul) = exp(-(m - v) / 4)
-  uint32_t* mrow = (A.mask && is_row && t < A.T) ? A.mask + ((int64_t)bh * A.T + t) * A.mask_words : nullptr;
 
-  uint32_t g = 0;  // global tile counter across sweeps (drives every ring phase)
-  for (int sweep = 0; sweep < 16; ++sweep) {
-    const int more = __syncthreads_or(is_row && level != kLvDone);
+  uint32_t g = 0;      // tiles consumed so far, over all sweeps (drives every ring phase)
+  uint32_t loads = 0;  // producer: K tiles issued
+  uint32_t mmas = 0;   // MMA issuer: MMAs issued
+  bool q_issued = false;
+  for (int sweep = 0; sweep < kPfMaxSweeps; ++sweep) {
+    const int more = __syncthreads_or(level != kLvDone);
     const int abort = __syncthreads_or(!alive);
     if (!more || abort || ntiles == 0) break;
-    if (is_row && level == kLvLin && lin == 0) dscale = 1.f;
-    if (is_row && (level == kLvLin || level == kLvKey))
+    if (epi && (level == kLvLin0 || level == kLvLin || level == kLvKey)) {
+#pragma unroll 4
       for (int i = 0; i < kPfBins; ++i) {
-        S.hist[i][row] = 0;
-        S.hcnt[i][row] = 0;
+        S.hist[half][i][row] = 0;
+        S.hcnt[half][i][row] = 0;
       }
-    if (is_row) {
-      ncand = 0;
-      if (level == kLvCollect) ngt = 0;
     }
+    ncand = 0;
+    if (level != kLvTie) ngt = 0;
+    if (level == kLvMax) m = -INFINITY;
 
-    if (warp == 4) {
+    if (warp == kPfProducerWarp) {
       // ---------------- TMA producer ----------------
       if (lane == 0) {
         if (sweep == 0) {
           mbar_expect_tx(&S.q_full, kPfRows * kIdxDim * 2);
           tma_load_4d(S.qtile, &qmap, &S.q_full, 0, t0, h, b);
+          q_issued = true;
         }
         for (int i = 0; i < ntiles; ++i) {
           const uint32_t gi = g + i, st = gi % kPfStages, ph = (gi / kPfStages) & 1;
-          if (!mbar_wait(&S.k_empty[st], ph ^ 1, alive, A.err)) break;
+          if (!mbar_wait(&S.k_empty[st], ph ^ 1, alive, A.err, A.budget)) break;
           mbar_expect_tx(&S.k_full[st], kPfTileBytes);
           tma_load_4d(S.ktile[st], &kmap, &S.k_full[st], 0, i * kPfKeys, kvh, b);
+          loads = gi + 1;
         }
       }
-    } else if (warp == 5) {
+    } else if (warp == kPfMmaWarp) {
       // ---------------- MMA issuer ----------------
       if (lane == 0) {
-        if (sweep == 0) mbar_wait(&S.q_full, 0, alive, A.err);
+        if (sweep == 0) mbar_wait(&S.q_full, 0, alive, A.err, A.budget);
         const uint64_t adesc = umma_desc_k_sw32(S.qtile);
         constexpr uint32_t idesc = umma_idesc_bf16_f32(kPfRows, kPfKeys);
         for (int i = 0; i < ntiles; ++i) {
           const uint32_t gi = g + i, st = gi % kPfStages, buf = gi & 1;
-          if (!mbar_wait(&S.k_full[st], (gi / kPfStages) & 1, alive, A.err)) break;
-          if (!mbar_wait(&S.t_empty[buf], ((gi >> 1) & 1) ^ 1, alive, A.err)) break;
+          if (!mbar_wait(&S.k_full[st], (gi / kPfStages) & 1, alive, A.err, A.budget)) break;
+          if (!mbar_wait(&S.t_empty[buf], ((gi >> 1) & 1) ^ 1, alive, A.err, A.budget)) break;
           tc_fence_after();
           umma_f16(tmem + buf * kPfKeys, adesc, umma_desc_k_sw32(S.ktile[st]), idesc, 0);
           umma_commit(&S.k_empty[st]);
           umma_commit(&S.t_full[buf]);
+          mmas = gi + 1;
         }
       }
     } else {
-      // ---------------- epilogue: one query row per thread ----------------
+      // ---------------- epilogue: two threads per query row ----------------
       const float mh = m;
+      const bool bracket = level == kLvLin || level == kLvKey || level == kLvCollect;
       for (int i = 0; i < ntiles; ++i) {
         const uint32_t gi = g + i, buf = gi & 1;
-        if (!mbar_wait(&S.t_full[buf], (gi >> 1) & 1, alive, A.err)) break;
+        const bool ok = __all_sync(0xffffffffu, mbar_wait(&S.t_full[buf], (gi >> 1) & 1, alive, A.err, A.budget));
+        if (!ok) {
+          alive = false;
+          break;
+        }
         tc_fence_after();
-        const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16) + buf * kPfKeys;
-        const int key0 = i * kPfKeys;
-        uint64_t mbits = 0ull;
+        const uint32_t tb = tmem + ((uint32_t)(quad * 32) << 16) + buf * kPfKeys;
+        // a TIE row is finished by its half-0 thread alone, over all 128 columns in position order
+        const bool tie_warp = half == 0 && __any_sync(0xffffffffu, level == kLvTie);
+        const int nch = tie_warp ? 4 : 2;
 #pragma unroll 1
-        for (int half = 0; half < 2; ++half) {  // two chunks of 32 columns
+        for (int c = 0; c < nch; ++c) {
+          const int col = tie_warp ? 32 * c : 64 * half + 32 * c;
           uint32_t v[32];
-          tmem_ld32(taddr + half * 32, v);
+          tmem_ld32(tb + col, v);
           tmem_ld_wait();
-          if (half == 1) {
+          if (c == nch - 1) {
             tc_fence_before();
-            mbar_arrive(&S.t_empty[buf]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&S.t_empty[buf]);
           }
-          if (level == kLvDone) continue;
-          const int kb = key0 + half * 32;
+          const int kb = i * kPfKeys + col;
           const int nv = pos - kb + 1;  // keys of this chunk inside the row's causal prefix
-          if (nv <= 0) continue;
+          const bool own = (col >> 6) == half;
+          const uint32_t vmask = nv >= 32 ? 0xffffffffu : (nv > 0 ? (1u << nv) - 1u : 0u);
           if (level == kLvMax) {
-            if (nv >= 32) {
+            if (own && nv > 0) {
+              float a0 = -INFINITY, a1 = -INFINITY, a2 = -INFINITY, a3 = -INFINITY;
+              if (nv >= 32) {
 #pragma unroll
-              for (int j = 0; j < 32; ++j) m = fmaxf(m, __uint_as_float(v[j]));
-            } else {
-#pragma unroll
-              for (int j = 0; j < 32; ++j)
-                if (j < nv) m = fmaxf(m, __uint_as_float(v[j]));
-            }
-          } else if (level == kLvTie) {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              if (j < nv) {
-                const float sv = __fadd_rn(__fmul_rn(__uint_as_float(v[j]), 0.25f), 0.0f);
-                const uint32_t k = score_key(sv);
-                const bool gt = k > tau_key;
-                bool sel = gt;
-                ngt += gt;
-                if (k == tau_key) {
-                  ++neq;
-                  sel = neq <= n_tau;
-                  if (neq == n_tau) tiepos = kb + j;
+                for (int q = 0; q < 4; ++q) {
+                  a0 = max3f(a0, __uint_as_float(v[8 * q + 0]), __uint_as_float(v[8 * q + 1]));
+                  a1 = max3f(a1, __uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3]));
+                  a2 = max3f(a2, __uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5]));
+                  a3 = max3f(a3, __uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7]));
                 }
-                mbits |= (uint64_t)sel << (half * 32 + j);
+              } else {
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                  if (j < nv) a0 = fmaxf(a0, __uint_as_float(v[j]));
+              }
+              m = max3f(m, max3f(a0, a1, a2), a3);
+            }
+          } else if (level == kLvLin0) {
+            if (own && nv > 0) {
+              // every key lands in a bin; consecutive keys are taken in pairs so that the two
+              // read-modify-writes overlap (a pair in one bin is added as one update)
+              uint64_t* H = &S.hist[half][0][row];
+#pragma unroll
+              for (int j = 0; j < 32; j += 2) {
+                const float u0 = __fsub_rn(mh, __uint_as_float(v[j]));
+                const float u1 = __fsub_rn(mh, __uint_as_float(v[j + 1]));
+                const int d0 = lin0_bin(u0), d1 = lin0_bin(u1);
+                const uint64_t w0 = j < nv ? pf_weight_u(u0, wmul, A.two_pow_frac) : 0ull;
+                const uint64_t w1 = j + 1 < nv ? pf_weight_u(u1, wmul, A.two_pow_frac) : 0ull;
+                const uint64_t h0 = H[d0 * kPfRows], h1 = H[d1 * kPfRows];
+                const bool same = d0 == d1;
+                const uint64_t s0 = h0 + w0 + (same ? w1 : 0ull);
+                const uint64_t s1 = same ? s0 : h1 + w1;
+                H[d0 * kPfRows] = s0;
+                H[d1 * kPfRows] = s1;
               }
             }
-          } else if (level == kLvLin && lin == 0) {
-            // every key lands in a bin; Z is the sum of the bins afterwards
-            const int nvc = nv < 32 ? nv : 32;
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              if (j < nvc) {
-                const float u = __fsub_rn(mh, __uint_as_float(v[j]));
-                const int d = u >= 31.f ? 31 : (u > 0.f ? (int)u : 0);  // also 0 for a NaN input
-                S.hist[d][row] += pf_weight_u(u, wmul, A.two_pow_frac);
-              }
-            }
-          } else if (level == kLvLin || level == kLvCollect) {
-            // keys inside the bracket [ulo, uhi) of u (two compares each); most chunks have none
-            uint32_t in = 0u;
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const float u = __fsub_rn(mh, __uint_as_float(v[j]));
-              const bool ok = j < nv;
-              in |= (uint32_t)(ok && u >= ulo && u < uhi) << j;
-              if (level == kLvCollect) ngt += ok && u < ulo;  // keys above the bracket
-            }
-            if (in) {
+          }
+          {
+            // bracket levels: two compares per key, keys inside handled column by column.  The
+            // warp-wide votes below are reached by every lane whatever its row's level.
+            uint32_t inb = 0u, above = 0u;
+            if (bracket && own) {
 #pragma unroll
               for (int j = 0; j < 32; ++j) {
-                if ((in >> j) & 1u) {
-                  const float u = __fsub_rn(mh, __uint_as_float(v[j]));
-                  if (level == kLvLin) {
-                    const int d = (int)__fmul_rn(u, dscale) - 32 * prefix;
-                    S.hist[d][row] += pf_weight_u(u, wmul, A.two_pow_frac);
-                    const uint16_t cc = S.hcnt[d][row];
-                    S.hcnt[d][row] = cc == 0xFFFFu ? cc : (uint16_t)(cc + 1u);
-                  } else if (ncand < kPfBins) {
-                    const float sv = __fadd_rn(__fmul_rn(__uint_as_float(v[j]), 0.25f), 0.0f);
-                    S.hist[ncand][row] = ((uint64_t)(uint32_t)(kb + j) << 32) | __float_as_uint(sv);
-                    ++ncand;
+                const float x = __uint_as_float(v[j]);
+                inb |= (uint32_t)(x > vlo && x <= vhi) << j;
+                above |= (uint32_t)(x > vhi) << j;
+              }
+              inb &= vmask;
+              if (level == kLvCollect) ngt += __popc(above & vmask);
+            }
+            if (__any_sync(0xffffffffu, inb != 0u)) {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) {
+                if (__ballot_sync(0xffffffffu, (inb >> j) & 1u) == 0u) continue;
+                if (!((inb >> j) & 1u)) continue;
+                const float x = __uint_as_float(v[j]);
+                const float u = __fsub_rn(mh, x);
+                if (level == kLvLin) {
+                  const int d = min(max((int)__fmul_rn(u, dscale) - 32 * prefix, 0), kPfBins - 1);
+                  hist_add(&S.hist[half][d][row], pf_weight_u(u, wmul, A.two_pow_frac));
+                  const uint8_t cc = S.hcnt[half][d][row];
+                  S.hcnt[half][d][row] = cc == 255 ? cc : (uint8_t)(cc + 1);
+                } else if (level == kLvKey) {
+                  const uint32_t k = score_key(canon_score(x));
+                  if (k >= kbase && (uint64_t)k < kend) {
+                    const int d = (int)((k - kbase) >> shift);
+                    hist_add(&S.hist[half][d][row], pf_weight_u(u, wmul, A.two_pow_frac));
                   }
+                } else {  // COLLECT
+                  if (ncand < kPfBins)
+                    S.hist[half][ncand][row] = ((uint64_t)(uint32_t)(kb + j) << 32) | __float_as_uint(x);
+                  ++ncand;
                 }
               }
             }
-          } else {  // KEY fallback: exact digits of the score key inside the bracket
-            const int nvc = nv < 32 ? nv : 32;
+            if (level == kLvMask && own) {
+              uint32_t bits = 0u;
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              if (j < nvc) {
-                const float u = __fsub_rn(mh, __uint_as_float(v[j]));
-                const bool inb = tail ? u >= 31.f : (u >= ulo && u < uhi);
-                const float sv = __fadd_rn(__fmul_rn(__uint_as_float(v[j]), 0.25f), 0.0f);
-                const uint32_t k = score_key(sv);
-                if (inb && k >= kbase && (uint64_t)k < kend) {
-                  const int d = (int)((k - kbase) >> shift);
-                  S.hist[d][row] += pf_weight_u(u, wmul, A.two_pow_frac);
+              for (int j = 0; j < 32; ++j) {
+                const float x = __uint_as_float(v[j]);
+                bits |= (uint32_t)(x > vtau || (x == vtau && kb + j <= tiepos)) << j;
+              }
+              bits &= vmask;
+              if ((kb >> 5) < A.mask_words) mrow[kb >> 5] = bits;
+            } else if (level == kLvTie && half == 0) {
+              uint32_t bits = 0u;
+#pragma unroll
+              for (int j = 0; j < 32; ++j) {
+                if (j < nv) {
+                  const float x = __uint_as_float(v[j]);
+                  const bool gt = x > vtau;
+                  bool sel = gt;
+                  ngt += gt;
+                  if (x == vtau) {
+                    ++neq;
+                    sel = neq <= n_tau;
+                    if (neq == n_tau) tiepos = kb + j;
+                  }
+                  bits |= (uint32_t)sel << j;
                 }
               }
+              if (mrow && (kb >> 5) < A.mask_words) mrow[kb >> 5] = bits;
             }
           }
-        }
-        if (level == kLvTie && mrow) {
-          const int w0 = key0 >> 5;
-          if (w0 < A.mask_words) mrow[w0] = (uint32_t)mbits;
-          if (w0 + 1 < A.mask_words) mrow[w0 + 1] = (uint32_t)(mbits >> 32);
         }
       }
-      // ---- end of sweep: advance this row's bracket ----
-      if (is_row && level != kLvDone && alive) {
-        if (level == kLvMax) {
-          level = kLvLin;  // m is the raw maximum
-          lin = 0;
-          prefix = 0;
-        } else if (level == kLvTie) {
-          if (mrow)  // words past the block's last tile
-            for (int64_t w = 2 * (int64_t)ntiles; w < (A.N + 31) / 32; ++w) mrow[w] = 0u;
-          const int64_t qrow = (int64_t)bh * A.T + t;
-          A.tau_bits[qrow] = __float_as_uint(key_score(tau_key));
-          A.tiepos[qrow] = tiepos;
-          A.count[qrow] = ngt + n_tau;
-          level = kLvDone;
-        } else if (level == kLvCollect) {
-          // sort the candidates by (score desc, position asc), then take them in order
-          for (int a = 1; a < ncand; ++a) {
-            const uint64_t x = S.hist[a][row];
-            const uint32_t xk = score_key(__uint_as_float((uint32_t)x));
-            const uint32_t xp = (uint32_t)(x >> 32);
-            int bI = a - 1;
-            while (bI >= 0) {
-              const uint64_t y = S.hist[bI][row];
-              const uint32_t yk = score_key(__uint_as_float((uint32_t)y));
-              if (yk > xk || (yk == xk && (uint32_t)(y >> 32) < xp)) break;
-              S.hist[bI + 1][row] = y;
-              --bI;
-            }
-            S.hist[bI + 1][row] = x;
+      if (half == 1) {
+        S.pmax[row] = m;
+        S.pn[row] = ncand;
+        S.pgt[row] = ngt;
+      }
+    }
+    g += ntiles;
+    __syncthreads();  // both halves' partial results are in shared memory
+
+    // ---- end of sweep: the row's half-0 thread advances its bracket ----
+    if (owner && level != kLvDone && alive) {
+      if (level == kLvMax) {
+        m = fmaxf(m, S.pmax[row]);  // m is the raw maximum
+        level = kLvLin0;
+      } else if (level == kLvTie) {
+        const int64_t w_end = 4 * (int64_t)ntiles;
+        if (mrow)  // words past the block's last tile
+          for (int64_t w = w_end; w < words; ++w) mrow[w] = 0u;
+        A.tau_bits[qrow] = __float_as_uint(key_score(tau_key));
+        A.tiepos[qrow] = tiepos;
+        A.count[qrow] = ngt + min(n_tau, neq);
+        level = kLvDone;
+      } else if (level == kLvMask) {
+        if (mrow)
+          for (int64_t w = 4 * (int64_t)ntiles; w < words; ++w) mrow[w] = 0u;
+        level = kLvDone;
+      } else if (level == kLvCollect) {
+        // both halves' candidates, sorted by (score desc, position asc), taken in order
+        const int n0 = min(ncand, kPfBins);
+        const int n1 = min(S.pn[row], kPfBins - n0);
+        for (int a = 0; a < n1; ++a) S.hist[0][n0 + a][row] = S.hist[1][a][row];
+        const int n = n0 + n1;
+        const int gt_all = ngt + S.pgt[row];
+        for (int a = 1; a < n; ++a) {
+          const uint64_t x = S.hist[0][a][row];
+          const float xv = __uint_as_float((uint32_t)x);
+          const uint32_t xp = (uint32_t)(x >> 32);
+          int bI = a - 1;
+          while (bI >= 0) {
+            const uint64_t y = S.hist[0][bI][row];
+            const float yv = __uint_as_float((uint32_t)y);
+            if (yv > xv || (yv == xv && (uint32_t)(y >> 32) < xp)) break;
+            S.hist[0][bI + 1][row] = y;
+            --bI;
           }
-          const uint64_t need = target - mass_above;
-          uint64_t cum = 0;
-          int taken = ncand;
-          for (int a = 0; a < ncand; ++a) {
-            const float sa = __uint_as_float((uint32_t)S.hist[a][row]);
-            cum += pf_weight_u(__fsub_rn(mh, __fmul_rn(sa, 4.f)), wmul, A.two_pow_frac);
-            if (cum >= need) {
-              taken = a + 1;
-              break;
+          S.hist[0][bI + 1][row] = x;
+        }
+        const uint64_t need = target - mass_above;
+        uint64_t cum = 0;
+        int taken = n;
+        for (int a = 0; a < n; ++a) {
+          cum += pf_weight_u(__fsub_rn(m, __uint_as_float((uint32_t)S.hist[0][a][row])), wmul, A.two_pow_frac);
+          if (cum >= need) {
+            taken = a + 1;
+            break;
+          }
+        }
+        if (taken < 1) taken = 1;
+        const uint64_t last = S.hist[0][taken - 1][row];
+        vtau = __uint_as_float((uint32_t)last);
+        tiepos = (int)(last >> 32);
+        A.tau_bits[qrow] = __float_as_uint(canon_score(vtau));
+        A.tiepos[qrow] = tiepos;
+        A.count[qrow] = gt_all + taken;
+        level = mrow ? kLvMask : kLvDone;  // the selection mask needs one more sweep
+      } else {  // LIN0, LIN or KEY: find the cut bin
+        if (level == kLvLin0) {
+          uint64_t Z = 0;
+          for (int i = 0; i < kPfBins; ++i) {
+            const uint64_t hv = S.hist[0][i][row] + S.hist[1][i][row];
+            S.hist[0][i][row] = hv;
+            Z += hv;
+          }
+          const double tt = ceil((double)A.p * (double)Z);
+          const uint64_t tg = tt >= (double)Z ? Z : (uint64_t)tt;
+          target = tg < 1 ? 1 : tg;
+        } else {
+          for (int i = 0; i < kPfBins; ++i) {
+            S.hist[0][i][row] += S.hist[1][i][row];
+            const int cc = (int)S.hcnt[0][i][row] + (int)S.hcnt[1][i][row];
+            S.hcnt[0][i][row] = (uint8_t)(cc > 255 ? 255 : cc);
+          }
+        }
+        // the first bin (in score order) where the cumulative mass reaches the target; should
+        // rounding ever leave it short, the last non-empty bin
+        const uint64_t need = target - mass_above;
+        uint64_t cum = 0, cum_nz = 0;
+        int cut = -1, last_nz = level == kLvKey ? kPfBins - 1 : 0;
+        for (int r = 0; r < kPfBins; ++r) {
+          const int bin = level == kLvKey ? kPfBins - 1 - r : r;
+          const uint64_t hv = S.hist[0][bin][row];
+          if (hv) {
+            last_nz = bin;
+            cum_nz = cum;
+          }
+          if (cum + hv >= need) {
+            cut = bin;
+            break;
+          }
+          cum += hv;
+        }
+        if (cut < 0) {
+          cut = last_nz;
+          cum = cum_nz;
+        }
+        mass_above += cum;
+        if (level == kLvLin0 || level == kLvLin) {
+          if (level == kLvLin0 && cut == kPfBins - 1) {
+            // tail bin (u >= 31, i.e. s <= max s - 7.75): exact digits over its keys
+            const float hi_s = __fmul_rn(__fsub_rn(m, 31.f), 0.25f);
+            const float mg = 1e-5f * (fabsf(hi_s) + 8.f) + 1e-30f;
+            kbase = 0u;
+            kend = (uint64_t)score_key(__fadd_rn(hi_s + mg, 0.0f)) + 1;
+            shift = 0;
+            while (((kend - kbase - 1) >> shift) >= (uint64_t)kPfBins) ++shift;
+            vlo = -INFINITY;
+            vhi = vmax_u_ge(m, 31.f);
+            level = kLvKey;
+          } else {
+            const int in_bin = level == kLvLin0 ? 255 : (int)S.hcnt[0][cut][row];  // level 0 keeps no counts
+            prefix = level == kLvLin0 ? cut : 32 * prefix + cut;  // full bin index at level `lin`
+            const float ulo = (float)prefix / dscale;             // exact: dscale is a power of two
+            const float uhi = (float)(prefix + 1) / dscale;
+            vlo = vmax_u_ge(m, uhi);
+            vhi = vmax_u_ge(m, ulo);
+            if (in_bin <= kPfBins) {
+              level = kLvCollect;
+            } else if (lin < 3) {
+              ++lin;
+              dscale *= 32.f;
+              level = kLvLin;
+            } else {
+              // still too many keys: exact digits inside this bracket of u
+              const float hi_s = __fmul_rn(__fsub_rn(m, ulo), 0.25f);
+              const float lo_s = __fmul_rn(__fsub_rn(m, uhi), 0.25f);
+              const float mg = 1e-5f * (fabsf(hi_s) + fabsf(lo_s) + uhi) + 1e-30f;
+              kbase = score_key(__fadd_rn(lo_s - mg, 0.0f));
+              kend = (uint64_t)score_key(__fadd_rn(hi_s + mg, 0.0f)) + 1;
+              shift = 0;
+              while (((kend - kbase - 1) >> shift) >= (uint64_t)kPfBins) ++shift;
+              level = kLvKey;
             }
           }
-          if (taken < 1) taken = 1;
-          const uint64_t last = S.hist[taken - 1][row];
-          tau_key = score_key(__uint_as_float((uint32_t)last));
-          n_tau = 0;
-          for (int a = 0; a < taken; ++a) n_tau += score_key(__uint_as_float((uint32_t)S.hist[a][row])) == tau_key;
-          const int cnt = ngt + taken;
-          if (mrow) {  // the selection mask needs one more sweep
+        } else {  // KEY
+          kbase += (uint32_t)cut << shift;
+          const uint64_t e = (uint64_t)kbase + (uint64_t(1) << shift);
+          kend = e < kend ? e : kend;
+          if (shift == 0) {
+            tau_key = kbase;
+            const float st = key_score(tau_key);
+            const uint64_t w_tau = pf_weight_u(__fsub_rn(m, __fmul_rn(st, 4.f)), wmul, A.two_pow_frac);
+            const uint64_t rem = target - mass_above;
+            const uint64_t nt = w_tau ? (rem + w_tau - 1) / w_tau : 1;
+            n_tau = (int)(nt < 1 ? 1 : (nt > 0x7fffffffull ? 0x7fffffffull : nt));
+            vtau = __fmul_rn(st, 4.f);
             ngt = 0;
             neq = 0;
             tiepos = -1;
             level = kLvTie;
           } else {
-            const int64_t qrow = (int64_t)bh * A.T + t;
-            A.tau_bits[qrow] = __float_as_uint(key_score(tau_key));
-            A.tiepos[qrow] = (int)(last >> 32);
-            A.count[qrow] = cnt;
-            level = kLvDone;
-          }
-        } else {  // LIN or KEY: find the cut bin
-          if (level == kLvLin && lin == 0) {
-            uint64_t Z = 0;
-            for (int i = 0; i < kPfBins; ++i) Z += S.hist[i][row];
-            const double tt = ceil((double)A.p * (double)Z);
-            uint64_t tg = tt >= (double)Z ? Z : (uint64_t)tt;
-            target = tg < 1 ? 1 : tg;
-          }
-          const uint64_t need = target - mass_above;
-          uint64_t cum = 0;
-          int cut = 0;
-          for (int r = 0; r < kPfBins; ++r) {
-            const int bin = level == kLvKey ? kPfBins - 1 - r : r;
-            const uint64_t hv = S.hist[bin][row];
-            if (cum + hv >= need) {
-              cut = bin;
-              break;
-            }
-            cum += hv;
-          }
-          mass_above += cum;
-          if (level == kLvLin) {
-            if (lin == 0 && cut == 31) {
-              // tail bin (u >= 31, i.e. s <= max s - 7.75): exact digits over its keys
-              tail = 1;
-              const float hi_s = __fmul_rn(__fsub_rn(mh, 31.f), 0.25f);
-              const float mg = 1e-5f * (fabsf(hi_s) + 8.f) + 1e-30f;
-              kbase = 0u;
-              kend = (uint64_t)score_key(__fadd_rn(hi_s + mg, 0.0f)) + 1;
-              shift = 0;
-              while (((kend - kbase - 1) >> shift) >= (uint64_t)kPfBins) ++shift;
-              level = kLvKey;
-            } else {
-              const uint32_t in_bin = lin == 0 ? 0xFFFFu : S.hcnt[cut][row];  // level 0 keeps no counts
-              prefix = lin == 0 ? cut : 32 * prefix + cut;  // full bin index at level `lin`
-              ulo = (float)prefix / dscale;                  // exact: dscale is a power of two
-              uhi = (float)(prefix + 1) / dscale;
-              if (in_bin <= (uint32_t)kPfBins) {
-                level = kLvCollect;
-              } else if (lin < 3) {
-                ++lin;
-                dscale *= 32.f;
-              } else {
-                // still too many keys: exact digits inside this bracket of u
-                const float hi_s = __fmul_rn(__fsub_rn(mh, ulo), 0.25f);
-                const float lo_s = __fmul_rn(__fsub_rn(mh, uhi), 0.25f);
-                const float mg = 1e-5f * (fabsf(hi_s) + fabsf(lo_s) + uhi) + 1e-30f;
-                kbase = score_key(__fadd_rn(lo_s - mg, 0.0f));
-                kend = (uint64_t)score_key(__fadd_rn(hi_s + mg, 0.0f)) + 1;
-                shift = 0;
-                while (((kend - kbase - 1) >> shift) >= (uint64_t)kPfBins) ++shift;
-                level = kLvKey;
-              }
-            }
-          } else {  // KEY
-            kbase += (uint32_t)cut << shift;
-            const uint64_t e = (uint64_t)kbase + (uint64_t(1) << shift);
-            kend = e < kend ? e : kend;
-            if (shift == 0) {
-              tau_key = kbase;
-              const float st = key_score(tau_key);
-              const uint64_t w_tau = pf_weight_u(__fsub_rn(mh, __fmul_rn(st, 4.f)), wmul, A.two_pow_frac);
-              const uint64_t rem = target - mass_above;
-              uint64_t nt = w_tau ? (rem + w_tau - 1) / w_tau : 1;
-              n_tau = (int)(nt < 1 ? 1 : nt);
-              ngt = 0;
-              neq = 0;
-              tiepos = -1;
-              level = kLvTie;
-            } else {
-              shift = shift >= 5 ? shift - 5 : 0;
-            }
+            shift = shift >= 5 ? shift - 5 : 0;
           }
         }
       }
     }
-    g += ntiles;
+    if (owner) {
+      PfRowState& R = S.rs[row];
+      R.level = level;
+      R.m = m;
+      R.vlo = vlo;
+      R.vhi = vhi;
+      R.dscale = dscale;
+      R.prefix = prefix;
+      R.kbase = kbase;
+      R.shift = shift;
+      R.kend = kend;
+      R.vtau = vtau;
+      R.tiepos = tiepos;
+    }
+    __syncthreads();
+    if (epi && half == 1) {
+      const PfRowState& R = S.rs[row];
+      level = R.level;
+      m = R.m;
+      vlo = R.vlo;
+      vhi = R.vhi;
+      dscale = R.dscale;
+      prefix = R.prefix;
+      kbase = R.kbase;
+      shift = R.shift;
+      kend = R.kend;
+      vtau = R.vtau;
+      tiepos = R.tiepos;
+    }
   }
 
-  // ---- wind down: the last accumulator commit has landed before TMEM is freed
-  if (warp == 5 && lane == 0 && g > 0) {
-    const uint32_t last = g - 1;
-    mbar_wait(&S.t_full[last & 1], (last >> 1) & 1, alive, A.err);
+  // ---- wind down: every copy and MMA this CTA issued lands before its tensor
+  // memory is freed and it exits, even after a wait gave up
+  if (warp == kPfMmaWarp && lane == 0 && mmas > 0) {
+    const uint32_t last = mmas - 1;
+    mbar_drain(&S.t_full[last & 1], (last >> 1) & 1, A.err);
+  }
+  if (warp == kPfProducerWarp && lane == 0) {
+    if (q_issued) mbar_drain(&S.q_full, 0, A.err);
+    for (uint32_t i = loads > (uint32_t)kPfStages ? loads - kPfStages : 0u; i < loads; ++i)
+      mbar_drain(&S.k_full[i % kPfStages], (i / kPfStages) & 1, A.err);
   }
   tc_fence_before();
   __syncthreads();
@@ -476,36 +647,7 @@ __global__ void topp_prefill_all_kernel(PfArgs A, int rows) {
   }
 }
 
-// ---- host ---------------------------------------------------------------------
-static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
-  return fn;
-}
-
-// Tensor map over a [B, H, R, 16] bf16 view, box of `box_rows` rows, 32-byte swizzle.
-bool make_idx_map(CUtensorMap* map, const View4& v, int64_t B, int64_t H, int64_t R, int box_rows) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[4] = {16, (cuuint64_t)R, (cuuint64_t)H, (cuuint64_t)B};
-  cuuint64_t st1 = (cuuint64_t)v.sn * 2, st2 = (cuuint64_t)v.sh * 2, st3 = (cuuint64_t)v.sb * 2;
-  if (R <= 1) st1 = 32;
-  if (H <= 1) st2 = st1 * (cuuint64_t)(R > 0 ? R : 1);
-  if (B <= 1) st3 = st2 * (cuuint64_t)(H > 0 ? H : 1);
-  cuuint64_t strides[3] = {st1, st2, st3};
-  cuuint32_t box[4] = {16, (cuuint32_t)box_rows, 1, 1};
-  cuuint32_t estr[4] = {1, 1, 1, 1};
-  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(v.data), dims, strides, box,
-                        estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B,
-                        CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
+// ---- host side ------------------------------------------------------------------
 
 cudaError_t launch_topp_prefill(const LaunchToppPrefill& a, cudaStream_t stream) {
   const int64_t rows = a.B * a.Hq * a.T;
@@ -527,6 +669,7 @@ cudaError_t launch_topp_prefill(const LaunchToppPrefill& a, cudaStream_t stream)
   A.mask = a.mask;
   A.mask_words = a.mask_words;
   A.err = a.err;
+  A.budget = wait_budget_cycles();
   if (a.p >= 1.f) {
     topp_prefill_all_kernel<<<(unsigned)((rows + 255) / 256), 256, 0, stream>>>(A, (int)rows);
     return cudaGetLastError();
@@ -534,8 +677,9 @@ cudaError_t launch_topp_prefill(const LaunchToppPrefill& a, cudaStream_t stream)
   CUtensorMap qmap, kmap;
   if (!make_idx_map(&qmap, a.q_idx, a.B, a.Hq, a.T, kPfRows)) return cudaErrorInvalidValue;
   if (!make_idx_map(&kmap, a.k_idx, a.B, a.Hk, a.N, kPfKeys)) return cudaErrorInvalidValue;
-  const size_t smem = sizeof(PfSmem) + 256;
+  const size_t smem = sizeof(PfSmem) + 1024;
   cudaFuncSetAttribute(topp_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaFuncSetAttribute(topp_prefill_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
   const dim3 grid((unsigned)(((a.T + kPfRows - 1) / kPfRows) * a.B * a.Hq));
   topp_prefill_kernel<<<grid, kPfThreads, smem, stream>>>(qmap, kmap, A);
   return cudaGetLastError();

@@ -27,7 +27,8 @@ EXPORTED = ("rtp_index_project", "rtp_topp_select", "rtp_topp_select_workspace_s
             "rtp_sparse_attn_decode", "rtp_sparse_attn_decode_workspace_size", "rtp_sparse_attn_decode_noalloc",
             "rtp_sparse_attn_prefill", "rtp_sparse_attn_prefill_workspace_size",
             "rtp_window_attn", "rtp_window_attn_workspace_size",
-            "rtp_poll_device_error", "rtp_status_string", "rtp_last_cuda_error", "rtp_version")
+            "rtp_poll_device_error", "rtp_set_wait_budget_cycles", "rtp_status_string", "rtp_last_cuda_error",
+            "rtp_version")
 
 
 class RtpTensor(ctypes.Structure):
@@ -68,6 +69,7 @@ def _load() -> ctypes.CDLL:
         "rtp_window_attn": ([T, T, T, vp, i32, f32, T, vp, sz, vp], i32),
         "rtp_window_attn_workspace_size": ([i64, i64, i64, i64, i64, i32], sz),
         "rtp_poll_device_error": ([P(i32)], i32),
+        "rtp_set_wait_budget_cycles": ([i64], i32),
         "rtp_status_string": ([i32], ctypes.c_char_p),
         "rtp_last_cuda_error": ([], i32),
         "rtp_version": ([], i32),
@@ -304,6 +306,11 @@ def poll_device_error() -> int:
     code = ctypes.c_int32(0)
     _check(_lib.rtp_poll_device_error(ctypes.byref(code)), "rtp_poll_device_error")
     return int(code.value)
+
+
+def set_wait_budget_cycles(cycles: int) -> None:
+    """Budget of each bounded device wait in later prefill launches (0 = default)."""
+    _check(_lib.rtp_set_wait_budget_cycles(int(cycles)), "rtp_set_wait_budget_cycles")
 
 
 def version() -> int:

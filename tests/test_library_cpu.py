@@ -268,3 +268,42 @@ def test_header_is_plain_c_and_links_against_the_library(tmp_path):
                         "-L", libdir, "-lrtp", "-Wl,-rpath," + libdir, "-o", str(exe)], capture_output=True, text=True)
     assert r.returncode == 0, r.stderr
     assert subprocess.run([str(exe)]).returncode == 0
+
+
+def test_noalloc_scratch_size_matches_the_header():
+    # the Python wrapper's copy of RTP_NOALLOC_SCRATCH_BYTES is the header's value
+    rtp = _lib()
+    with open(os.path.join(ROOT, "include", "rtp.h")) as f:
+        m = re.search(r"#define\s+RTP_NOALLOC_SCRATCH_BYTES\s+\((\d+)u\s*<<\s*(\d+)\)", f.read())
+    assert m, "RTP_NOALLOC_SCRATCH_BYTES not found in rtp.h"
+    assert int(m.group(1)) << int(m.group(2)) == rtp.NOALLOC_SCRATCH_BYTES
+
+
+def test_noalloc_validates_before_touching_the_device():
+    # on a machine without a GPU any CUDA call would fail with RTP_ERR_CUDA (6):
+    # an invalid call must be refused by the argument checks alone
+    rtp = _lib()
+    L = rtp.lib()
+    by = ctypes.byref
+    q = _desc(rtp, [2, 8, 1, 128])
+    k = _desc(rtp, [2, 2, 64, 128])
+    o = _desc(rtp, [2, 8, 1, 128], dtype=0)
+    s = _sel(rtp)
+    fn = L.rtp_sparse_attn_decode_noalloc
+    assert fn(by(q), by(k), by(k), None, None, 0.088, by(o), None) == 1                       # no selection
+    assert fn(by(q), by(k), by(k), None, by(_sel(rtp, mask=False)), 0.088, by(o), None) == 1  # no mask
+    assert fn(by(q), by(k), by(k), None, by(s), float("nan"), by(o), None) == 1               # bad scale
+    assert fn(by(_desc(rtp, [2, 8, 2, 128])), by(k), by(k), None, by(s), 0.088,
+              by(_desc(rtp, [2, 8, 2, 128], dtype=0)), None) == 2                             # T != 1
+    assert fn(by(q), by(k), by(_desc(rtp, [2, 2, 64, 128], dtype=0)), None, by(s), 0.088, by(o), None) == 3
+    big = _desc(rtp, [4096, 32, 1, 128])
+    kv = _desc(rtp, [4096, 8, 4096, 128])
+    assert fn(by(big), by(kv), by(kv), None, by(_sel(rtp, words=128)), 0.088,
+              by(_desc(rtp, [4096, 32, 1, 128], dtype=0)), None) == 7                         # beyond the scratch
+
+
+def test_wait_budget_setter_validates():
+    rtp = _lib()
+    with pytest.raises(rtp.RtpError):
+        rtp.set_wait_budget_cycles(-1)
+    rtp.set_wait_budget_cycles(0)  # restores the default
