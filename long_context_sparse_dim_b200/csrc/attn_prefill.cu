@@ -7,18 +7,28 @@
 // tokens the indexer picks); "RTPurbo: Turning Dense LLMs into Sparse Attention
 // Models ...", "Three Key Insights" 1 (local heads keep a window) and 3.
 //
-// Design (B200): a CTA takes one query head and 128 query tokens; K/V tiles of
-// 64 keys stream through a two-stage cp.async ring (256-byte rows, XOR
-// swizzle).  Eight warps each own 16 query rows and run the flash-attention
-// recurrence on mma.sync (S = Q K^T, online softmax, P as a bf16 hi + lo pair,
-// O += P V).  For the sparse form, key j is admitted for token i iff
-// s_ij > tau_i or (s_ij == tau_i and j <= tiepos_i): the indexer tile s is
-// recomputed with exactly the instruction the selection used (tcgen05.mma
-// kind::f16, M=128, N=64, K=16, projected tiles fed by TMA with the 32-byte
-// swizzle), so the predicate sees bit-identical scores.  A ninth warp issues
-// those TMA loads and MMAs; warps 0-3 read the accumulators from TMEM (one
-// token per lane) and publish a 128 x 64 admission bitmap per tile in shared
-// memory; warps skip tiles where none of their rows admits a key.
+// Design (B200, tcgen05): a CTA takes one query head and 128 query tokens
+// (TMEM lane r = token r) and streams 128-key K/V tiles through a two-stage
+// TMA ring (128-byte swizzle, no multicast).  Per tile:
+//   S = Q K^T       tcgen05.mma M=128 N=128, eight K=16 slices over the head
+//                   dim, into one of two TMEM buffers (double-buffered)
+//   softmax         warps 0-3, one query row per thread: pass 1 takes the
+//                   row maximum over the admitted keys, pass 2 writes
+//                   P = 2^(s * scale * log2 e - m) over S in place as a bf16
+//                   hi + lo pair (so P V keeps fp32-level precision)
+//   O = P V         tcgen05.mma with A = P read from TMEM and B = V as an
+//                   MN-major operand, hi and lo parts, into a TMEM O tile
+//   fold            warps 4-7 (same TMEM lane quadrants, one row per thread)
+//                   add O into fp32 registers with the online-softmax
+//                   rescaling 2^(m_old - m_new), rounding to nearest every
+//                   tile (no drift over a million keys); the softmax hands
+//                   them each tile's row maximum and sum through shared memory
+// Warp 8 issues the TMA loads, warp 9 the MMAs; every hand-off is an mbarrier
+// and every wait is time-bounded.  For the sparse form, key j is admitted for
+// token i iff s_ij > tau_i or (s_ij == tau_i and j <= tiepos_i): the indexer
+// tile s is recomputed with exactly the instruction the selection used
+// (tcgen05.mma kind::f16, M=128, N=128, K=16 over 128-key tiles aligned as in
+// the selection), so the predicate sees bit-identical scores.
 #include <math.h>
 
 #include "launch.h"
@@ -28,35 +38,36 @@ namespace rtp {
 
 namespace {
 
-constexpr int kApRows = 128;
-constexpr int kApKeys = 64;
-constexpr int kApMathWarps = 8;
-constexpr int kApRowBytes = kHeadDim * 2;                 // 256 B
-constexpr int kApTileBytes = kApKeys * kApRowBytes;       // 16 KB per K or V tile
-constexpr int kApIdxTileBytes = kApKeys * kIdxDim * 2;    // 2 KB
+constexpr int kAtRows = 128;                          // query rows per CTA (MMA M, TMEM lanes)
+constexpr int kAtKeys = 128;                          // keys per tile
+constexpr int kAtStages = 2;                          // K/V ring
+constexpr int kAtSoftWarps = 4;                       // warps 0-3: softmax
+constexpr int kAtCorrWarps = 4;                       // warps 4-7: O fold and output
+constexpr int kAtProducerWarp = 8, kAtMmaWarp = 9;
+constexpr int kAtThreads = 10 * 32;
+constexpr int kAtHalfBytes = kAtKeys * 128;           // 128 rows x 64 bf16 (one 128-byte-swizzled half)
+constexpr int kAtTileBytes = 2 * kAtHalfBytes;        // one Q, K or V tile: 32 KB
+constexpr int kAtIdxBytes = kAtKeys * kIdxDim * 2;    // 4 KB
+constexpr uint32_t kTmemS = 0, kTmemO = 256, kTmemIdx = 384, kAtTmemCols = 512;
 constexpr float kLog2eF = 1.4426950408889634f;
-// The MMA accumulators are folded into a round-to-nearest fp32 sum every
-// kApFlush tiles: tensor-core accumulation does not round to nearest, so one
-// accumulator carried over a million keys would drift by ~1e-3 relative.
-constexpr int kApFlush = 16;
 
-struct ApSmem {
-  alignas(1024) uint8_t qidx[kApRows * kIdxDim * 2];      // 4 KB (sparse form)
-  alignas(1024) uint8_t kidx[2][kApIdxTileBytes];          // 2 x 2 KB (sparse form)
-  alignas(128) uint8_t q[kApRows * kApRowBytes];          // 32 KB
-  alignas(128) uint8_t kv[2][2][kApTileBytes];            // [stage][K,V] 64 KB
-  uint32_t bits[2][kApRows][2];                           // admission bitmaps, double-buffered
-  float otot[kApMathWarps][64][32];                       // round-to-nearest running output sums
-  uint64_t qidx_full;
-  uint64_t kidx_full[2];
-  uint64_t kidx_empty[2];
-  uint64_t t_full[2];
-  uint64_t t_empty[2];
+struct AtSmem {
+  alignas(1024) uint8_t q[kAtTileBytes];
+  alignas(1024) uint8_t k[kAtStages][kAtTileBytes];
+  alignas(1024) uint8_t v[kAtStages][kAtTileBytes];
+  alignas(1024) uint8_t qidx[kAtRows * kIdxDim * 2];  // sparse form
+  alignas(1024) uint8_t kidx[kAtStages][kAtIdxBytes];
+  uint64_t q_full;
+  uint64_t k_full[kAtStages], v_full[kAtStages], kv_empty[kAtStages];
+  uint64_t s_full[2], p_full[2], s_free[2];
+  uint64_t idx_full, idx_free;
+  uint64_t o_full, o_free;
+  uint64_t stat_full[2], stat_free[2];
+  float2 stat[2][kAtRows];  // per tile (double-buffered): the row's maximum and sum of P
   uint32_t tmem_base;
 };
 
-struct ApArgs {
-  View4 q, k, v;
+struct AtArgs {
   const int32_t* lens;
   const uint32_t* tau_bits;
   const int32_t* tiepos;
@@ -68,374 +79,348 @@ struct ApArgs {
   long long budget;
 };
 
-RTP_DEVICE uint32_t ap_swz(int r, int c) { return (uint32_t)(r * kApRowBytes + ((c ^ (r & 7)) << 4)); }
-
-RTP_DEVICE void cp16(uint32_t dst, const void* src, bool pred) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(pred ? 16 : 0));
-}
-RTP_DEVICE void cp_commit() { asm volatile("cp.async.commit_group;\n" ::); }
-RTP_DEVICE void cp_wait_all() { asm volatile("cp.async.wait_group 0;\n" ::); }
-RTP_DEVICE void ldsm4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-               : "r"(addr));
-}
-RTP_DEVICE void ldsm4t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-               : "r"(addr));
-}
-RTP_DEVICE void mma16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};\n"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
 RTP_DEVICE float ex2a(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
   return y;
 }
-RTP_DEVICE void named_sync(int id, int n) { asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(n) : "memory"); }
+
+// Bits j of a 32-key chunk with lo <= j <= hi.
+RTP_DEVICE uint32_t band32(int lo, int hi) {
+  if (hi < 0 || lo > 31 || hi < lo) return 0u;
+  const int l = max(lo, 0), r = min(hi, 31);
+  const uint32_t upto = r >= 31 ? 0xffffffffu : ((1u << (r + 1)) - 1u);
+  return upto & ~((1u << l) - 1u);
+}
 
 }  // namespace
 
 template <bool SPARSE>
-__global__ void __launch_bounds__(kApMathWarps * 32 + (SPARSE ? 32 : 0))
-attn_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap, ApArgs A) {
+__global__ void __launch_bounds__(kAtThreads, 1)
+attn_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
+                    const __grid_constant__ CUtensorMap vmap, const __grid_constant__ CUtensorMap qimap,
+                    const __grid_constant__ CUtensorMap kimap, AtArgs A) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
-  ApSmem& S = *reinterpret_cast<ApSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  AtSmem& S = *reinterpret_cast<AtSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int g = lane >> 2, c = lane & 3;
-  const int t0 = blockIdx.x * kApRows;
+  // heaviest (latest) query blocks first
+  const int t0 = ((int)gridDim.x - 1 - (int)blockIdx.x) * kAtRows;
   const int bh = blockIdx.y;
   const int b = bh / A.Hq, h = bh % A.Hq, kvh = h / A.G;
   int n_b = A.N;
   if (A.lens) n_b = min(max(A.lens[b], 0), A.N);
   const int qbase = n_b - A.T;
-  const int t_last = min(t0 + kApRows, A.T) - 1;
+  const int t_last = min(t0 + kAtRows, A.T) - 1;
   const int kmax = min(qbase + t_last, n_b - 1);  // last key any row of the block sees
-  int klo = 0;
-  if (!SPARSE) klo = max(0, qbase + t0 - A.W + 1);
-  const int tile0 = klo / kApKeys;
-  const int ntiles = kmax >= klo ? (kmax / kApKeys) - tile0 + 1 : 0;
-  bool alive = true;
+  const int klo = SPARSE ? 0 : max(0, qbase + t0 - A.W + 1);
+  const int tile0 = klo / kAtKeys;
+  const int ntiles = kmax >= klo ? (kmax / kAtKeys) - tile0 + 1 : 0;
 
-  if (SPARSE) {
-    if (tid == 0) {
-      mbar_init(&S.qidx_full, 1);
-      for (int i = 0; i < 2; ++i) {
-        mbar_init(&S.kidx_full[i], 1);
-        mbar_init(&S.kidx_empty[i], 1);
-        mbar_init(&S.t_full[i], 1);
-        mbar_init(&S.t_empty[i], 128);
-      }
-      mbar_fence_init();
+  if (tid == 0) {
+    mbar_init(&S.q_full, 1);
+    for (int i = 0; i < kAtStages; ++i) {
+      mbar_init(&S.k_full[i], 1);
+      mbar_init(&S.v_full[i], 1);
+      mbar_init(&S.kv_empty[i], 1);
     }
-    if (warp == 0) tmem_alloc(&S.tmem_base, 2 * kApKeys);
-    tc_fence_before();
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&S.s_full[i], 1);
+      mbar_init(&S.p_full[i], kAtSoftWarps);
+      mbar_init(&S.s_free[i], 1);
+    }
+    mbar_init(&S.idx_full, 1);
+    mbar_init(&S.idx_free, kAtSoftWarps);
+    mbar_init(&S.o_full, 1);
+    mbar_init(&S.o_free, kAtCorrWarps);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&S.stat_full[i], kAtSoftWarps);
+      mbar_init(&S.stat_free[i], kAtCorrWarps);
+    }
+    mbar_fence_init();
   }
+  if (warp == 0) tmem_alloc(&S.tmem_base, kAtTmemCols);
+  tc_fence_before();
   __syncthreads();
-  if (SPARSE) tc_fence_after();
-  const uint32_t tmem = SPARSE ? S.tmem_base : 0u;
+  tc_fence_after();
+  const uint32_t tmem = S.tmem_base;
+  bool alive = true;
+  uint32_t loads = 0, pvs = 0, qks = 0;
+  bool q_issued = false;
 
-  const __nv_bfloat16* kbase = static_cast<const __nv_bfloat16*>(A.k.data) + b * A.k.sb + kvh * A.k.sh;
-  const __nv_bfloat16* vbase = static_cast<const __nv_bfloat16*>(A.v.data) + b * A.v.sb + kvh * A.v.sh;
-
-  if (SPARSE && warp == kApMathWarps) {
-    // ---------------- indexer: TMA + tcgen05.mma (one elected lane) ----------------
+  if (warp == kAtProducerWarp) {
+    // ---------------- TMA producer (one elected lane) ----------------
     if (lane == 0 && ntiles > 0) {
-      mbar_expect_tx(&S.qidx_full, kApRows * kIdxDim * 2);
-      tma_load_4d(S.qidx, &qmap, &S.qidx_full, 0, t0, h, b);
-      int loads = 0, mma_issued = 0;
-      for (int i = 0; i < ntiles && i < 2; ++i) {
-        mbar_expect_tx(&S.kidx_full[i], kApIdxTileBytes);
-        tma_load_4d(S.kidx[i], &kmap, &S.kidx_full[i], 0, (tile0 + i) * kApKeys, kvh, b);
-        loads = i + 1;
-      }
-      mbar_wait(&S.qidx_full, 0, alive, A.err, A.budget);
-      const uint64_t adesc = umma_desc_k_sw32(S.qidx);
-      constexpr uint32_t idesc = umma_idesc_bf16_f32(kApRows, kApKeys);
+      mbar_expect_tx(&S.q_full, kAtTileBytes + (SPARSE ? kAtRows * kIdxDim * 2 : 0));
+      tma_load_4d(S.q, &qmap, &S.q_full, 0, t0, h, b);
+      tma_load_4d(S.q + kAtHalfBytes, &qmap, &S.q_full, 64, t0, h, b);
+      if (SPARSE) tma_load_4d(S.qidx, &qimap, &S.q_full, 0, t0, h, b);
+      q_issued = true;
       for (int i = 0; i < ntiles; ++i) {
-        const int st = i & 1;
-        const uint32_t ph = (i >> 1) & 1;
-        if (!mbar_wait(&S.kidx_full[st], ph, alive, A.err, A.budget)) break;
-        if (!mbar_wait(&S.t_empty[st], ph ^ 1, alive, A.err, A.budget)) break;
+        const int st = i % kAtStages;
+        const uint32_t ph = (uint32_t)(i / kAtStages) & 1u;
+        if (!mbar_wait(&S.kv_empty[st], ph ^ 1u, alive, A.err, A.budget)) break;
+        const int key0 = (tile0 + i) * kAtKeys;
+        mbar_expect_tx(&S.k_full[st], kAtTileBytes + (SPARSE ? kAtIdxBytes : 0));
+        tma_load_4d(S.k[st], &kmap, &S.k_full[st], 0, key0, kvh, b);
+        tma_load_4d(S.k[st] + kAtHalfBytes, &kmap, &S.k_full[st], 64, key0, kvh, b);
+        if (SPARSE) tma_load_4d(S.kidx[st], &kimap, &S.k_full[st], 0, key0, kvh, b);
+        mbar_expect_tx(&S.v_full[st], kAtTileBytes);
+        tma_load_4d(S.v[st], &vmap, &S.v_full[st], 0, key0, kvh, b);
+        tma_load_4d(S.v[st] + kAtHalfBytes, &vmap, &S.v_full[st], 64, key0, kvh, b);
+        loads = (uint32_t)i + 1u;
+      }
+    }
+  } else if (warp == kAtMmaWarp) {
+    // ---------------- MMA issuer (one elected lane) ----------------
+    if (lane == 0 && ntiles > 0) {
+      mbar_wait(&S.q_full, 0, alive, A.err, A.budget);
+      constexpr uint32_t idesc_qk = umma_idesc_bf16_f32(kAtRows, kAtKeys);
+      constexpr uint32_t idesc_pv = umma_idesc_bf16_f32(kAtRows, kHeadDim) | (1u << 16);  // V is MN-major
+      const uint32_t qa = smem_addr(S.q);
+      // O = P_j V_j: A = the P tile (bf16 hi + lo) in TMEM, B = V_j in shared memory
+      auto issue_pv = [&](int j) -> bool {
+        const int st = j % kAtStages, bj = j & 1;
+        if (!mbar_wait(&S.p_full[bj], (uint32_t)(j >> 1) & 1u, alive, A.err, A.budget)) return false;
+        if (!mbar_wait(&S.o_free, ((uint32_t)j & 1u) ^ 1u, alive, A.err, A.budget)) return false;
+        if (!mbar_wait(&S.v_full[st], (uint32_t)(j / kAtStages) & 1u, alive, A.err, A.budget)) return false;
         tc_fence_after();
-        umma_f16(tmem + st * kApKeys, adesc, umma_desc_k_sw32(S.kidx[st]), idesc, 0);
-        umma_commit(&S.kidx_empty[st]);
-        umma_commit(&S.t_full[st]);
-        mma_issued = i + 1;
-        if (i + 2 < ntiles) {  // refill this stage once the MMA has read it
-          if (!mbar_wait(&S.kidx_empty[st], ph, alive, A.err, A.budget)) break;
-          mbar_expect_tx(&S.kidx_full[st], kApIdxTileBytes);
-          tma_load_4d(S.kidx[st], &kmap, &S.kidx_full[st], 0, (tile0 + i + 2) * kApKeys, kvh, b);
-          loads = i + 3;
+        const uint32_t va = smem_addr(S.v[st]);
+#pragma unroll
+        for (int kk = 0; kk < kAtKeys / 16; ++kk) {
+          const uint64_t bdesc = umma_desc_sw128(va + (uint32_t)kk * 16u * 128u, kAtHalfBytes);
+          const uint32_t a_hi =
+              tmem + kTmemS + (uint32_t)bj * kAtKeys + 32u * (uint32_t)(kk >> 1) + 8u * (uint32_t)(kk & 1);
+          umma_f16_tmem_a(tmem + kTmemO, a_hi, bdesc, idesc_pv, kk > 0 ? 1u : 0u);
+          umma_f16_tmem_a(tmem + kTmemO, a_hi + 16u, bdesc, idesc_pv, 1u);
         }
-      }
-      // wind down: the last MMA and every TMA load issued land before TMEM is freed
-      if (ntiles > 0) {
-        mbar_drain(&S.qidx_full, 0, A.err);
-        for (int i = loads > 2 ? loads - 2 : 0; i < loads; ++i)
-          mbar_drain(&S.kidx_full[i & 1], (i >> 1) & 1, A.err);
-        if (mma_issued > 0)
-          mbar_drain(&S.t_full[(mma_issued - 1) & 1], ((mma_issued - 1) >> 1) & 1, A.err);
-      }
-    }
-  } else {
-    // ---------------- math warps 0-7 ----------------
-    const uint32_t qs = smem_addr(S.q);
-    // Q tile: 128 rows x 16 chunks
-    for (int i = tid; i < kApRows * 16; i += kApMathWarps * 32) {
-      const int r = i >> 4, ch = i & 15;
-      const int t = t0 + r;
-      const bool ok = t < A.T;
-      const __nv_bfloat16* src = static_cast<const __nv_bfloat16*>(A.q.data) + b * A.q.sb + h * A.q.sh +
-                                 (int64_t)(ok ? t : t0) * A.q.sn + ch * 8;
-      cp16(qs + ap_swz(r, ch), src, ok);
-    }
-    auto load_kv = [&](int i, int st) {
-      const int key0 = (tile0 + i) * kApKeys;
-      const uint32_t ks = smem_addr(S.kv[st][0]), vs = smem_addr(S.kv[st][1]);
+        umma_commit(&S.o_full);
+        umma_commit(&S.s_free[bj]);
+        umma_commit(&S.kv_empty[st]);
+        pvs = (uint32_t)j + 1u;
+        return true;
+      };
+      bool ok = alive;
+      for (int i = 0; i < ntiles && ok; ++i) {
+        const int st = i % kAtStages, bi = i & 1;
+        if (!mbar_wait(&S.k_full[st], (uint32_t)(i / kAtStages) & 1u, alive, A.err, A.budget)) break;
+        if (!mbar_wait(&S.s_free[bi], ((uint32_t)(i >> 1) & 1u) ^ 1u, alive, A.err, A.budget)) break;
+        tc_fence_after();
+        const uint32_t ka = smem_addr(S.k[st]);
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int idx = tid + u * kApMathWarps * 32;  // 0..1023
-        const int r = idx >> 4, ch = idx & 15;
-        const int key = key0 + r;
-        const bool ok = key >= klo && key <= kmax;
-        const int kk = ok ? key : klo;
-        cp16(ks + ap_swz(r, ch), kbase + (int64_t)kk * A.k.sn + ch * 8, ok);
-        cp16(vs + ap_swz(r, ch), vbase + (int64_t)kk * A.v.sn + ch * 8, ok);
-      }
-    };
-    if (ntiles > 0) load_kv(0, 0);
-    cp_commit();
-
-    // per-row thresholds for the indexer epilogue (warps 0-3: row = tid)
-    float tau = 0.f;
-    int tpos = -1, prow = -1;
-    if (SPARSE && warp < 4) {
-      const int t = t0 + tid;
-      prow = t < A.T ? qbase + t : -1;
-      if (t < A.T && prow >= 0) {
-        const int64_t qrow = (int64_t)bh * A.T + t;
-        tau = __uint_as_float(A.tau_bits[qrow]);
-        tpos = A.tiepos[qrow];
-      }
-    }
-    // this warp's two rows per thread
-    const int ra = warp * 16 + g, rb = ra + 8;
-    const int pa = (t0 + ra < A.T) ? qbase + t0 + ra : -1;
-    const int pb = (t0 + rb < A.T) ? qbase + t0 + rb : -1;
-
-    cp_wait_all();
-    named_sync(1, kApMathWarps * 32);
-    uint32_t qf[8][4];
-#pragma unroll
-    for (int kk = 0; kk < 8; ++kk) {
-      const int r = warp * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-      ldsm4(qs + ap_swz(r, 2 * kk + (lane >> 4)), qf[kk][0], qf[kk][1], qf[kk][2], qf[kk][3]);
-    }
-    float o[16][4];
-#pragma unroll
-    for (int nt = 0; nt < 16; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
-    float ma = -INFINITY, mb = -INFINITY, la = 0.f, lb = 0.f;
-    float* ot = &S.otot[warp][0][0];  // this thread's 64 sums at ot[e * 32 + lane]
-#pragma unroll
-    for (int e = 0; e < 64; ++e) ot[e * 32 + lane] = 0.f;
-    float ca = 1.f, cb = 1.f;  // rescale factors applied to o since the last fold
-    auto fold = [&]() {
-#pragma unroll
-      for (int nt = 0; nt < 16; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          float& acc = ot[(nt * 4 + e) * 32 + lane];
-          acc = __fmaf_rn(acc, e < 2 ? ca : cb, o[nt][e]);
-          o[nt][e] = 0.f;
+        for (int kk = 0; kk < kHeadDim / 16; ++kk) {
+          const uint32_t off = (uint32_t)(kk >> 2) * kAtHalfBytes + 32u * (uint32_t)(kk & 3);
+          umma_f16(tmem + kTmemS + (uint32_t)bi * kAtKeys, umma_desc_sw128(qa + off, 16),
+                   umma_desc_sw128(ka + off, 16), idesc_qk, kk > 0 ? 1u : 0u);
         }
-      ca = cb = 1.f;
-    };
-
-    for (int i = 0; i < ntiles; ++i) {
-      const int st = i & 1;
-      const int key0 = (tile0 + i) * kApKeys;
-      if (i + 1 < ntiles) load_kv(i + 1, st ^ 1);
-      cp_commit();
-      if (SPARSE && warp < 4) {
-        // admission bitmap of row `tid` for this tile
-        uint32_t w0 = 0u, w1 = 0u;
-        if (mbar_wait(&S.t_full[st], (i >> 1) & 1, alive, A.err, A.budget)) {
+        umma_commit(&S.s_full[bi]);
+        qks = (uint32_t)i + 1u;
+        if (SPARSE) {
+          if (!mbar_wait(&S.idx_free, ((uint32_t)i & 1u) ^ 1u, alive, A.err, A.budget)) break;
           tc_fence_after();
-          uint32_t v0[32], v1[32];
-          const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16) + st * kApKeys;
-          tmem_ld32(taddr, v0);
-          tmem_ld32(taddr + 32, v1);
-          tmem_ld_wait();
-          tc_fence_before();
-          mbar_arrive(&S.t_empty[st]);
-          const int nv = prow - key0 + 1;
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const float s0 = __fadd_rn(__fmul_rn(__uint_as_float(v0[j]), 0.25f), 0.0f);
-            const float s1 = __fadd_rn(__fmul_rn(__uint_as_float(v1[j]), 0.25f), 0.0f);
-            const bool a0 = j < nv && (s0 > tau || (s0 == tau && key0 + j <= tpos));
-            const bool a1 = j + 32 < nv && (s1 > tau || (s1 == tau && key0 + 32 + j <= tpos));
-            w0 |= (uint32_t)a0 << j;
-            w1 |= (uint32_t)a1 << j;
-          }
+          umma_f16(tmem + kTmemIdx, umma_desc_k_sw32(S.qidx), umma_desc_k_sw32(S.kidx[st]), idesc_qk, 0u);
+          umma_commit(&S.idx_full);
         }
-        S.bits[st][tid][0] = w0;
-        S.bits[st][tid][1] = w1;
+        if (i > 0) ok = issue_pv(i - 1);
       }
-      // K/V tile i (committed one group earlier) and the bitmap are ready
-      asm volatile("cp.async.wait_group 1;\n" ::);
-      named_sync(1, kApMathWarps * 32);
-
-      // admission of this thread's rows: bits over the tile's 64 keys
-      uint64_t adm_a, adm_b;
+      if (ok && alive && qks == (uint32_t)ntiles) issue_pv(ntiles - 1);
+    }
+  } else if (warp < kAtSoftWarps) {
+    // ---------------- softmax: one query row per thread ----------------
+    const int row = tid;
+    const int t = t0 + row;
+    const int pos = t < A.T ? qbase + t : -1;  // -1: no keys
+    float tau = 0.f;
+    int tpos = -1;
+    if (SPARSE && pos >= 0) {
+      const int64_t qrow = (int64_t)bh * A.T + t;
+      tau = __uint_as_float(A.tau_bits[qrow]);
+      tpos = A.tiepos[qrow];
+    }
+    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    float m_run = -INFINITY;  // running maximum of the scaled logits (log2 units)
+    for (int i = 0; i < ntiles; ++i) {
+      const int bi = i & 1;
+      const int key0 = (tile0 + i) * kAtKeys;
+      // admission bits of this row over the tile's 128 keys
+      uint32_t adm[4];
       if (SPARSE) {
-        adm_a = ((uint64_t)S.bits[st][ra][1] << 32) | S.bits[st][ra][0];
-        adm_b = ((uint64_t)S.bits[st][rb][1] << 32) | S.bits[st][rb][0];
+        const bool ok = __all_sync(0xffffffffu, mbar_wait(&S.idx_full, (uint32_t)i & 1u, alive, A.err, A.budget));
+        if (!ok) {
+          alive = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t v[32];
+          tmem_ld32(lane_base + kTmemIdx + 32u * (uint32_t)c, v);
+          tmem_ld_wait();
+          uint32_t bits = 0u;
+#pragma unroll
+          for (int jj = 0; jj < 32; ++jj) {
+            const float s = __fadd_rn(__fmul_rn(__uint_as_float(v[jj]), 0.25f), 0.0f);
+            bits |= (uint32_t)(s > tau || (s == tau && key0 + 32 * c + jj <= tpos)) << jj;
+          }
+          adm[c] = bits & band32(0, pos - key0 - 32 * c);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.idx_free);
       } else {
-        auto band = [&](int p) -> uint64_t {
-          if (p < 0) return 0ull;
-          const int lo = max(p - A.W + 1, 0) - key0, hi = p - key0;  // admitted tile columns [lo, hi]
-          if (hi < 0 || lo > 63) return 0ull;
-          const int l = max(lo, 0), r = min(hi, 63);
-          const uint64_t upto = r >= 63 ? ~0ull : ((1ull << (r + 1)) - 1ull);
-          return upto & ~((1ull << l) - 1ull);
-        };
-        adm_a = band(pa);
-        adm_b = band(pb);
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          adm[c] = pos < 0 ? 0u : band32(max(pos - A.W + 1, 0) - key0 - 32 * c, pos - key0 - 32 * c);
       }
-      if (__any_sync(0xffffffffu, (adm_a | adm_b) != 0ull)) {
-        const uint32_t ks = smem_addr(S.kv[st][0]), vs = smem_addr(S.kv[st][1]);
-        float sacc[8][4];
-#pragma unroll
-        for (int nt = 0; nt < 8; ++nt) sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-#pragma unroll
-          for (int np = 0; np < 4; ++np) {
-            const int key = 16 * np + (lane & 7) + ((lane >> 4) << 3);
-            uint32_t b0, b1, b2, b3;
-            ldsm4(ks + ap_swz(key, 2 * kk + ((lane >> 3) & 1)), b0, b1, b2, b3);
-            mma16816(sacc[2 * np], qf[kk][0], qf[kk][1], qf[kk][2], qf[kk][3], b0, b1);
-            mma16816(sacc[2 * np + 1], qf[kk][0], qf[kk][1], qf[kk][2], qf[kk][3], b2, b3);
-          }
-        }
-        // masked, scaled logits and the tile maxima of rows a (g) and b (g + 8)
-        float mxa = -INFINITY, mxb = -INFINITY;
-#pragma unroll
-        for (int nt = 0; nt < 8; ++nt) {
-          const int j0 = 8 * nt + 2 * c;
-          sacc[nt][0] = ((adm_a >> j0) & 1ull) ? sacc[nt][0] * A.scale_log2 : -INFINITY;
-          sacc[nt][1] = ((adm_a >> (j0 + 1)) & 1ull) ? sacc[nt][1] * A.scale_log2 : -INFINITY;
-          sacc[nt][2] = ((adm_b >> j0) & 1ull) ? sacc[nt][2] * A.scale_log2 : -INFINITY;
-          sacc[nt][3] = ((adm_b >> (j0 + 1)) & 1ull) ? sacc[nt][3] * A.scale_log2 : -INFINITY;
-          mxa = fmaxf(mxa, fmaxf(sacc[nt][0], sacc[nt][1]));
-          mxb = fmaxf(mxb, fmaxf(sacc[nt][2], sacc[nt][3]));
-        }
-        mxa = fmaxf(mxa, __shfl_xor_sync(0xffffffffu, mxa, 1));
-        mxa = fmaxf(mxa, __shfl_xor_sync(0xffffffffu, mxa, 2));
-        mxb = fmaxf(mxb, __shfl_xor_sync(0xffffffffu, mxb, 1));
-        mxb = fmaxf(mxb, __shfl_xor_sync(0xffffffffu, mxb, 2));
-        const float mna = fmaxf(ma, mxa), mnb = fmaxf(mb, mxb);
-        const float ala = mna == -INFINITY ? 1.f : ex2a(ma - mna);
-        const float alb = mnb == -INFINITY ? 1.f : ex2a(mb - mnb);
-        ma = mna;
-        mb = mnb;
-        la *= ala;
-        lb *= alb;
-        ca *= ala;
-        cb *= alb;
-#pragma unroll
-        for (int nt = 0; nt < 16; ++nt) {
-          o[nt][0] *= ala;
-          o[nt][1] *= ala;
-          o[nt][2] *= alb;
-          o[nt][3] *= alb;
-        }
-        // P in A-fragment form (hi and lo bf16 parts), k-step j covers keys 16j..16j+15
-        uint32_t ph[4][4], pl[4][4];
-#pragma unroll
-        for (int nt = 0; nt < 8; ++nt) {
-          const float p0 = sacc[nt][0] == -INFINITY ? 0.f : ex2a(sacc[nt][0] - mna);
-          const float p1 = sacc[nt][1] == -INFINITY ? 0.f : ex2a(sacc[nt][1] - mna);
-          const float p2 = sacc[nt][2] == -INFINITY ? 0.f : ex2a(sacc[nt][2] - mnb);
-          const float p3 = sacc[nt][3] == -INFINITY ? 0.f : ex2a(sacc[nt][3] - mnb);
-          la += p0 + p1;
-          lb += p2 + p3;
-          const uint32_t hab = pack_bf16x2(p0, p1), hcd = pack_bf16x2(p2, p3);
-          const uint32_t lab = pack_bf16x2(p0 - bf16_lo(hab), p1 - bf16_hi(hab));
-          const uint32_t lcd = pack_bf16x2(p2 - bf16_lo(hcd), p3 - bf16_hi(hcd));
-          const int j = nt >> 1, hi8 = nt & 1;
-          ph[j][hi8 * 2 + 0] = hab;  // a0 / a2: row g
-          ph[j][hi8 * 2 + 1] = hcd;  // a1 / a3: row g + 8
-          pl[j][hi8 * 2 + 0] = lab;
-          pl[j][hi8 * 2 + 1] = lcd;
-        }
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-#pragma unroll
-          for (int np = 0; np < 8; ++np) {
-            const int key = 16 * j + (lane & 7) + ((lane >> 3) & 1) * 8;
-            uint32_t b0, b1, b2, b3;
-            ldsm4t(vs + ap_swz(key, 2 * np + (lane >> 4)), b0, b1, b2, b3);
-            mma16816(o[2 * np], ph[j][0], ph[j][1], ph[j][2], ph[j][3], b0, b1);
-            mma16816(o[2 * np], pl[j][0], pl[j][1], pl[j][2], pl[j][3], b0, b1);
-            mma16816(o[2 * np + 1], ph[j][0], ph[j][1], ph[j][2], ph[j][3], b2, b3);
-            mma16816(o[2 * np + 1], pl[j][0], pl[j][1], pl[j][2], pl[j][3], b2, b3);
-          }
-        }
+      const bool ok =
+          __all_sync(0xffffffffu, mbar_wait(&S.s_full[bi], (uint32_t)(i >> 1) & 1u, alive, A.err, A.budget));
+      if (!ok) {
+        alive = false;
+        break;
       }
-      if ((i % kApFlush) == kApFlush - 1) fold();
-      named_sync(1, kApMathWarps * 32);  // the stage is free for the prefetch two tiles ahead
+      tc_fence_after();
+      const uint32_t sb = lane_base + kTmemS + (uint32_t)bi * kAtKeys;
+      // pass 1: the tile maximum of the admitted logits
+      float tmax = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t v[32];
+        tmem_ld32(sb + 32u * (uint32_t)c, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj)
+          tmax = fmaxf(tmax, ((adm[c] >> jj) & 1u) ? __uint_as_float(v[jj]) : -INFINITY);
+      }
+      const float m_new = fmaxf(m_run, tmax * A.scale_log2);
+      // pass 2: P = 2^(s * scale * log2 e - m_new) as bf16 hi + lo, written over S
+      float lsum = 0.f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t v[32];
+        tmem_ld32(sb + 32u * (uint32_t)c, v);
+        tmem_ld_wait();
+        uint32_t hi[16], lo[16];
+#pragma unroll
+        for (int jj = 0; jj < 16; ++jj) {
+          const float e0 = ex2a(__fmaf_rn(__uint_as_float(v[2 * jj]), A.scale_log2, -m_new));
+          const float e1 = ex2a(__fmaf_rn(__uint_as_float(v[2 * jj + 1]), A.scale_log2, -m_new));
+          const float p0 = ((adm[c] >> (2 * jj)) & 1u) ? e0 : 0.f;
+          const float p1 = ((adm[c] >> (2 * jj + 1)) & 1u) ? e1 : 0.f;
+          lsum += p0 + p1;
+          hi[jj] = pack_bf16x2(p0, p1);
+          lo[jj] = pack_bf16x2(p0 - bf16_lo(hi[jj]), p1 - bf16_hi(hi[jj]));
+        }
+        tmem_st16(sb + 32u * (uint32_t)c, hi);
+        tmem_st16(sb + 32u * (uint32_t)c + 16u, lo);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.p_full[bi]);
+      m_run = m_new;
+      // hand the tile's (maximum, sum) to the fold
+      if (!__all_sync(0xffffffffu,
+                      mbar_wait(&S.stat_free[bi], ((uint32_t)(i >> 1) & 1u) ^ 1u, alive, A.err, A.budget))) {
+        alive = false;
+        break;
+      }
+      S.stat[bi][row] = make_float2(m_new, lsum);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.stat_full[bi]);
     }
-    cp_wait_all();
-    fold();
+  } else if (warp < kAtSoftWarps + kAtCorrWarps) {
+    // ---------------- fold and output: one query row per thread ----------------
+    const int row = tid - kAtSoftWarps * 32;
+    const int t = t0 + row;
+    const uint32_t lane_base = tmem + ((uint32_t)((warp - kAtSoftWarps) * 32) << 16);
+    float o[kHeadDim];
 #pragma unroll
-    for (int nt = 0; nt < 16; ++nt)
+    for (int d = 0; d < kHeadDim; ++d) o[d] = 0.f;
+    float m_t = -INFINITY, l_t = 0.f;  // reference maximum and denominator of o
+    for (int j = 0; j < ntiles; ++j) {
+      const int bj = j & 1;
+      if (!__all_sync(0xffffffffu,
+                      mbar_wait(&S.stat_full[bj], (uint32_t)(j >> 1) & 1u, alive, A.err, A.budget))) {
+        alive = false;
+        break;
+      }
+      const float2 st = S.stat[bj][row];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.stat_free[bj]);
+      if (!__all_sync(0xffffffffu, mbar_wait(&S.o_full, (uint32_t)j & 1u, alive, A.err, A.budget))) {
+        alive = false;
+        break;
+      }
+      tc_fence_after();
+      // O_j was computed relative to st.x; rescale the running sum to it
+      const float alpha = st.x == -INFINITY ? 1.f : ex2a(m_t - st.x);
 #pragma unroll
-      for (int e = 0; e < 4; ++e) o[nt][e] = ot[(nt * 4 + e) * 32 + lane];
+      for (int c = 0; c < kHeadDim / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(lane_base + kTmemO + 32u * (uint32_t)c, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj) o[32 * c + jj] = __fmaf_rn(o[32 * c + jj], alpha, __uint_as_float(v[jj]));
+      }
+      l_t = __fmaf_rn(l_t, alpha, st.y);
+      if (st.x != -INFINITY) m_t = st.x;
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.o_free);
+    }
+
     // ---- normalise and store ----
-    la += __shfl_xor_sync(0xffffffffu, la, 1);
-    la += __shfl_xor_sync(0xffffffffu, la, 2);
-    lb += __shfl_xor_sync(0xffffffffu, lb, 1);
-    lb += __shfl_xor_sync(0xffffffffu, lb, 2);
-    const float ia = la > 0.f ? 1.f / la : 0.f, ib = lb > 0.f ? 1.f / lb : 0.f;
-    const int ta = t0 + ra, tb = t0 + rb;
-#pragma unroll
-    for (int nt = 0; nt < 16; ++nt) {
-      const int d = 8 * nt + 2 * c;
+    if (t < A.T) {
+      const float inv = l_t > 0.f ? 1.f / l_t : 0.f;
       if (A.o_bf16) {
-        __nv_bfloat16* oa = static_cast<__nv_bfloat16*>(A.o.data) + b * A.o.sb + h * A.o.sh;
-        if (ta < A.T)
-          *reinterpret_cast<uint32_t*>(oa + (int64_t)ta * A.o.sn + d) = pack_bf16x2(o[nt][0] * ia, o[nt][1] * ia);
-        if (tb < A.T)
-          *reinterpret_cast<uint32_t*>(oa + (int64_t)tb * A.o.sn + d) = pack_bf16x2(o[nt][2] * ib, o[nt][3] * ib);
+        __nv_bfloat16* orow =
+            static_cast<__nv_bfloat16*>(A.o.data) + b * A.o.sb + h * A.o.sh + (int64_t)t * A.o.sn;
+#pragma unroll
+        for (int d = 0; d < kHeadDim; d += 8) {
+          uint4 w;
+          w.x = pack_bf16x2(o[d] * inv, o[d + 1] * inv);
+          w.y = pack_bf16x2(o[d + 2] * inv, o[d + 3] * inv);
+          w.z = pack_bf16x2(o[d + 4] * inv, o[d + 5] * inv);
+          w.w = pack_bf16x2(o[d + 6] * inv, o[d + 7] * inv);
+          *reinterpret_cast<uint4*>(orow + d) = w;
+        }
       } else {
-        float* of = static_cast<float*>(A.o.data) + b * A.o.sb + h * A.o.sh;
-        if (ta < A.T) *reinterpret_cast<float2*>(of + (int64_t)ta * A.o.sn + d) = make_float2(o[nt][0] * ia, o[nt][1] * ia);
-        if (tb < A.T) *reinterpret_cast<float2*>(of + (int64_t)tb * A.o.sn + d) = make_float2(o[nt][2] * ib, o[nt][3] * ib);
+        float* orow = static_cast<float*>(A.o.data) + b * A.o.sb + h * A.o.sh + (int64_t)t * A.o.sn;
+#pragma unroll
+        for (int d = 0; d < kHeadDim; d += 4)
+          *reinterpret_cast<float4*>(orow + d) =
+              make_float4(o[d] * inv, o[d + 1] * inv, o[d + 2] * inv, o[d + 3] * inv);
       }
     }
   }
-  if (SPARSE) {
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 0) tmem_free(tmem, 2 * kApKeys);
+
+  // ---- wind down: every copy and MMA issued lands before TMEM is freed, even
+  // after a wait gave up (the last commit of this thread covers all earlier MMAs)
+  if (warp == kAtMmaWarp && lane == 0) {
+    if (pvs > 0 && pvs >= qks) {
+      mbar_drain(&S.o_full, (pvs - 1u) & 1u, A.err);
+    } else if (qks > 0) {
+      const uint32_t last = qks - 1u;
+      if (SPARSE && qks > 0) mbar_drain(&S.idx_full, last & 1u, A.err);
+      mbar_drain(&S.s_full[last & 1u], (last >> 1) & 1u, A.err);
+    }
   }
+  if (warp == kAtProducerWarp && lane == 0) {
+    if (q_issued) mbar_drain(&S.q_full, 0, A.err);
+    for (uint32_t i = loads > (uint32_t)kAtStages ? loads - kAtStages : 0u; i < loads; ++i) {
+      mbar_drain(&S.k_full[i % kAtStages], (i / kAtStages) & 1u, A.err);
+      mbar_drain(&S.v_full[i % kAtStages], (i / kAtStages) & 1u, A.err);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_free(tmem, kAtTmemCols);
 }
 
-// ---- host ---------------------------------------------------------------------
+// ---- host side ------------------------------------------------------------------
+
 cudaError_t launch_attn_prefill(const LaunchAttnPrefill& a, cudaStream_t stream) {
   if (a.B * a.Hq * a.T == 0) return cudaSuccess;
-  ApArgs A;
-  A.q = a.q;
-  A.k = a.k;
-  A.v = a.v;
+  AtArgs A;
   A.lens = a.lens;
   A.tau_bits = a.tau_bits;
   A.tiepos = a.tiepos;
@@ -450,18 +435,20 @@ cudaError_t launch_attn_prefill(const LaunchAttnPrefill& a, cudaStream_t stream)
   A.o_bf16 = a.o_bf16 ? 1 : 0;
   A.err = a.err;
   A.budget = wait_budget_cycles();
-  const size_t smem = sizeof(ApSmem) + 1024;
-  const dim3 grid((unsigned)((a.T + kApRows - 1) / kApRows), (unsigned)(a.B * a.Hq));
+  CUtensorMap qmap, kmap, vmap, qimap{}, kimap{};
+  if (!make_row_map(&qmap, a.q, a.B, a.Hq, a.T, kAtRows)) return cudaErrorInvalidValue;
+  if (!make_row_map(&kmap, a.k, a.B, a.Hk, a.N, kAtKeys)) return cudaErrorInvalidValue;
+  if (!make_row_map(&vmap, a.v, a.B, a.Hk, a.N, kAtKeys)) return cudaErrorInvalidValue;
+  const size_t smem = sizeof(AtSmem) + 1024;
+  const dim3 grid((unsigned)((a.T + kAtRows - 1) / kAtRows), (unsigned)(a.B * a.Hq));
   if (a.W > 0) {
-    CUtensorMap dummy{};
     cudaFuncSetAttribute(attn_prefill_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    attn_prefill_kernel<false><<<grid, kApMathWarps * 32, smem, stream>>>(dummy, dummy, A);
+    attn_prefill_kernel<false><<<grid, kAtThreads, smem, stream>>>(qmap, kmap, vmap, qimap, kimap, A);
   } else {
-    CUtensorMap qmap, kmap;
-    if (!make_idx_map(&qmap, a.q_idx, a.B, a.Hq, a.T, kApRows)) return cudaErrorInvalidValue;
-    if (!make_idx_map(&kmap, a.k_idx, a.B, a.Hk, a.N, kApKeys)) return cudaErrorInvalidValue;
+    if (!make_idx_map(&qimap, a.q_idx, a.B, a.Hq, a.T, kAtRows)) return cudaErrorInvalidValue;
+    if (!make_idx_map(&kimap, a.k_idx, a.B, a.Hk, a.N, kAtKeys)) return cudaErrorInvalidValue;
     cudaFuncSetAttribute(attn_prefill_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    attn_prefill_kernel<true><<<grid, kApMathWarps * 32 + 32, smem, stream>>>(qmap, kmap, A);
+    attn_prefill_kernel<true><<<grid, kAtThreads, smem, stream>>>(qmap, kmap, vmap, qimap, kimap, A);
   }
   return cudaGetLastError();
 }

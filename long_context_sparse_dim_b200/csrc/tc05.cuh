@@ -115,6 +115,22 @@ RTP_DEVICE uint64_t umma_desc_k_sw32(const void* tile) {
          | (6ull << 61);                // layout: 32-byte swizzle
 }
 
+// Shared-memory matrix descriptor of a 128-byte-swizzled tile as a TMA load
+// with CU_TENSOR_MAP_SWIZZLE_128B writes it: rows of 128 bytes (64 bf16),
+// 8-row atoms 1024 bytes apart (stride byte offset).  K-major operands (Q, K):
+// one MMA K-slice of 16 elements is 32 bytes of a row, so slice k of a
+// 64-column half starts `32 * k` bytes in; the leading byte offset is unused.
+// MN-major operands (V as the B operand of P V, keys on K, head dims on N):
+// the leading byte offset is the distance between the two 64-column halves
+// of the tile, and slice k (16 keys) starts `16 * 128 * k` bytes in.
+RTP_DEVICE uint64_t umma_desc_sw128(uint32_t saddr, uint32_t lbo_bytes) {
+  return ((uint64_t)(saddr >> 4) & 0x3FFFull)                // start address
+         | ((uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16)    // leading byte offset
+         | ((uint64_t)(1024u >> 4) << 32)                     // stride byte offset: 8 rows x 128 B
+         | (1ull << 46)                                       // descriptor version
+         | (2ull << 61);                                      // layout: 128-byte swizzle
+}
+
 // Instruction descriptor: D fp32, A/B bf16, both K-major, shape M x N.
 __host__ __device__ constexpr uint32_t umma_idesc_bf16_f32(int M, int N) {
   return (1u << 4)                      // D format fp32
@@ -130,6 +146,16 @@ RTP_DEVICE void umma_f16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem_d),
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+// The same MMA with the A operand (M x 16, bf16 pairs packed in 32-bit columns,
+// row m in lane m) read from tensor memory at `tmem_a`.
+RTP_DEVICE void umma_f16_tmem_a(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc, uint32_t idesc,
+                                uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(tmem_d),
+      "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate));
 }
 // Arrive on `bar` once all previously issued tcgen05.mma of this thread completed.
 RTP_DEVICE void umma_commit(uint64_t* bar) {
@@ -170,5 +196,16 @@ RTP_DEVICE void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
       : "r"(taddr));
 }
 RTP_DEVICE void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }
+
+// 32 lanes x 16 consecutive 32-bit columns from registers: thread (lane l of
+// the warp's quadrant) writes row (quadrant*32 + l), columns col .. col+15.
+RTP_DEVICE void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};\n" ::
+          "r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+RTP_DEVICE void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory"); }
 
 }  // namespace rtp
