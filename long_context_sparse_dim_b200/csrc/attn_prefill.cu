@@ -12,19 +12,25 @@
 // TMA ring (128-byte swizzle, no multicast).  Per tile:
 //   S = Q K^T       tcgen05.mma M=128 N=128, eight K=16 slices over the head
 //                   dim, into one of two TMEM buffers (double-buffered)
-//   softmax         warps 0-3, one query row per thread: pass 1 takes the
-//                   row maximum over the admitted keys, pass 2 writes
-//                   P = 2^(s * scale * log2 e - m) over S in place as a bf16
-//                   hi + lo pair (so P V keeps fp32-level precision)
+//   softmax         warps 0-7, two threads per query row (warps w and w+4
+//                   share TMEM lane quadrant w % 4, each takes 64 of the
+//                   tile's keys): pass 1 takes the row maximum over the
+//                   admitted keys (the halves meet at a 64-thread named
+//                   barrier), pass 2 writes P = 2^(s * scale * log2 e - m)
+//                   over S in place as a bf16 hi + lo pair (so P V keeps
+//                   fp32-level precision): the 16 keys of MMA slice k keep
+//                   their hi words in columns 16k .. 16k+7, lo in 16k+8 ..
 //   O = P V         tcgen05.mma with A = P read from TMEM and B = V as an
 //                   MN-major operand, hi and lo parts, into a TMEM O tile
-//   fold            warps 4-7 (same TMEM lane quadrants, one row per thread)
-//                   add O into fp32 registers with the online-softmax
-//                   rescaling 2^(m_old - m_new), rounding to nearest every
-//                   tile (no drift over a million keys); the softmax hands
-//                   them each tile's row maximum and sum through shared memory
-// Warp 8 issues the TMA loads, warp 9 the MMAs; every hand-off is an mbarrier
-// and every wait is time-bounded.  For the sparse form, key j is admitted for
+//   fold            warps 8-15 (two threads per row, 64 head dims each) add O
+//                   into fp32 registers with the online-softmax rescaling
+//                   2^(m_old - m_new), rounding to nearest every tile (no
+//                   drift over a million keys); the softmax hands them each
+//                   tile's row maximum and sums through shared memory
+// Warp 16 issues the TMA loads, warp 17 the MMAs; every hand-off is an
+// mbarrier and every wait is time-bounded.  Eighteen warps put five on two of
+// the SM's four sub-partitions (16K registers each), so a thread may hold at
+// most 96 registers.  For the sparse form, key j is admitted for
 // token i iff s_ij > tau_i or (s_ij == tau_i and j <= tiepos_i): the indexer
 // tile s is recomputed with exactly the instruction the selection used
 // (tcgen05.mma kind::f16, M=128, N=128, K=16 over 128-key tiles aligned as in
@@ -41,10 +47,10 @@ namespace {
 constexpr int kAtRows = 128;                          // query rows per CTA (MMA M, TMEM lanes)
 constexpr int kAtKeys = 128;                          // keys per tile
 constexpr int kAtStages = 2;                          // K/V ring
-constexpr int kAtSoftWarps = 4;                       // warps 0-3: softmax
-constexpr int kAtCorrWarps = 4;                       // warps 4-7: O fold and output
-constexpr int kAtProducerWarp = 8, kAtMmaWarp = 9;
-constexpr int kAtThreads = 10 * 32;
+constexpr int kAtSoftWarps = 8;                       // warps 0-7: softmax, two threads per row
+constexpr int kAtCorrWarps = 8;                       // warps 8-15: O fold and output, two threads per row
+constexpr int kAtProducerWarp = 16, kAtMmaWarp = 17;
+constexpr int kAtThreads = 18 * 32;
 constexpr int kAtHalfBytes = kAtKeys * 128;           // 128 rows x 64 bf16 (one 128-byte-swizzled half)
 constexpr int kAtTileBytes = 2 * kAtHalfBytes;        // one Q, K or V tile: 32 KB
 constexpr int kAtIdxBytes = kAtKeys * kIdxDim * 2;    // 4 KB
@@ -63,7 +69,8 @@ struct AtSmem {
   uint64_t idx_full, idx_free;
   uint64_t o_full, o_free;
   uint64_t stat_full[2], stat_free[2];
-  float2 stat[2][kAtRows];  // per tile (double-buffered): the row's maximum and sum of P
+  float2 stat[2][2][kAtRows];  // per tile (double-buffered) and column half: the row's maximum, sum of P
+  float pmax[2][2][kAtRows];   // per tile (double-buffered) and column half: the row's partial maximum
   uint32_t tmem_base;
 };
 
@@ -85,6 +92,14 @@ RTP_DEVICE float ex2a(float x) {
   return y;
 }
 
+RTP_DEVICE float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;\n" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+RTP_DEVICE void named_sync(int id, int n) { asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(n) : "memory"); }
+
 // Bits j of a 32-key chunk with lo <= j <= hi.
 RTP_DEVICE uint32_t band32(int lo, int hi) {
   if (hi < 0 || lo > 31 || hi < lo) return 0u;
@@ -96,7 +111,7 @@ RTP_DEVICE uint32_t band32(int lo, int hi) {
 }  // namespace
 
 template <bool SPARSE>
-__global__ void __launch_bounds__(kAtThreads, 1)
+__global__ void __maxnreg__(96)
 attn_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
                     const __grid_constant__ CUtensorMap vmap, const __grid_constant__ CUtensorMap qimap,
                     const __grid_constant__ CUtensorMap kimap, AtArgs A) {
@@ -188,10 +203,9 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
 #pragma unroll
         for (int kk = 0; kk < kAtKeys / 16; ++kk) {
           const uint64_t bdesc = umma_desc_sw128(va + (uint32_t)kk * 16u * 128u, kAtHalfBytes);
-          const uint32_t a_hi =
-              tmem + kTmemS + (uint32_t)bj * kAtKeys + 32u * (uint32_t)(kk >> 1) + 8u * (uint32_t)(kk & 1);
+          const uint32_t a_hi = tmem + kTmemS + (uint32_t)bj * kAtKeys + 16u * (uint32_t)kk;
           umma_f16_tmem_a(tmem + kTmemO, a_hi, bdesc, idesc_pv, kk > 0 ? 1u : 0u);
-          umma_f16_tmem_a(tmem + kTmemO, a_hi + 16u, bdesc, idesc_pv, 1u);
+          umma_f16_tmem_a(tmem + kTmemO, a_hi + 8u, bdesc, idesc_pv, 1u);
         }
         umma_commit(&S.o_full);
         umma_commit(&S.s_free[bj]);
@@ -225,24 +239,25 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
       if (ok && alive && qks == (uint32_t)ntiles) issue_pv(ntiles - 1);
     }
   } else if (warp < kAtSoftWarps) {
-    // ---------------- softmax: one query row per thread ----------------
-    const int row = tid;
+    // ---------------- softmax: two threads per query row, 64 keys each ----------------
+    const int quad = warp & 3, hf = warp >> 2;
+    const int row = quad * 32 + lane;
     const int t = t0 + row;
     const int pos = t < A.T ? qbase + t : -1;  // -1: no keys
-    float tau = 0.f;
+    float vtau = 0.f;  // raw indexer accumulator of the cut score (4 tau, an exact scaling)
     int tpos = -1;
     if (SPARSE && pos >= 0) {
       const int64_t qrow = (int64_t)bh * A.T + t;
-      tau = __uint_as_float(A.tau_bits[qrow]);
+      vtau = __fmul_rn(__uint_as_float(A.tau_bits[qrow]), 4.f);
       tpos = A.tiepos[qrow];
     }
-    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16) + 64u * (uint32_t)hf;
     float m_run = -INFINITY;  // running maximum of the scaled logits (log2 units)
     for (int i = 0; i < ntiles; ++i) {
       const int bi = i & 1;
-      const int key0 = (tile0 + i) * kAtKeys;
-      // admission bits of this row over the tile's 128 keys
-      uint32_t adm[4];
+      const int kh = (tile0 + i) * kAtKeys + 64 * hf;  // first key of this thread's half
+      // admission bits of this row over the half's 64 keys
+      uint32_t adm[2];
       if (SPARSE) {
         const bool ok = __all_sync(0xffffffffu, mbar_wait(&S.idx_full, (uint32_t)i & 1u, alive, A.err, A.budget));
         if (!ok) {
@@ -251,25 +266,25 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
         }
         tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 2; ++c) {
           uint32_t v[32];
           tmem_ld32(lane_base + kTmemIdx + 32u * (uint32_t)c, v);
           tmem_ld_wait();
           uint32_t bits = 0u;
 #pragma unroll
           for (int jj = 0; jj < 32; ++jj) {
-            const float s = __fadd_rn(__fmul_rn(__uint_as_float(v[jj]), 0.25f), 0.0f);
-            bits |= (uint32_t)(s > tau || (s == tau && key0 + 32 * c + jj <= tpos)) << jj;
+            const float x = __uint_as_float(v[jj]);
+            bits |= (uint32_t)(x > vtau || (x == vtau && kh + 32 * c + jj <= tpos)) << jj;
           }
-          adm[c] = bits & band32(0, pos - key0 - 32 * c);
+          adm[c] = bits & band32(0, pos - kh - 32 * c);
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&S.idx_free);
       } else {
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
-          adm[c] = pos < 0 ? 0u : band32(max(pos - A.W + 1, 0) - key0 - 32 * c, pos - key0 - 32 * c);
+        for (int c = 0; c < 2; ++c)
+          adm[c] = pos < 0 ? 0u : band32(max(pos - A.W + 1, 0) - kh - 32 * c, pos - kh - 32 * c);
       }
       const bool ok =
           __all_sync(0xffffffffu, mbar_wait(&S.s_full[bi], (uint32_t)(i >> 1) & 1u, alive, A.err, A.budget));
@@ -279,62 +294,76 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
       }
       tc_fence_after();
       const uint32_t sb = lane_base + kTmemS + (uint32_t)bi * kAtKeys;
-      // pass 1: the tile maximum of the admitted logits
+      // pass 1: the maximum of the admitted logits, over both halves of the row
       float tmax = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 2; ++c) {
         uint32_t v[32];
         tmem_ld32(sb + 32u * (uint32_t)c, v);
         tmem_ld_wait();
 #pragma unroll
-        for (int jj = 0; jj < 32; ++jj)
-          tmax = fmaxf(tmax, ((adm[c] >> jj) & 1u) ? __uint_as_float(v[jj]) : -INFINITY);
+        for (int jj = 0; jj < 32; jj += 2)
+          tmax = max3f(tmax, ((adm[c] >> jj) & 1u) ? __uint_as_float(v[jj]) : -INFINITY,
+                       ((adm[c] >> (jj + 1)) & 1u) ? __uint_as_float(v[jj + 1]) : -INFINITY);
       }
+      S.pmax[bi][hf][row] = tmax;
+      named_sync(1 + quad, 64);  // warps quad and quad + 4
+      tmax = fmaxf(S.pmax[bi][0][row], S.pmax[bi][1][row]);
       const float m_new = fmaxf(m_run, tmax * A.scale_log2);
+      // reference of the exponentials; masked logits are -inf, so while no key of
+      // the row is admitted yet (m_new = -inf) any finite reference gives P = 0
+      const float m_ref = m_new == -INFINITY ? 0.f : m_new;
       // pass 2: P = 2^(s * scale * log2 e - m_new) as bf16 hi + lo, written over S
+      // (16 keys at a time: slice q of 16 keys, which occupied columns
+      // 16q .. 16q+15 as S, keeps its 8 hi words in 16q .. 16q+7 and its 8 lo
+      // words in 16q+8 .. 16q+15, so a store only overwrites what was just read)
       float lsum = 0.f;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t v[32];
-        tmem_ld32(sb + 32u * (uint32_t)c, v);
+      for (int q = 0; q < 4; ++q) {
+        const int c = q >> 1, sub = q & 1;
+        uint32_t v[16];
+        tmem_ld16(sb + 16u * (uint32_t)q, v);
         tmem_ld_wait();
-        uint32_t hi[16], lo[16];
+        uint32_t hi[8], lo[8];
 #pragma unroll
-        for (int jj = 0; jj < 16; ++jj) {
-          const float e0 = ex2a(__fmaf_rn(__uint_as_float(v[2 * jj]), A.scale_log2, -m_new));
-          const float e1 = ex2a(__fmaf_rn(__uint_as_float(v[2 * jj + 1]), A.scale_log2, -m_new));
-          const float p0 = ((adm[c] >> (2 * jj)) & 1u) ? e0 : 0.f;
-          const float p1 = ((adm[c] >> (2 * jj + 1)) & 1u) ? e1 : 0.f;
+        for (int jj = 0; jj < 8; ++jj) {
+          const int k0 = 16 * sub + 2 * jj;
+          const float x0 = ((adm[c] >> k0) & 1u) ? __uint_as_float(v[2 * jj]) : -INFINITY;
+          const float x1 = ((adm[c] >> (k0 + 1)) & 1u) ? __uint_as_float(v[2 * jj + 1]) : -INFINITY;
+          const float p0 = ex2a(__fmaf_rn(x0, A.scale_log2, -m_ref));
+          const float p1 = ex2a(__fmaf_rn(x1, A.scale_log2, -m_ref));
           lsum += p0 + p1;
           hi[jj] = pack_bf16x2(p0, p1);
           lo[jj] = pack_bf16x2(p0 - bf16_lo(hi[jj]), p1 - bf16_hi(hi[jj]));
         }
-        tmem_st16(sb + 32u * (uint32_t)c, hi);
-        tmem_st16(sb + 32u * (uint32_t)c + 16u, lo);
+        tmem_st8(sb + 16u * (uint32_t)q, hi);
+        tmem_st8(sb + 16u * (uint32_t)q + 8u, lo);
       }
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.p_full[bi]);
       m_run = m_new;
-      // hand the tile's (maximum, sum) to the fold
+      // hand the tile's (maximum, partial sum) to the fold
       if (!__all_sync(0xffffffffu,
                       mbar_wait(&S.stat_free[bi], ((uint32_t)(i >> 1) & 1u) ^ 1u, alive, A.err, A.budget))) {
         alive = false;
         break;
       }
-      S.stat[bi][row] = make_float2(m_new, lsum);
+      S.stat[bi][hf][row] = make_float2(m_new, lsum);
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.stat_full[bi]);
     }
   } else if (warp < kAtSoftWarps + kAtCorrWarps) {
-    // ---------------- fold and output: one query row per thread ----------------
-    const int row = tid - kAtSoftWarps * 32;
+    // ---------------- fold and output: two threads per query row, 64 head dims each ----------------
+    const int cw = warp - kAtSoftWarps;
+    const int quad = cw & 3, hf = cw >> 2;
+    const int row = quad * 32 + lane;
     const int t = t0 + row;
-    const uint32_t lane_base = tmem + ((uint32_t)((warp - kAtSoftWarps) * 32) << 16);
-    float o[kHeadDim];
+    const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16) + kTmemO + 64u * (uint32_t)hf;
+    float o[64];
 #pragma unroll
-    for (int d = 0; d < kHeadDim; ++d) o[d] = 0.f;
+    for (int d = 0; d < 64; ++d) o[d] = 0.f;
     float m_t = -INFINITY, l_t = 0.f;  // reference maximum and denominator of o
     for (int j = 0; j < ntiles; ++j) {
       const int bj = j & 1;
@@ -343,7 +372,7 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
         alive = false;
         break;
       }
-      const float2 st = S.stat[bj][row];
+      const float2 s0 = S.stat[bj][0][row], s1 = S.stat[bj][1][row];
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.stat_free[bj]);
       if (!__all_sync(0xffffffffu, mbar_wait(&S.o_full, (uint32_t)j & 1u, alive, A.err, A.budget))) {
@@ -351,31 +380,33 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
         break;
       }
       tc_fence_after();
-      // O_j was computed relative to st.x; rescale the running sum to it
-      const float alpha = st.x == -INFINITY ? 1.f : ex2a(m_t - st.x);
+      // O_j was computed relative to s0.x (= s1.x); rescale the running sum to it
+      const float mj = s0.x;
+      const float alpha = mj == -INFINITY ? 1.f : ex2a(m_t - mj);
 #pragma unroll
-      for (int c = 0; c < kHeadDim / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32(lane_base + kTmemO + 32u * (uint32_t)c, v);
+      for (int c = 0; c < 4; ++c) {
+        uint32_t v[16];
+        tmem_ld16(lane_base + 16u * (uint32_t)c, v);
         tmem_ld_wait();
 #pragma unroll
-        for (int jj = 0; jj < 32; ++jj) o[32 * c + jj] = __fmaf_rn(o[32 * c + jj], alpha, __uint_as_float(v[jj]));
+        for (int jj = 0; jj < 16; ++jj) o[16 * c + jj] = __fmaf_rn(o[16 * c + jj], alpha, __uint_as_float(v[jj]));
       }
-      l_t = __fmaf_rn(l_t, alpha, st.y);
-      if (st.x != -INFINITY) m_t = st.x;
+      l_t = __fmaf_rn(l_t, alpha, s0.y + s1.y);
+      if (mj != -INFINITY) m_t = mj;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.o_free);
     }
 
-    // ---- normalise and store ----
+    // ---- normalise and store this thread's 64 head dims ----
     if (t < A.T) {
       const float inv = l_t > 0.f ? 1.f / l_t : 0.f;
+      const int d0 = 64 * hf;
       if (A.o_bf16) {
         __nv_bfloat16* orow =
-            static_cast<__nv_bfloat16*>(A.o.data) + b * A.o.sb + h * A.o.sh + (int64_t)t * A.o.sn;
+            static_cast<__nv_bfloat16*>(A.o.data) + b * A.o.sb + h * A.o.sh + (int64_t)t * A.o.sn + d0;
 #pragma unroll
-        for (int d = 0; d < kHeadDim; d += 8) {
+        for (int d = 0; d < 64; d += 8) {
           uint4 w;
           w.x = pack_bf16x2(o[d] * inv, o[d + 1] * inv);
           w.y = pack_bf16x2(o[d + 2] * inv, o[d + 3] * inv);
@@ -384,9 +415,9 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
           *reinterpret_cast<uint4*>(orow + d) = w;
         }
       } else {
-        float* orow = static_cast<float*>(A.o.data) + b * A.o.sb + h * A.o.sh + (int64_t)t * A.o.sn;
+        float* orow = static_cast<float*>(A.o.data) + b * A.o.sb + h * A.o.sh + (int64_t)t * A.o.sn + d0;
 #pragma unroll
-        for (int d = 0; d < kHeadDim; d += 4)
+        for (int d = 0; d < 64; d += 4)
           *reinterpret_cast<float4*>(orow + d) =
               make_float4(o[d] * inv, o[d + 1] * inv, o[d + 2] * inv, o[d + 3] * inv);
       }
