@@ -7,9 +7,10 @@
 // tokens the indexer picks); "RTPurbo: Turning Dense LLMs into Sparse Attention
 // Models ...", "Three Key Insights" 1 (local heads keep a window) and 3.
 //
-// Design (B200, tcgen05): a CTA takes one query head and 128 query tokens
-// (TMEM lane r = token r) and streams 128-key K/V tiles through a two-stage
-// TMA ring (128-byte swizzle, no multicast).  Per tile:
+// Design (B200, tcgen05): a CTA takes the G query heads of one KV head x 128/G
+// query tokens, 128 rows in all (TMEM lane r = row r), and streams 128-key K/V
+// tiles of that KV head through a two-stage TMA ring (128-byte swizzle, no
+// multicast); each tile is read once for the whole GQA group.  Per tile:
 //   S = Q K^T       tcgen05.mma M=128 N=128, eight K=16 slices over the head
 //                   dim, into one of two TMEM buffers (double-buffered)
 //   softmax         warps 0-7, two threads per query row (warps w and w+4
@@ -79,6 +80,7 @@ struct AtArgs {
   const uint32_t* tau_bits;
   const int32_t* tiepos;
   int Hq, Hk, G, T, N, W;
+  int TB;  // tokens per block (the block holds G heads x TB tokens)
   float scale_log2;
   MutView4 o;
   int o_bf16;
@@ -118,14 +120,17 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   AtSmem& S = *reinterpret_cast<AtSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  // heaviest (latest) query blocks first
-  const int t0 = ((int)gridDim.x - 1 - (int)blockIdx.x) * kAtRows;
-  const int bh = blockIdx.y;
-  const int b = bh / A.Hq, h = bh % A.Hq, kvh = h / A.G;
+  // A block holds the G query heads of one KV head x TB consecutive tokens (row
+  // r: head r / TB of the group, token t0 + r % TB), so every K/V tile it loads
+  // serves all G heads.  Heaviest (latest) token blocks first.
+  const int TB = A.TB;
+  const int t0 = ((int)gridDim.x - 1 - (int)blockIdx.x) * TB;
+  const int bk = blockIdx.y;
+  const int b = bk / A.Hk, kvh = bk % A.Hk;
   int n_b = A.N;
   if (A.lens) n_b = min(max(A.lens[b], 0), A.N);
   const int qbase = n_b - A.T;
-  const int t_last = min(t0 + kAtRows, A.T) - 1;
+  const int t_last = min(t0 + TB, A.T) - 1;
   const int kmax = min(qbase + t_last, n_b - 1);  // last key any row of the block sees
   const int klo = SPARSE ? 0 : max(0, qbase + t0 - A.W + 1);
   const int tile0 = klo / kAtKeys;
@@ -165,10 +170,14 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
   if (warp == kAtProducerWarp) {
     // ---------------- TMA producer (one elected lane) ----------------
     if (lane == 0 && ntiles > 0) {
-      mbar_expect_tx(&S.q_full, kAtTileBytes + (SPARSE ? kAtRows * kIdxDim * 2 : 0));
-      tma_load_4d(S.q, &qmap, &S.q_full, 0, t0, h, b);
-      tma_load_4d(S.q + kAtHalfBytes, &qmap, &S.q_full, 64, t0, h, b);
-      if (SPARSE) tma_load_4d(S.qidx, &qimap, &S.q_full, 0, t0, h, b);
+      // one box of TB rows per head of the group (and per 64-column half)
+      mbar_expect_tx(&S.q_full, A.G * TB * (kHeadDim + (SPARSE ? kIdxDim : 0)) * 2);
+      for (int g = 0; g < A.G; ++g) {
+        const int hq = kvh * A.G + g;
+        tma_load_4d(S.q + g * TB * 128, &qmap, &S.q_full, 0, t0, hq, b);
+        tma_load_4d(S.q + kAtHalfBytes + g * TB * 128, &qmap, &S.q_full, 64, t0, hq, b);
+        if (SPARSE) tma_load_4d(S.qidx + g * TB * kIdxDim * 2, &qimap, &S.q_full, 0, t0, hq, b);
+      }
       q_issued = true;
       for (int i = 0; i < ntiles; ++i) {
         const int st = i % kAtStages;
@@ -242,12 +251,14 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
     // ---------------- softmax: two threads per query row, 64 keys each ----------------
     const int quad = warp & 3, hf = warp >> 2;
     const int row = quad * 32 + lane;
-    const int t = t0 + row;
+    const bool in_block = row < A.G * TB;
+    const int h = kvh * A.G + (in_block ? row / TB : 0);
+    const int t = in_block ? t0 + row % TB : A.T;
     const int pos = t < A.T ? qbase + t : -1;  // -1: no keys
     float vtau = 0.f;  // raw indexer accumulator of the cut score (4 tau, an exact scaling)
     int tpos = -1;
     if (SPARSE && pos >= 0) {
-      const int64_t qrow = (int64_t)bh * A.T + t;
+      const int64_t qrow = ((int64_t)b * A.Hq + h) * A.T + t;
       vtau = __fmul_rn(__uint_as_float(A.tau_bits[qrow]), 4.f);
       tpos = A.tiepos[qrow];
     }
@@ -359,7 +370,9 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
     const int cw = warp - kAtSoftWarps;
     const int quad = cw & 3, hf = cw >> 2;
     const int row = quad * 32 + lane;
-    const int t = t0 + row;
+    const bool in_block = row < A.G * TB;
+    const int h = kvh * A.G + (in_block ? row / TB : 0);
+    const int t = in_block ? t0 + row % TB : A.T;
     const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16) + kTmemO + 64u * (uint32_t)hf;
     float o[64];
 #pragma unroll
@@ -466,17 +479,18 @@ cudaError_t launch_attn_prefill(const LaunchAttnPrefill& a, cudaStream_t stream)
   A.o_bf16 = a.o_bf16 ? 1 : 0;
   A.err = a.err;
   A.budget = wait_budget_cycles();
+  A.TB = prefill_tokens_per_block(A.G);
   CUtensorMap qmap, kmap, vmap, qimap{}, kimap{};
-  if (!make_row_map(&qmap, a.q, a.B, a.Hq, a.T, kAtRows)) return cudaErrorInvalidValue;
+  if (!make_row_map(&qmap, a.q, a.B, a.Hq, a.T, A.TB)) return cudaErrorInvalidValue;
   if (!make_row_map(&kmap, a.k, a.B, a.Hk, a.N, kAtKeys)) return cudaErrorInvalidValue;
   if (!make_row_map(&vmap, a.v, a.B, a.Hk, a.N, kAtKeys)) return cudaErrorInvalidValue;
   const size_t smem = sizeof(AtSmem) + 1024;
-  const dim3 grid((unsigned)((a.T + kAtRows - 1) / kAtRows), (unsigned)(a.B * a.Hq));
+  const dim3 grid((unsigned)((a.T + A.TB - 1) / A.TB), (unsigned)(a.B * a.Hk));
   if (a.W > 0) {
     cudaFuncSetAttribute(attn_prefill_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     attn_prefill_kernel<false><<<grid, kAtThreads, smem, stream>>>(qmap, kmap, vmap, qimap, kimap, A);
   } else {
-    if (!make_idx_map(&qimap, a.q_idx, a.B, a.Hq, a.T, kAtRows)) return cudaErrorInvalidValue;
+    if (!make_idx_map(&qimap, a.q_idx, a.B, a.Hq, a.T, A.TB)) return cudaErrorInvalidValue;
     if (!make_idx_map(&kimap, a.k_idx, a.B, a.Hk, a.N, kAtKeys)) return cudaErrorInvalidValue;
     cudaFuncSetAttribute(attn_prefill_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     attn_prefill_kernel<true><<<grid, kAtThreads, smem, stream>>>(qmap, kmap, vmap, qimap, kimap, A);

@@ -82,6 +82,12 @@ struct LaunchToppPrefill {
 };
 cudaError_t launch_topp_prefill(const LaunchToppPrefill& a, cudaStream_t stream);
 
+// Prefill kernels pack the G = Hq / Hk query heads of one KV head into a block
+// of 128 rows: TB tokens per head, TB = 128 / G rounded down to a multiple of 8
+// (the TMA swizzle atom); G must be at most 16.
+inline int prefill_tokens_per_block(int G) { return (128 / G) & ~7; }
+constexpr int kPrefillMaxGroup = 16;
+
 // Prefill attention (T query tokens per sequence, bf16): sparse form (threshold
 // selection + projected tiles) when W == 0, sliding window when W > 0.
 struct LaunchAttnPrefill {

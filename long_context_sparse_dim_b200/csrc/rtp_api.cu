@@ -144,6 +144,7 @@ rtp_status rtp_topp_select(const rtp_tensor* q_idx, const rtp_tensor* k_idx, con
     return s;
   if (T != 1) {
     if (q_idx->dtype != RTP_BF16) return RTP_ERR_DTYPE;  // the tensor-core score tiles take bf16
+    if (q_idx->shape[1] / k_idx->shape[1] > rtp::kPrefillMaxGroup) return RTP_ERR_UNSUPPORTED;
     rtp::LaunchToppPrefill a;
     a.q_idx = view(q_idx);
     a.k_idx = view(k_idx);
@@ -270,6 +271,7 @@ rtp_status rtp_sparse_attn_prefill(const rtp_tensor* q, const rtp_tensor* k, con
   if (q->dtype != RTP_BF16 || q_idx->dtype != RTP_BF16 || k_idx->dtype != RTP_BF16) return RTP_ERR_DTYPE;
   if (!same_bhn(q, q_idx) || !same_bhn(k, k_idx)) return RTP_ERR_SHAPE;
   if (q->shape[2] > k->shape[2]) return RTP_ERR_SHAPE;
+  if (q->shape[1] / k->shape[1] > rtp::kPrefillMaxGroup) return RTP_ERR_UNSUPPORTED;
   rtp::LaunchAttnPrefill a;
   a.q = view(q);
   a.k = view(k);
@@ -312,6 +314,7 @@ rtp_status rtp_window_attn(const rtp_tensor* q, const rtp_tensor* k, const rtp_t
   if (T != 1) {
     if (q->dtype != RTP_BF16) return RTP_ERR_DTYPE;  // the prefill kernels take bf16
     if (T > N) return RTP_ERR_SHAPE;
+    if (q->shape[1] / k->shape[1] > rtp::kPrefillMaxGroup) return RTP_ERR_UNSUPPORTED;
     rtp::LaunchAttnPrefill a;
     a.q = view(q);
     a.k = view(k);

@@ -39,9 +39,8 @@
 // (KEY) until one value is left; a TIE sweep then counts the keys above it and
 // locates the ties in position order.
 // Every bracket is an interval (vlo, vhi] of raw accumulators, precomputed
-// once per row and sweep, so testing a key costs two compares; keys inside a
-// bracket (rare after LIN 1) are handled per column with a warp-uniform
-// ballot.  Masses are integers, so the cut does not depend on the order in
+// once per row and sweep, so testing a key costs two compares; each thread
+// then walks its own keys inside the bracket.  Masses are integers, so the cut does not depend on the order in
 // which threads add them.
 #include <math.h>
 
@@ -101,6 +100,8 @@ struct PfSmem {
 struct PfArgs {
   const int32_t* lens;
   int Hq, Hk, G, T, N;
+  int TB;  // tokens per block
+  int GP;  // query heads per block (TB * GP <= 128 rows)
   float p;
   float two_pow_frac;
   uint32_t* tau_bits;
@@ -159,18 +160,21 @@ topp_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   PfSmem& S = *reinterpret_cast<PfSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  // 1-D grid ordered longest causal prefix first across all heads, so every SM
-  // receives a mix of long and short blocks
-  const int nb = (A.T + kPfRows - 1) / kPfRows;
-  const int heads = (int)(gridDim.x / nb);
-  const int t0 = (nb - 1 - (int)blockIdx.x / heads) * kPfRows;
-  const int bh = (int)blockIdx.x % heads;
-  const int b = bh / A.Hq, h = bh % A.Hq, kvh = h / A.G;
+  // A block holds GP query heads of one KV head x TB consecutive tokens (row r:
+  // head hq0 + r / TB, token t0 + r % TB), so the projected-key tiles it
+  // streams serve all GP heads.  1-D grid ordered longest causal prefix
+  // first across all KV heads, so every SM receives a mix of long and short blocks.
+  const int TB = A.TB, GP = A.GP;  // GP query heads per block (all G of the group, or 1)
+  const int nb = (A.T + TB - 1) / TB;
+  const int hblocks = (int)(gridDim.x / nb);
+  const int t0 = (nb - 1 - (int)blockIdx.x / hblocks) * TB;
+  const int bg = (int)blockIdx.x % hblocks;
+  const int b = bg / (A.Hq / GP), hq0 = (bg % (A.Hq / GP)) * GP, kvh = hq0 / A.G;
   int n_b = A.N;
   if (A.lens) n_b = min(max(A.lens[b], 0), A.N);
   const int qbase = n_b - A.T;  // position of query token 0
   // keys needed by the block: 0 .. position of its last token
-  const int t_last = min(t0 + kPfRows, A.T) - 1;
+  const int t_last = min(t0 + TB, A.T) - 1;
   const int kmax = min(qbase + t_last, n_b - 1);
   const int ntiles = kmax >= 0 ? kmax / kPfKeys + 1 : 0;
   const int64_t words = (A.N + 31) / 32;
@@ -198,10 +202,12 @@ topp_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
   const bool epi = warp < kPfEpiWarps;
   const int quad = warp & 3, half = (warp >> 2) & 1;
   const int row = quad * 32 + lane;
-  const int t = t0 + row;
+  const bool in_block = row < GP * TB;
+  const int h = hq0 + (in_block ? row / TB : 0);
+  const int t = in_block ? t0 + row % TB : A.T;
   const int pos = qbase + t;
   const bool owner = epi && half == 0;
-  const int64_t qrow = (int64_t)bh * A.T + t;
+  const int64_t qrow = ((int64_t)b * A.Hq + h) * A.T + t;
   int level = (epi && t < A.T && pos >= 0) ? kLvMax : kLvDone;
   uint32_t* mrow = (A.mask && epi && t < A.T) ? A.mask + qrow * A.mask_words : nullptr;
   if (owner && t < A.T && pos < 0) {  // a token before the sequence: no keys
@@ -244,8 +250,10 @@ topp_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
       // ---------------- TMA producer ----------------
       if (lane == 0) {
         if (sweep == 0) {
-          mbar_expect_tx(&S.q_full, kPfRows * kIdxDim * 2);
-          tma_load_4d(S.qtile, &qmap, &S.q_full, 0, t0, h, b);
+          // one box of TB rows per head of the group; rows past G * TB stay unused
+          mbar_expect_tx(&S.q_full, GP * TB * kIdxDim * 2);
+          for (int g = 0; g < GP; ++g)
+            tma_load_4d(S.qtile + g * TB * kIdxDim * 2, &qmap, &S.q_full, 0, t0, hq0 + g, b);
           q_issued = true;
         }
         for (int i = 0; i < ntiles; ++i) {
@@ -344,8 +352,7 @@ topp_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
             }
           }
           {
-            // bracket levels: two compares per key, keys inside handled column by column.  The
-            // warp-wide votes below are reached by every lane whatever its row's level.
+            // bracket levels: two compares per key; the keys inside are handled one by one
             uint32_t inb = 0u, above = 0u;
             if (bracket && own) {
 #pragma unroll
@@ -357,12 +364,17 @@ topp_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
               inb &= vmask;
               if (level == kLvCollect) ngt += __popc(above & vmask);
             }
-            if (__any_sync(0xffffffffu, inb != 0u)) {
+            if (inb) {
+              // each lane walks its own keys inside the bracket (about one in twelve at
+              // the first linear level, far fewer later): the chunk goes to a small
+              // per-thread array so that a key can be picked by its column
+              float xs[32];
 #pragma unroll
-              for (int j = 0; j < 32; ++j) {
-                if (__ballot_sync(0xffffffffu, (inb >> j) & 1u) == 0u) continue;
-                if (!((inb >> j) & 1u)) continue;
-                const float x = __uint_as_float(v[j]);
+              for (int j = 0; j < 32; ++j) xs[j] = __uint_as_float(v[j]);
+              while (inb) {
+                const int j = __ffs(inb) - 1;
+                inb &= inb - 1u;
+                const float x = xs[j];
                 const float u = __fsub_rn(mh, x);
                 if (level == kLvLin) {
                   const int d = min(max((int)__fmul_rn(u, dscale) - 32 * prefix, 0), kPfBins - 1);
@@ -674,13 +686,15 @@ cudaError_t launch_topp_prefill(const LaunchToppPrefill& a, cudaStream_t stream)
     topp_prefill_all_kernel<<<(unsigned)((rows + 255) / 256), 256, 0, stream>>>(A, (int)rows);
     return cudaGetLastError();
   }
+  A.GP = A.G;
+  A.TB = prefill_tokens_per_block(A.GP);
   CUtensorMap qmap, kmap;
-  if (!make_idx_map(&qmap, a.q_idx, a.B, a.Hq, a.T, kPfRows)) return cudaErrorInvalidValue;
+  if (!make_idx_map(&qmap, a.q_idx, a.B, a.Hq, a.T, A.TB)) return cudaErrorInvalidValue;
   if (!make_idx_map(&kmap, a.k_idx, a.B, a.Hk, a.N, kPfKeys)) return cudaErrorInvalidValue;
   const size_t smem = sizeof(PfSmem) + 1024;
   cudaFuncSetAttribute(topp_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   cudaFuncSetAttribute(topp_prefill_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-  const dim3 grid((unsigned)(((a.T + kPfRows - 1) / kPfRows) * a.B * a.Hq));
+  const dim3 grid((unsigned)(((a.T + A.TB - 1) / A.TB) * a.B * (a.Hq / A.GP)));
   topp_prefill_kernel<<<grid, kPfThreads, smem, stream>>>(qmap, kmap, A);
   return cudaGetLastError();
 }
