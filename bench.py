@@ -388,6 +388,8 @@ def run_ours(args, wl, rank, world, local_rank):
 
     # end to end through the public API with host buffers
     e2e = _e2e(layer, inst, wl, dev, max(args.steps, E2E_MIN_STEPS))
+    dense = _dense_decode(layer, wl, dev, step_ms)
+    budget = _budget_decode(layer, wl)
 
     line = {
         "metric": METRIC, "value": world * wl.B / (step_ms * 1e-3), "unit": "tokens/s", "n_gpus": world,
@@ -411,6 +413,8 @@ def run_ours(args, wl, rank, world, local_rank):
         "selection": {"mean_selected_fraction": sel_rows / (wl.B * R * G * wl.N),
                       "mean_group_union_fraction": union_rows / (wl.B * R * wl.N)},
         "e2e": e2e,
+        "dense_comparator": dense,
+        "budget": budget,
         "gpu_launches": 5 * args.steps,
         "streams": "window attention (local heads) forked onto a second stream after the projections",
         "timing_events": f"around both attention launches of every {EVENT_EVERY}th timed step",
@@ -428,6 +432,54 @@ def run_ours(args, wl, rank, world, local_rank):
     if rank == 0:
         print(json.dumps(line), flush=True)
     return 0
+
+
+PAGES_SPEEDUP = "the pages report up to 9.36x prefill at 1M context and ~2.01x decode over full attention " \
+                "(hardware, precision and baseline not stated; context only)"
+
+
+def _timed(fn, reps):
+    import torch
+    fn()
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(reps):
+        fn()
+    b.record()
+    b.synchronize()
+    return a.elapsed_time(b) / reps
+
+
+def _dense_decode(layer, wl, dev, step_ms, reps=200):
+    """Our own dense comparator: every query head attends all n cached keys
+    (rtp_window_attn with W = N over all heads), against the sparse step."""
+    import torch
+    from long_context_sparse_dim_b200 import rtp
+    o = torch.empty(layer.q.shape, dtype=torch.float32, device=dev)
+    ws = rtp.workspace(rtp.window_attn_workspace_size(wl.B, wl.Hq, 1, wl.Hkv, wl.N, wl.N), dev)
+    ms = _timed(lambda: rtp.window_attn(layer.q, layer.k, layer.v, layer.lens, wl.N, layer.scale, o, ws), reps)
+    return {"kernel": "rtp_window_attn with W = N over all query heads (full attention, same kernel as the "
+                      "local heads)", "ms": ms, "sparse_step_ms": step_ms, "speedup": ms / step_ms,
+            "bytes": wl.B * wl.Hkv * wl.N * ROW_BYTES[wl.dtype], "pages": PAGES_SPEEDUP}
+
+
+def _budget_decode(layer, wl, reps=200):
+    """Dynamic top-p against a fixed top-k budget of the same mean size: the
+    spread of the per-query counts, and the cost of both selections."""
+    import torch
+    from long_context_sparse_dim_b200 import rtp
+    cnt = layer.sel.count.cpu().numpy().astype(np.float64)
+    k = max(int(round(cnt.mean())), 1)
+    sel_k = rtp.Selection.empty(layer.sel.count.numel(), wl.N, layer.q.device)
+    topp_ms = _timed(lambda: rtp.topp_select(layer.q_idx, layer.k_idx, layer.lens, layer.p, layer.sel,
+                                             layer.ws_sel), reps)
+    topk_ms = _timed(lambda: rtp.topk_select(layer.q_idx, layer.k_idx, layer.lens, k, sel_k, layer.ws_sel), reps)
+    return {"topp_p": wl.p, "topp_count": {"min": int(cnt.min()), "mean": float(cnt.mean()),
+                                            "max": int(cnt.max()), "std": float(cnt.std())},
+            "topk_k": k, "topp_select_ms": topp_ms, "topk_select_ms": topk_ms,
+            "queries": int(cnt.size)}
 
 
 def _step_with_events(layer, ev, side):
@@ -628,6 +680,16 @@ def measure_prefill(args, wl, dev, world, steps, warmup, with_cpu):
         "streams": "window attention (local heads) forked onto a second stream inside each step",
         "clocks": clock_info,
     }
+    # our own dense comparator: causal full attention of every query head (W = N)
+    o_dense = torch.empty(layer.o.shape, dtype=layer.o.dtype, device=dev)
+    dense_ms = _timed(lambda: rtp.window_attn(layer.q, layer.k, layer.v, layer.lens, N, layer.scale, o_dense,
+                                              None), max(1, min(steps, 3)))
+    out["dense_comparator"] = {"kernel": "rtp_window_attn with W = N over all query heads (causal full "
+                                         "attention, same tcgen05 kernel as the local heads)",
+                               "ms": dense_ms, "sparse_step_ms": step_ms, "speedup": dense_ms / step_ms,
+                               "flop": 4.0 * 128 * int((pos + 1).sum()) * wl.Hq,
+                               "pages": PAGES_SPEEDUP}
+    del o_dense
     out["e2e"] = _e2e_prefill(layer, inst, dev, side, max(1, min(steps, 3)))
     if with_cpu:
         out["cpu_baseline"] = cpu_baseline_prefill(inst, wl, args.cpu_budget)

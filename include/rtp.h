@@ -134,6 +134,20 @@ RTP_API rtp_status rtp_topp_select(const rtp_tensor* q_idx, const rtp_tensor* k_
                            rtp_stream_t stream);
 RTP_API size_t rtp_topp_select_workspace_size(int64_t B, int64_t Hq, int64_t T, int64_t Hk, int64_t N);
 
+/* ---- a3 variant: a fixed top-k cut through the same selection -------------
+ * Decode form (T == 1) only; arguments and results as rtp_topp_select, with k
+ * in place of p: query (b, h) keeps the min(k, n) keys of highest indexer
+ * score s (ties to the lower position), n = lens[b] (or N).  k < 1 is
+ * RTP_ERR_INVALID_ARG, T != 1 RTP_ERR_UNSUPPORTED.  The kernel is the top-p
+ * selection's with every key weighing 1, so its passes count keys.
+ * Cites: "Full Attention Strikes Back ... (RTPurbo)", Key findings (dynamic
+ * top-p set against a fixed top-k budget); "RTPurbo: Turning Dense LLMs ...",
+ * "Three Key Insights" 3.  Workspace: rtp_topp_select_workspace_size().
+ */
+RTP_API rtp_status rtp_topk_select(const rtp_tensor* q_idx, const rtp_tensor* k_idx, const int32_t* lens,
+                                   int32_t k, const rtp_selection* out, void* workspace, size_t workspace_bytes,
+                                   rtp_stream_t stream);
+
 /* ---- a4 (decode): exact attention over each query's selected keys -------
  *   q      [B, Hq, 1, 128]  bf16 or f32 (retrieval query heads)
  *   k, v   [B, Hk, N, 128]  same dtype (full KV cache of the retrieval heads)

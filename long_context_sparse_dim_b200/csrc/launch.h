@@ -56,6 +56,7 @@ struct LaunchToppDecode {
   const int32_t* lens;
   int64_t B, Hq, Hk, N;
   float p;
+  int32_t topk;  // > 0: keep the topk highest-scoring keys instead of the top-p mass
   bool bf16;
   uint32_t* tau_bits;
   int32_t* tiepos;

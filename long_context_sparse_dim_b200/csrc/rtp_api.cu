@@ -174,6 +174,45 @@ rtp_status rtp_topp_select(const rtp_tensor* q_idx, const rtp_tensor* k_idx, con
   a.Hk = k_idx->shape[1];
   a.N = N;
   a.p = p;
+  a.topk = 0;
+  a.bf16 = q_idx->dtype == RTP_BF16;
+  a.tau_bits = out->tau_bits;
+  a.tiepos = out->tiepos;
+  a.count = out->count;
+  a.mask = out->mask;
+  a.mask_words = out->mask_words;
+  return cuda_status(rtp::launch_topp_decode(a, (cudaStream_t)stream));
+}
+
+rtp_status rtp_topk_select(const rtp_tensor* q_idx, const rtp_tensor* k_idx, const int32_t* lens, int32_t k,
+                           const rtp_selection* out, void* workspace, size_t workspace_bytes,
+                           rtp_stream_t stream) {
+  rtp_status s;
+  if ((s = check4(q_idx, 16)) != RTP_OK) return s;
+  if ((s = check4(k_idx, 16)) != RTP_OK) return s;
+  if (q_idx->dtype != k_idx->dtype) return RTP_ERR_DTYPE;
+  if (q_idx->shape[0] != k_idx->shape[0]) return RTP_ERR_SHAPE;
+  if (k_idx->shape[1] < 1 || q_idx->shape[1] % k_idx->shape[1]) return RTP_ERR_SHAPE;
+  if (k < 1) return RTP_ERR_INVALID_ARG;
+  if (!out || !out->tau_bits || !out->tiepos || !out->count) return RTP_ERR_INVALID_ARG;
+  const int64_t N = k_idx->shape[2];
+  if (out->mask && out->mask_words < (N + 31) / 32) return RTP_ERR_SHAPE;
+  if (q_idx->shape[2] != 1) return RTP_ERR_UNSUPPORTED;  // decode form only
+  if ((s = check_workspace(workspace, workspace_bytes,
+                           rtp_topp_select_workspace_size(q_idx->shape[0], q_idx->shape[1], 1, k_idx->shape[1],
+                                                          N))) != RTP_OK)
+    return s;
+  if (!rtp::topp_decode_supported(N)) return RTP_ERR_UNSUPPORTED;
+  rtp::LaunchToppDecode a;
+  a.q_idx = view(q_idx);
+  a.k_idx = view(k_idx);
+  a.lens = lens;
+  a.B = q_idx->shape[0];
+  a.Hq = q_idx->shape[1];
+  a.Hk = k_idx->shape[1];
+  a.N = N;
+  a.p = 1.f;
+  a.topk = k;
   a.bf16 = q_idx->dtype == RTP_BF16;
   a.tau_bits = out->tau_bits;
   a.tiepos = out->tiepos;

@@ -1,4 +1,5 @@
-// a2 + a3 (decode): indexer scores of every cached key and the dynamic top-p cut.
+// a2 + a3 (decode): indexer scores of every cached key and the dynamic top-p cut
+// (or, through the same passes with every key weighing 1, a fixed top-k cut).
 //
 // "RTPurbo: Turning Dense LLMs into Sparse Attention Models with Just a Few
 // Hundred Training Steps", "Three Key Insights" 3: per query, cumulative top-p
@@ -117,9 +118,11 @@ RTP_DEVICE float ex2f_fast(float x) {
   return y;
 }
 
-// Fixed-point top-p weight round(2^((s - m) log2 e) * 2^frac).  Every use of a
-// weight in the cut goes through this one function.
-RTP_DEVICE uint64_t sel_weight(float s, float m, float two_pow_frac) {
+// Fixed-point top-p weight round(2^((s - m) log2 e) * 2^frac), or 1 for the
+// fixed top-k cut (`unit`): the same passes then count keys instead of weighing
+// them.  Every use of a weight in the cut goes through this one function.
+RTP_DEVICE uint64_t sel_weight(float s, float m, float two_pow_frac, bool unit) {
+  if (unit) return 1ull;
   const float e = ex2f_fast(__fmul_rn(__fsub_rn(s, m), 1.4426950408889634f));
   return __float2ull_rn(__fmul_rn(e, two_pow_frac));
 }
@@ -180,11 +183,12 @@ RTP_DEVICE void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.
 RTP_DEVICE void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;\n" ::: "memory"); }
 
 // Cluster-wide histogram of `hb` (256 bins) and the bin holding the cut:
-// with `first`, Z = total mass and target = ceil(p Z) are set first.  Bins are
+// with `first`, Z = total mass and target = ceil(p Z) are set first (for the
+// top-k cut, Z is the number of keys and the target min(k, Z)).  Bins are
 // taken in descending score order (`ascending_bins`: bin 0 holds the highest
 // scores).  Returns the cut bin; mass_above grows by the mass before it.
 RTP_DEVICE int cluster_cut(SelSmem& S, cg::cluster_group& cluster, const uint64_t* hb, bool first,
-                           bool ascending_bins, float p, uint64_t& target, uint64_t& mass_above) {
+                           bool ascending_bins, float p, int topk, uint64_t& target, uint64_t& mass_above) {
   const int tid = threadIdx.x;
   const int C = (int)cluster.num_blocks();
   cluster.sync();  // every CTA's histogram of this pass is complete
@@ -201,10 +205,14 @@ RTP_DEVICE int cluster_cut(SelSmem& S, cg::cluster_group& cluster, const uint64_
   }
   uint64_t excl, Z;
   const uint64_t incl = block_scan_u64(mine, S.wsum, excl, &Z);
-  if (first) {  // Z = total mass; target = ceil(p Z)
-    const double t = ceil((double)p * (double)Z);
-    const uint64_t tt = t >= (double)Z ? Z : (uint64_t)t;
-    target = tt < 1 ? 1 : tt;
+  if (first) {  // Z = total mass; target = ceil(p Z), or min(k, Z) keys
+    if (topk > 0) {
+      target = (uint64_t)topk < Z ? (uint64_t)topk : Z;
+    } else {
+      const double t = ceil((double)p * (double)Z);
+      const uint64_t tt = t >= (double)Z ? Z : (uint64_t)t;
+      target = tt < 1 ? 1 : tt;
+    }
   }
   const uint64_t need = target - mass_above;  // >= 1
   if (excl < need && need <= incl) {  // exactly one position holds the cut
@@ -224,7 +232,7 @@ RTP_DEVICE int cluster_cut(SelSmem& S, cg::cluster_group& cluster, const uint64_
 // the words of the keys above bin fb before the candidate barrier).  `need` is
 // the mass still to take inside bin fb: >= 1 and <= the bin's mass, which the
 // candidates' weights add up to exactly.
-RTP_DEVICE void resolve_candidates(SelSmem& S, int n, int fb, float m, float two_pow_frac, uint64_t need,
+RTP_DEVICE void resolve_candidates(SelSmem& S, int n, int fb, float m, float two_pow_frac, bool unit, uint64_t need,
                                    uint32_t* mrow, int qrow, uint32_t* tau_bits, int32_t* tiepos,
                                    int32_t* count) {
   const int tid = threadIdx.x;
@@ -242,7 +250,7 @@ RTP_DEVICE void resolve_candidates(SelSmem& S, int n, int fb, float m, float two
   for (int j = tid; j < n; j += kSelThreads) {
     const float sc = S.cand_s[j];
     const int d = sub_bin(sc, m, fb);
-    add_u64_pair(&S.u.r.lo[d], &S.u.r.hi[d], sel_weight(sc, m, two_pow_frac));
+    add_u64_pair(&S.u.r.lo[d], &S.u.r.hi[d], sel_weight(sc, m, two_pow_frac, unit));
     atomicAdd(&S.u.r.cnt[d], 1u);
   }
   __syncthreads();
@@ -284,7 +292,7 @@ RTP_DEVICE void resolve_candidates(SelSmem& S, int n, int fb, float m, float two
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
     const int idx = 4 * tid + k;
-    wv[k] = idx < ns ? sel_weight(S.u.r.ss[idx], m, two_pow_frac) : 0;
+    wv[k] = idx < ns ? sel_weight(S.u.r.ss[idx], m, two_pow_frac, unit) : 0;
     tot += wv[k];
   }
   uint64_t run;
@@ -320,7 +328,7 @@ RTP_DEVICE void resolve_candidates(SelSmem& S, int n, int fb, float m, float two
 template <typename T>
 __global__ void __maxnreg__(96)
 topp_query_kernel(View4 qv, View4 kv, const int32_t* __restrict__ lens, int Hq, int G, int N,
-                   int n_chunk, float p, float two_pow_frac, uint32_t* __restrict__ tau_bits,
+                   int n_chunk, float p, int topk, float two_pow_frac, uint32_t* __restrict__ tau_bits,
                    int32_t* __restrict__ tiepos, int32_t* __restrict__ count,
                    uint32_t* __restrict__ mask, int64_t mask_words) {
   pdl_wait();
@@ -331,6 +339,7 @@ topp_query_kernel(View4 qv, View4 kv, const int32_t* __restrict__ lens, int Hq, 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int qrow = blockIdx.x / C;
   const int b = qrow / Hq, h = qrow % Hq, kvh = h / G;
+  const bool unit = topk > 0;  // fixed top-k: every key weighs 1
 
   extern __shared__ __align__(16) unsigned char smem_raw[];
   SelSmem& S = *reinterpret_cast<SelSmem*>(smem_raw);
@@ -346,7 +355,7 @@ topp_query_kernel(View4 qv, View4 kv, const int32_t* __restrict__ lens, int Hq, 
 
   // Trivial cuts: no candidates, or p >= 1 (every candidate).  Uniform over the
   // cluster, taken before any distributed-shared-memory access.
-  if (n_b == 0 || p >= 1.f) {
+  if (n_b == 0 || (!unit && p >= 1.f) || (unit && topk >= n_b)) {
     const bool all = n_b > 0;
     for (int wi = tid; wi * 32 < n_chunk; wi += kSelThreads) {
       const int w = (c0 >> 5) + wi;
@@ -430,7 +439,7 @@ topp_query_kernel(View4 qv, View4 kv, const int32_t* __restrict__ lens, int Hq, 
       const int i = base + u * kSelThreads + tid;
       if (i < nloc) {
         const int f = fine_bin(sc[u], m);
-        add_u64_pair(&S.u.f.lo[f], &S.u.f.hi[f], sel_weight(sc[u], m, two_pow_frac));
+        add_u64_pair(&S.u.f.lo[f], &S.u.f.hi[f], sel_weight(sc[u], m, two_pow_frac, unit));
       }
     }
   }
@@ -446,7 +455,7 @@ topp_query_kernel(View4 qv, View4 kv, const int32_t* __restrict__ lens, int Hq, 
     S.hist[0][tid] = a;
   }
   uint64_t target = 0, mass_above = 0;
-  const int lin = cluster_cut(S, cluster, S.hist[0], true, true, p, target, mass_above);
+  const int lin = cluster_cut(S, cluster, S.hist[0], true, true, p, topk, target, mass_above);
 
   if (lin < kBins - 1) {
     // ---- the fine bin of the cut, from the 16 fine bins under coarse bin lin --
@@ -516,7 +525,7 @@ topp_query_kernel(View4 qv, View4 kv, const int32_t* __restrict__ lens, int Hq, 
     const uint32_t ntot = *cluster.map_shared_rank(&S.ncand, 0);
     cluster_arrive();  // this CTA's last distributed access
     if (ntot <= (uint32_t)kCandCap) {
-      if (rank == 0) resolve_candidates(S, (int)ntot, fb, m, two_pow_frac, target - S.fine_above, mrow, qrow,
+      if (rank == 0) resolve_candidates(S, (int)ntot, fb, m, two_pow_frac, unit, target - S.fine_above, mrow, qrow,
                                         tau_bits, tiepos, count);
       // rank 0 keeps its shared memory until every CTA has read the candidate total
       if (rank == 0) cluster_wait();
@@ -555,7 +564,7 @@ topp_query_kernel(View4 qv, View4 kv, const int32_t* __restrict__ lens, int Hq, 
         const uint32_t k = score_key(sc);
         if (k >= kbase && (uint64_t)k < kend) {
           const int d = (int)((uint64_t)(k - kbase) >> shift);
-          add_u64_pair(&wlo[d], &whi[d], sel_weight(sc, m, two_pow_frac));
+          add_u64_pair(&wlo[d], &whi[d], sel_weight(sc, m, two_pow_frac, unit));
         }
       }
     }
@@ -568,7 +577,7 @@ topp_query_kernel(View4 qv, View4 kv, const int32_t* __restrict__ lens, int Hq, 
       hb[tid] = a;
     }
     // digit bins: bin 255 holds the highest keys
-    const int cb = cluster_cut(S, cluster, hb, false, false, p, target, mass_above);
+    const int cb = cluster_cut(S, cluster, hb, false, false, p, topk, target, mass_above);
     kbase += (uint32_t)cb << shift;
     const uint64_t e = (uint64_t)kbase + (uint64_t(1) << shift);
     kend = e < kend ? e : kend;
@@ -612,7 +621,7 @@ topp_query_kernel(View4 qv, View4 kv, const int32_t* __restrict__ lens, int Hq, 
     tau_cnt += S.tcount[r];
     if (r < rank) before += (int)S.tcount[r];
   }
-  const uint64_t w_tau = sel_weight(tau, m, two_pow_frac);
+  const uint64_t w_tau = sel_weight(tau, m, two_pow_frac, unit);
   const uint64_t rem = target - mass_above;
   uint64_t n_tau64 = w_tau ? (rem + w_tau - 1) / w_tau : (uint64_t)tau_cnt;
   if (n_tau64 < 1) n_tau64 = 1;
@@ -695,11 +704,11 @@ cudaError_t launch_topp_decode(const LaunchToppDecode& a, cudaStream_t stream) {
   const size_t smem = sizeof(SelSmem) + (size_t)n_chunk * sizeof(float);
   if (a.bf16)
     return launch_cluster(topp_query_kernel<__nv_bfloat16>, (int)(Q * C), C, smem, stream, a.q_idx, a.k_idx, a.lens,
-                          (int)a.Hq, G, (int)a.N, (int)n_chunk, a.p, two_pow_frac, a.tau_bits, a.tiepos, a.count,
-                          a.mask, a.mask_words);
+                          (int)a.Hq, G, (int)a.N, (int)n_chunk, a.p, (int)a.topk, two_pow_frac, a.tau_bits, a.tiepos,
+                          a.count, a.mask, a.mask_words);
   return launch_cluster(topp_query_kernel<float>, (int)(Q * C), C, smem, stream, a.q_idx, a.k_idx, a.lens, (int)a.Hq,
-                        G, (int)a.N, (int)n_chunk, a.p, two_pow_frac, a.tau_bits, a.tiepos, a.count, a.mask,
-                        a.mask_words);
+                        G, (int)a.N, (int)n_chunk, a.p, (int)a.topk, two_pow_frac, a.tau_bits, a.tiepos, a.count,
+                        a.mask, a.mask_words);
 }
 
 }  // namespace rtp

@@ -26,11 +26,11 @@
 // around the cut score.  All arithmetic is on the raw accumulator v = 4 s (the
 // score scaling is exact), with u = m - v for the row maximum m:
 //   MAX      row maximum m (3-input max, two independent halves)
-//   LIN0     32 bins of u (1/4 nat each, the last one the tail u >= 31), with
+//   LIN0     32 bins of u, 1/4 nat each (1/2 nat for caches longer than 2^17
+//            keys, whose cut can lie deeper), the last one the tail, with
 //            64-bit fixed-point masses; Z is their sum
-//   LIN 1-3  32 sub-bins of the previous cut bin (widths 1/128, 1/4096,
-//            1/131072 nat; power-of-two rescaling of u is exact), masses and
-//            counts
+//   LIN 1-3  32 sub-bins of the previous cut bin (each level 32 times finer;
+//            power-of-two rescaling of u is exact), masses and counts
 //   COLLECT  once the cut bin holds <= 32 keys, their (v, position) pairs are
 //            kept and sorted by (score desc, position asc) to finish the cut
 //   MASK     (only when a mask is requested) one more sweep writes it
@@ -71,7 +71,7 @@ struct PfRowState {
   int level;
   float m;         // raw row maximum
   float vlo, vhi;  // bracket: raw accumulators v with vlo < v <= vhi
-  float dscale;    // LIN: 32^lin
+  float dscale;    // LIN: c0 * 32^lin
   int prefix;      // LIN: full bin index of the bracket at the previous level
   uint32_t kbase;  // KEY: lowest score key of the digit range
   int shift;       // KEY: digit shift
@@ -102,6 +102,7 @@ struct PfArgs {
   int Hq, Hk, G, T, N;
   int TB;  // tokens per block
   int GP;  // query heads per block (TB * GP <= 128 rows)
+  float c0;  // level-0 bins per raw unit (1, or 1/2 for long caches: a 16-nat range before the tail)
   float p;
   float two_pow_frac;
   uint32_t* tau_bits;
@@ -217,7 +218,7 @@ topp_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
     if (mrow)
       for (int64_t w = 0; w < words; ++w) mrow[w] = 0u;
   }
-  float m = -INFINITY, vlo = 0.f, vhi = 0.f, dscale = 1.f, vtau = 0.f;
+  float m = -INFINITY, vlo = 0.f, vhi = 0.f, dscale = A.c0, vtau = 0.f;
   int prefix = 0, shift = 0, tiepos = -1, ngt = 0, neq = 0, ncand = 0;
   uint32_t kbase = 0;
   uint64_t kend = 0;
@@ -339,7 +340,7 @@ topp_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
               for (int j = 0; j < 32; j += 2) {
                 const float u0 = __fsub_rn(mh, __uint_as_float(v[j]));
                 const float u1 = __fsub_rn(mh, __uint_as_float(v[j + 1]));
-                const int d0 = lin0_bin(u0), d1 = lin0_bin(u1);
+                const int d0 = lin0_bin(__fmul_rn(u0, A.c0)), d1 = lin0_bin(__fmul_rn(u1, A.c0));
                 const uint64_t w0 = j < nv ? pf_weight_u(u0, wmul, A.two_pow_frac) : 0ull;
                 const uint64_t w1 = j + 1 < nv ? pf_weight_u(u1, wmul, A.two_pow_frac) : 0ull;
                 const uint64_t h0 = H[d0 * kPfRows], h1 = H[d1 * kPfRows];
@@ -533,15 +534,16 @@ topp_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
         mass_above += cum;
         if (level == kLvLin0 || level == kLvLin) {
           if (level == kLvLin0 && cut == kPfBins - 1) {
-            // tail bin (u >= 31, i.e. s <= max s - 7.75): exact digits over its keys
-            const float hi_s = __fmul_rn(__fsub_rn(m, 31.f), 0.25f);
+            // tail bin (u >= 31 / c0, i.e. s <= max s - 7.75 / c0): exact digits over its keys
+            const float u_tail = 31.f / A.c0;  // exact: c0 is a power of two
+            const float hi_s = __fmul_rn(__fsub_rn(m, u_tail), 0.25f);
             const float mg = 1e-5f * (fabsf(hi_s) + 8.f) + 1e-30f;
             kbase = 0u;
             kend = (uint64_t)score_key(__fadd_rn(hi_s + mg, 0.0f)) + 1;
             shift = 0;
             while (((kend - kbase - 1) >> shift) >= (uint64_t)kPfBins) ++shift;
             vlo = -INFINITY;
-            vhi = vmax_u_ge(m, 31.f);
+            vhi = vmax_u_ge(m, u_tail);
             level = kLvKey;
           } else {
             const int in_bin = level == kLvLin0 ? 255 : (int)S.hcnt[0][cut][row];  // level 0 keeps no counts
@@ -686,6 +688,7 @@ cudaError_t launch_topp_prefill(const LaunchToppPrefill& a, cudaStream_t stream)
     topp_prefill_all_kernel<<<(unsigned)((rows + 255) / 256), 256, 0, stream>>>(A, (int)rows);
     return cudaGetLastError();
   }
+  A.c0 = a.N > (int64_t(1) << 17) ? 0.5f : 1.f;
   A.GP = A.G;
   A.TB = prefill_tokens_per_block(A.GP);
   CUtensorMap qmap, kmap;

@@ -23,7 +23,7 @@ RTP_F32, RTP_BF16 = 0, 1
 STATUS_NAMES = {0: "RTP_OK", 1: "RTP_ERR_INVALID_ARG", 2: "RTP_ERR_SHAPE", 3: "RTP_ERR_DTYPE",
                 4: "RTP_ERR_ALIGNMENT", 5: "RTP_ERR_WORKSPACE", 6: "RTP_ERR_CUDA", 7: "RTP_ERR_UNSUPPORTED"}
 
-EXPORTED = ("rtp_index_project", "rtp_topp_select", "rtp_topp_select_workspace_size",
+EXPORTED = ("rtp_index_project", "rtp_topp_select", "rtp_topp_select_workspace_size", "rtp_topk_select",
             "rtp_sparse_attn_decode", "rtp_sparse_attn_decode_workspace_size", "rtp_sparse_attn_decode_noalloc",
             "rtp_sparse_attn_prefill", "rtp_sparse_attn_prefill_workspace_size",
             "rtp_window_attn", "rtp_window_attn_workspace_size",
@@ -61,6 +61,7 @@ def _load() -> ctypes.CDLL:
         "rtp_index_project": ([T, T, T, vp], i32),
         "rtp_topp_select": ([T, T, vp, f32, S, vp, sz, vp], i32),
         "rtp_topp_select_workspace_size": ([i64, i64, i64, i64, i64], sz),
+        "rtp_topk_select": ([T, T, vp, i32, S, vp, sz, vp], i32),
         "rtp_sparse_attn_decode": ([T, T, T, vp, S, f32, T, vp, sz, vp], i32),
         "rtp_sparse_attn_decode_workspace_size": ([i64, i64, i64, i64], sz),
         "rtp_sparse_attn_decode_noalloc": ([T, T, T, vp, S, f32, T, vp], i32),
@@ -188,6 +189,14 @@ def topp_select(q_idx: torch.Tensor, k_idx: torch.Tensor, lens: Optional[torch.T
     _check(_lib.rtp_topp_select(ctypes.byref(tensor_desc(q_idx)), ctypes.byref(tensor_desc(k_idx)),
                                 _ptr(lens), float(p), ctypes.byref(sel.desc()), w, nb, _stream(stream)),
            "rtp_topp_select")
+
+
+def topk_select(q_idx: torch.Tensor, k_idx: torch.Tensor, lens: Optional[torch.Tensor], k: int,
+                sel: Selection, ws: Optional[torch.Tensor] = None, stream=None) -> None:
+    w, nb = _ws(ws)
+    _check(_lib.rtp_topk_select(ctypes.byref(tensor_desc(q_idx)), ctypes.byref(tensor_desc(k_idx)),
+                                _ptr(lens), int(k), ctypes.byref(sel.desc()), w, nb, _stream(stream)),
+           "rtp_topk_select")
 
 
 def sparse_attn_decode_workspace_size(B, Hq, Hk, N) -> int:

@@ -6,5 +6,5 @@ leg of ``bench.py`` -- never by the product path.
 from .rtp_oracle import (  # noqa: F401
     D_IDX, INDEXER_SCALE, LayerOracle, QueryResult, Selection, attend, index_project,
     indexer_scores, local_query, needle_recall, retrieval_query, round_bf16, round_storage,
-    topp_select, window_keys,
+    topk_select, topp_select, window_keys,
 )

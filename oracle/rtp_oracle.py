@@ -158,6 +158,26 @@ def topp_select(s: np.ndarray, p: float) -> Selection:
                      Z=Z, mass=float(w[chosen].sum()), order=order)
 
 
+def topk_select(s: np.ndarray, k: int) -> Selection:
+    """The fixed top-k budget the pages set dynamic top-p against ([A] "Key
+    findings", [B] insight 3): the min(k, n) keys of highest score, ties taken
+    by lower position (R3).  Same fields as ``topp_select`` (Z and mass are the
+    softmax masses of that set, for comparison)."""
+    s = np.asarray(s, dtype=np.float64)
+    n = s.shape[0]
+    if k < 1:
+        raise ValueError("k must be >= 1")
+    if n == 0:
+        return Selection(np.zeros(0, np.int64), 0, float("-inf"), -1, 0.0, 0.0, np.zeros(0, np.int64))
+    w = np.exp(s - s.max())
+    order = np.lexsort((np.arange(n), -s))
+    kk = min(k, n)
+    chosen = order[:kk]
+    last = int(order[kk - 1])
+    return Selection(idx=np.sort(chosen), count=kk, tau=float(s[last]), tiepos=last,
+                     Z=float(w.sum()), mass=float(w[chosen].sum()), order=order)
+
+
 # --------------------------------------------------------------------------
 # step 3: attention over a key set ([A] TL;DR "sparse attention", R7)
 # --------------------------------------------------------------------------

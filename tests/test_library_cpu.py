@@ -307,3 +307,16 @@ def test_wait_budget_setter_validates():
     with pytest.raises(rtp.RtpError):
         rtp.set_wait_budget_cycles(-1)
     rtp.set_wait_budget_cycles(0)  # restores the default
+
+
+def test_topk_select_validation():
+    rtp = _lib()
+    L = rtp.lib()
+    by = ctypes.byref
+    qi = _desc(rtp, [2, 8, 1, 16])
+    ki = _desc(rtp, [2, 2, 64, 16])
+    s = _sel(rtp)
+    assert L.rtp_topk_select(by(qi), by(ki), None, 0, by(s), None, 0, None) == 1          # k < 1
+    assert L.rtp_topk_select(by(qi), by(ki), None, 5, None, None, 0, None) == 1           # no selection
+    assert L.rtp_topk_select(by(_desc(rtp, [2, 8, 3, 16])), by(ki), None, 5, by(s), None, 0, None) == 7  # T != 1
+    assert L.rtp_topk_select(by(_desc(rtp, [2, 7, 1, 16])), by(ki), None, 5, by(s), None, 0, None) == 2

@@ -385,3 +385,64 @@ def test_gqa_mapping_and_head_roles():
                 assert o[0] == pytest.approx(pos)         # window of one key: the token itself
             else:
                 assert 0.0 < o[0] < pos                   # an average over keys 0 .. pos
+
+
+# --------------------------------------------------------------------------
+# the fixed top-k variant (the budget the pages set dynamic top-p against)
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("seed", range(6))
+def test_topk_k_one_is_the_first_argmax(seed):
+    # k = 1 keeps the first occurrence of the maximum (numpy's argmax), ties included
+    rng = np.random.default_rng(100 + seed)
+    s = np.round(rng.standard_normal(40), 1)       # rounded: repeated values
+    r = oracle.topk_select(s, 1)
+    assert r.count == 1 and int(r.idx[0]) == int(np.argmax(s))
+
+
+@pytest.mark.parametrize("seed,k", [(0, 3), (1, 10), (2, 39), (3, 40), (4, 55), (5, 17)])
+def test_topk_invariants(seed, k):
+    # |S| = min(k, n); every selected score >= every unselected one; among equal
+    # scores at the boundary the selected positions precede the unselected ones
+    rng = np.random.default_rng(200 + seed)
+    s = np.round(rng.standard_normal(40), 1)
+    r = oracle.topk_select(s, k)
+    n = s.size
+    assert r.count == min(k, n) == r.idx.size
+    sel = np.zeros(n, bool)
+    sel[r.idx] = True
+    if sel.all():
+        return
+    assert s[sel].min() >= s[~sel].max()
+    tau = s[sel].min()
+    assert np.flatnonzero(sel & (s == tau)).max() < np.flatnonzero(~sel & (s == tau)).min() \
+        if (~sel & (s == tau)).any() else True
+    # the k largest values, as a multiset, are numpy's partition
+    np.testing.assert_array_equal(np.sort(s[sel]), np.sort(np.partition(s, n - r.count)[n - r.count:]))
+
+
+def test_topk_all_equal_keeps_the_lowest_positions():
+    r = oracle.topk_select(np.zeros(30), 7)
+    np.testing.assert_array_equal(r.idx, np.arange(7))
+    assert r.tiepos == 6 and r.tau == 0.0
+
+
+def test_topk_rejects_k_below_one():
+    with pytest.raises(ValueError):
+        oracle.topk_select(np.zeros(3), 0)
+
+
+# --------------------------------------------------------------------------
+# needle recall counts needles inside their query's SELECTED set only
+# --------------------------------------------------------------------------
+
+def test_needle_recall_hand_case():
+    # query (0, 0, 0) selected keys {1, 4} out of candidates 0..5; its needles sit
+    # at key 4 (selected) and key 2 (a candidate that was NOT selected); a needle
+    # of a local head (no selection) is not counted
+    sel = oracle.Selection(idx=np.array([1, 4]), count=2, tau=0.0, tiepos=4, Z=1.0, mass=1.0,
+                           order=np.arange(6))
+    res = {(0, 0, 0): oracle.QueryResult(np.zeros(4), sel, np.zeros(6)),
+           (0, 5, 0): oracle.QueryResult(np.zeros(4), None, None)}
+    needles = [(0, 0, 0, 0, 4), (0, 0, 0, 0, 2), (0, 1, 5, 0, 3)]
+    assert oracle.needle_recall(res, needles) == (1, 2)

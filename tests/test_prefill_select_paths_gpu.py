@@ -138,3 +138,17 @@ def test_prefill_select_mixed_paths_in_one_block():
     q0 = choices[np.arange(T) % choices.size]
     _check(q0, k0, 0.9, "mixed p=0.9")
     _check(q0, k0, 0.9999, "mixed p=0.9999")
+
+
+def test_prefill_select_long_cache_wide_level0_bins():
+    # caches longer than 2^17 keys take level-0 bins of 1/2 nat (a 15.5-nat range
+    # before the tail bin): an ordinary cut, and a cut in the (deeper) tail bin
+    rng = np.random.default_rng(25)
+    N, T = 140000, 128
+    k0 = rng.standard_normal(N)
+    _check(np.full(T, 4.0), k0, 0.95, "long p=0.95", rows=range(0, T, 9))
+    k1 = 0.5 * rng.standard_normal(N)
+    k1[11] = 22.0
+    res = _check(np.full(T, 4.0), k1, 0.999999, "long tail", rows=range(0, T, 17))
+    for ref, *_ in res.values():
+        assert ref.tau < 22.0 - 15.5
