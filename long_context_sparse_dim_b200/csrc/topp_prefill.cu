@@ -124,6 +124,21 @@ RTP_DEVICE uint64_t pf_weight_u(float u, float wmul, float two_pow_frac) {
 
 RTP_DEVICE float canon_score(float v) { return __fadd_rn(__fmul_rn(v, 0.25f), 0.0f); }
 
+RTP_DEVICE float min3f(float a, float b, float c) {
+  float r;
+  asm("min.f32 %0, %1, %2, %3;\n" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// (a - c, b - c) in one packed fp32x2 instruction.
+RTP_DEVICE void sub2(float a, float b, float c, float& ra, float& rb) {
+  uint64_t x, y, z;
+  asm("mov.b64 %0, {%1, %2};\n" : "=l"(x) : "f"(a), "f"(b));
+  asm("mov.b64 %0, {%1, %2};\n" : "=l"(y) : "f"(c), "f"(c));
+  asm("sub.rn.f32x2 %0, %1, %2;\n" : "=l"(z) : "l"(x), "l"(y));
+  asm("mov.b64 {%0, %1}, %2;\n" : "=f"(ra), "=f"(rb) : "l"(z));
+}
+
 RTP_DEVICE float max3f(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;\n" : "=f"(r) : "f"(a), "f"(b), "f"(c));
@@ -286,6 +301,12 @@ topp_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
       // ---------------- epilogue: two threads per query row ----------------
       const float mh = m;
       const bool bracket = level == kLvLin || level == kLvKey || level == kLvCollect;
+      // the screen: past the first linear level (a bracket 1/32 as wide or less) and with
+      // finite bounds; bhw is the half width plus a margin for the rounding of x - c
+      const bool screen = (level == kLvCollect || (level == kLvLin && dscale > 32.f * A.c0)) &&
+                          vlo > -INFINITY && vhi < INFINITY;
+      const float bc = __fmaf_rn(0.5f, vlo, 0.5f * vhi);
+      const float bhw = 0.5f * (vhi - vlo) + 1e-6f * fmaxf(fabsf(vlo), fabsf(vhi)) + 1e-30f;
       for (int i = 0; i < ntiles; ++i) {
         const uint32_t gi = g + i, buf = gi & 1;
         const bool ok = __all_sync(0xffffffffu, mbar_wait(&S.t_full[buf], (gi >> 1) & 1, alive, A.err, A.budget));
@@ -353,17 +374,39 @@ topp_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
             }
           }
           {
-            // bracket levels: two compares per key; the keys inside are handled one by one
-            uint32_t inb = 0u, above = 0u;
+            // bracket levels: the keys inside are found by two compares each, then handled one
+            // by one.  Past the first linear level a chunk rarely holds one, so a cheap screen
+            // (the least |x - c| over the chunk, c the bracket's centre) skips the compares.
+            uint32_t inb = 0u;
             if (bracket && own) {
+              bool maybe = true;
+              if (screen) {
+                float mn = INFINITY;
 #pragma unroll
-              for (int j = 0; j < 32; ++j) {
-                const float x = __uint_as_float(v[j]);
-                inb |= (uint32_t)(x > vlo && x <= vhi) << j;
-                above |= (uint32_t)(x > vhi) << j;
+                for (int j = 0; j < 32; j += 2) {
+                  float d0, d1;
+                  sub2(__uint_as_float(v[j]), __uint_as_float(v[j + 1]), bc, d0, d1);
+                  mn = min3f(mn, fabsf(d0), fabsf(d1));
+                }
+                maybe = mn <= bhw;
               }
-              inb &= vmask;
-              if (level == kLvCollect) ngt += __popc(above & vmask);
+              if (maybe) {
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                  const float x = __uint_as_float(v[j]);
+                  inb |= (uint32_t)(x > vlo && x <= vhi) << j;
+                }
+                inb &= vmask;
+              }
+              if (level == kLvCollect) {  // keys above the bracket
+                float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+                for (int j = 0; j < 32; j += 2) {
+                  a0 += (j < nv && __uint_as_float(v[j]) > vhi) ? 1.f : 0.f;
+                  a1 += (j + 1 < nv && __uint_as_float(v[j + 1]) > vhi) ? 1.f : 0.f;
+                }
+                ngt += (int)(a0 + a1);
+              }
             }
             if (inb) {
               // each lane walks its own keys inside the bracket (about one in twelve at
