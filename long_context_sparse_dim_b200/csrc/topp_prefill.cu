@@ -53,7 +53,7 @@ namespace {
 
 constexpr int kPfRows = 128;      // query rows per CTA (TMEM lanes)
 constexpr int kPfKeys = 128;      // keys per score tile (MMA N)
-constexpr int kPfStages = 4;      // K_idx tile ring
+constexpr int kPfStages = 2;      // K_idx tile ring (a tile's epilogue takes far longer than its load)
 constexpr int kPfBins = 32;       // histogram bins per row (also the candidate capacity)
 constexpr int kPfEpiWarps = 8;    // two per TMEM lane quadrant (column halves)
 constexpr int kPfProducerWarp = kPfEpiWarps;
@@ -86,6 +86,7 @@ struct PfSmem {
   uint64_t hist[2][kPfBins][kPfRows];  // per half: bin masses, or candidates (COLLECT)
   uint8_t hcnt[2][kPfBins][kPfRows];   // per half: bin counts (saturating at 255)
   PfRowState rs[kPfRows];
+  float xs[16][kPfEpiWarps * 32];  // per epilogue thread: 16 keys of a chunk, for picking keys by column
   float pmax[kPfRows];  // half 1's partial maximum
   int pn[kPfRows];      // half 1's candidate count
   int pgt[kPfRows];     // half 1's count of keys above the bracket
@@ -408,17 +409,19 @@ topp_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
                 ngt += (int)(a0 + a1);
               }
             }
-            if (inb) {
-              // each lane walks its own keys inside the bracket (about one in twelve at
-              // the first linear level, far fewer later): the chunk goes to a small
-              // per-thread array so that a key can be picked by its column
-              float xs[32];
+            // each lane walks its own keys inside the bracket (about one in twelve at the first
+            // linear level, far fewer later): each half chunk holding one goes to the thread's
+            // column of a shared array, so that a key can be picked by its index
 #pragma unroll
-              for (int j = 0; j < 32; ++j) xs[j] = __uint_as_float(v[j]);
-              while (inb) {
-                const int j = __ffs(inb) - 1;
-                inb &= inb - 1u;
-                const float x = xs[j];
+            for (int hh = 0; hh < 2; ++hh) {
+              uint32_t hb = (inb >> (16 * hh)) & 0xFFFFu;
+              if (!hb) continue;
+#pragma unroll
+              for (int j = 0; j < 16; ++j) S.xs[j][tid] = __uint_as_float(v[16 * hh + j]);
+              while (hb) {
+                const int j = 16 * hh + __ffs(hb) - 1;
+                hb &= hb - 1u;
+                const float x = S.xs[j - 16 * hh][tid];
                 const float u = __fsub_rn(mh, x);
                 if (level == kLvLin) {
                   const int d = min(max((int)__fmul_rn(u, dscale) - 32 * prefix, 0), kPfBins - 1);
