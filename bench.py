@@ -390,6 +390,8 @@ def run_ours(args, wl, rank, world, local_rank):
     e2e = _e2e(layer, inst, wl, dev, max(args.steps, E2E_MIN_STEPS))
     dense = _dense_decode(layer, wl, dev, step_ms)
     budget = _budget_decode(layer, wl)
+    cache = _cache_maintenance(inst, wl, dev, step_ms) if wl.Hkv > wl.R and wl.N > 4096 else None
+    split = _key_range_split(dev) if wl.name == DEFAULT_WORKLOAD else None
 
     line = {
         "metric": METRIC, "value": world * wl.B / (step_ms * 1e-3), "unit": "tokens/s", "n_gpus": world,
@@ -415,6 +417,8 @@ def run_ours(args, wl, rank, world, local_rank):
         "e2e": e2e,
         "dense_comparator": dense,
         "budget": budget,
+        "cache_maintenance": cache,
+        "key_range_split": split,
         "gpu_launches": 5 * args.steps,
         "streams": "window attention (local heads) forked onto a second stream after the projections",
         "timing_events": f"around both attention launches of every {EVENT_EVERY}th timed step",
@@ -480,6 +484,155 @@ def _budget_decode(layer, wl, reps=200):
                                             "max": int(cnt.max()), "std": float(cnt.std())},
             "topk_k": k, "topp_select_ms": topp_ms, "topk_select_ms": topk_ms,
             "queries": int(cnt.size)}
+
+
+def _cache_maintenance(inst, wl, dev, resident_step_ms, reps=200):
+    """Decode over caches the path keeps itself (CachedDecodeLayer): each step
+    appends the new token (rtp_kv_append: full cache + projected key for the
+    retrieval heads, a W-row ring for the local heads) before attending.
+    Reports the cache memory against a full cache of every head, the chunk
+    append of the prompt (HBM-bound copy + projection), the one-token append,
+    and the whole appending step against the resident-cache step."""
+    import torch
+    from long_context_sparse_dim_b200 import rtp
+    from long_context_sparse_dim_b200.layer import CachedDecodeLayer
+    dt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+    es = 2 if wl.dtype == "bf16" else 4
+    B, Hkv, R, N, W, D = wl.B, wl.Hkv, wl.R, wl.N, wl.W, 128
+    L = Hkv - R
+    k = torch.from_numpy(inst.k).to(dev, dt)
+    v = torch.from_numpy(inst.v).to(dev, dt)
+    P = torch.from_numpy(inst.P).to(dev, torch.float32)
+    layer = CachedDecodeLayer(B, wl.Hq, Hkv, N, R, W, wl.p, P, dtype=dt, device=dev)
+    T0 = N - 2 * reps - 16          # the prompt; the steps below append real rows up to N
+    kc, vc = k[:, :, :T0], v[:, :, :T0]
+    zeros = torch.zeros(B, dtype=torch.int32, device=dev)
+    lens_o = torch.empty(B, dtype=torch.int32, device=dev)
+    rl = torch.empty(B, dtype=torch.int32, device=dev)
+    args = (kc, vc, zeros, R, P, layer.k_cache, layer.v_cache, layer.k_idx, layer.k_ring, layer.v_ring, lens_o, rl)
+    chunk_ms = _timed(lambda: rtp.kv_append(*args), 10)
+    chunk_bytes = (2 * B * Hkv * T0 * D * es             # read every new K and V row
+                   + 2 * B * R * T0 * D * es + B * R * T0 * 16 * es   # full caches + projected keys
+                   + 2 * B * L * min(T0, W) * D * es)    # the rings keep the last W
+    peak, peak_kind = _peaks()
+    layer.set_lengths(zeros)
+    layer.append(kc, vc)
+    q = torch.from_numpy(inst.q).to(dev, dt)
+    layer.q.copy_(q)
+    side = torch.cuda.Stream(dev)
+
+    def feed(i):
+        layer.k_new.copy_(k[:, :, T0 + i: T0 + i + 1])
+        layer.v_new.copy_(v[:, :, T0 + i: T0 + i + 1])
+
+    for i in range(4):                      # warm-up, marshals both plans
+        feed(i)
+        layer.step(side_stream=side)
+    torch.cuda.synchronize()
+    # one-token append alone (positions of the next step; idempotent rewrites)
+    one = rtp.bind_kv_append(layer.k_new, layer.v_new, layer._lens[layer._cur], R, P, layer.k_cache, layer.v_cache,
+                             layer.k_idx, layer.k_ring, layer.v_ring, lens_o, rl)
+    append_ms = _timed(one, reps)
+    # the whole appending step, graph-replayed like the resident step
+    s = torch.cuda.Stream(dev)
+    s.wait_stream(torch.cuda.current_stream(dev))
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            for _ in range(reps):           # even: the host's plan choice comes back to the start
+                layer.step(side_stream=side)
+    torch.cuda.current_stream(dev).wait_stream(s)
+    torch.cuda.synchronize()
+    g.replay()                              # appends tokens T0+4 .. T0+4+reps-1 (upload untimed)
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    g.replay()                              # the next reps tokens, all below N
+    b.record()
+    b.synchronize()
+    step_ms = a.elapsed_time(b) / reps
+    ok = bool((layer.lens == T0 + 4 + 2 * reps).all().item())
+    full_bytes = 2 * B * Hkv * N * D * es + B * R * N * 16 * es
+    del g
+    return {"layer": "CachedDecodeLayer (rtp_kv_append + the decode calls)",
+            "cache_bytes": layer.cache_bytes(), "full_cache_bytes": full_bytes,
+            "cache_fraction": layer.cache_bytes() / full_bytes,
+            "prompt_append": {"tokens": T0, "ms": chunk_ms, "algorithmic_bytes": chunk_bytes,
+                              "achieved_gbs": chunk_bytes / (chunk_ms * 1e-3) / 1e9,
+                              "frac": chunk_bytes / (chunk_ms * 1e-3) / 1e9 / peak, "peak_kind": peak_kind},
+            "one_token_append_ms": append_ms,
+            "step_ms": step_ms, "resident_step_ms": resident_step_ms,
+            "tokens_per_s": B / (step_ms * 1e-3), "lengths_advanced": ok}
+
+
+def _key_range_split(dev, N=1 << 20, worlds=(1, 2, 4, 8), reps=50):
+    """One sequence of 2^20 keys (the layer shape of the decode workloads, W =
+    8192) decoded with its keys split by position over S ranks
+    (KeyRangeDecodeLayer), each rank's share of a step emulated on this one GPU:
+    the replicated query projection + top-p selection over all N keys, the
+    range attention over N / S rows, its block of local heads and the merge of
+    S partials.  The all-gather between the ranks (one row of 129 floats per
+    query head and rank) is not part of the emulation.  Inputs are random
+    device tensors; S = 1 is the unsplit step."""
+    import math
+    import torch
+    from long_context_sparse_dim_b200 import rtp
+    from long_context_sparse_dim_b200.split import key_ranges
+    B, Hq, Hkv, R, W, D, p = 1, 32, 8, 2, 8192, 128, 0.95
+    G, L = Hq // Hkv, Hkv - R
+    Hr = R * G
+    g = torch.Generator(device=dev).manual_seed(5)
+    k = torch.randn(B, R, N, D, generator=g, device=dev).to(torch.bfloat16)
+    v = torch.randn(B, R, N, D, generator=g, device=dev).to(torch.bfloat16)
+    q = torch.randn(B, Hq, 1, D, generator=g, device=dev).to(torch.bfloat16)
+    kw = torch.randn(B, L, W, D, generator=g, device=dev).to(torch.bfloat16)
+    vw = torch.randn(B, L, W, D, generator=g, device=dev).to(torch.bfloat16)
+    P = torch.from_numpy(np.ascontiguousarray(np.broadcast_to(wls.lowfreq_projection(), (R, 16, D)))).to(dev)
+    lens = torch.full((B,), N, dtype=torch.int32, device=dev)
+    wl_ = torch.full((B,), W, dtype=torch.int32, device=dev)
+    k_idx = torch.zeros(B, R, N, 16, dtype=torch.bfloat16, device=dev)
+    rtp.index_project(k, P, k_idx)
+    q_idx = torch.zeros(B, Hr, 1, 16, dtype=torch.bfloat16, device=dev)
+    sel = rtp.Selection.empty(B * Hr, N, dev)
+    scale = 1 / math.sqrt(D)
+
+    def select():
+        rtp.index_project(q[:, :Hr], P, q_idx)
+        rtp.topp_select(q_idx, k_idx, lens, p, sel)
+
+    sel_ms = _timed(select, reps)
+    out = {"N": N, "B": B, "W": W, "p": p, "selection_ms": sel_ms,
+           "selected_fraction": float(sel.count.float().mean().item()) / N, "ranks": {}}
+    for S in worlds:
+        lo, rows = key_ranges(N, S)[0]
+        l0, l1 = 0, -(-L // S)          # the busiest rank's block of local heads (ceil(L / S) of them)
+        o = torch.zeros(B, Hq, 1, D, device=dev)
+        lse = torch.zeros(B, Hq, device=dev)
+        ws = rtp.workspace(rtp.sparse_attn_decode_workspace_size(B, Hr, R, rows), dev)
+        kr, vr = k[:, :, lo:lo + rows], v[:, :, lo:lo + rows]
+        wsw = rtp.workspace(rtp.window_attn_workspace_size(B, (l1 - l0) * G, 1, l1 - l0, W, W), dev)
+        parts = torch.zeros(S, B, Hq, D, device=dev)
+        lses = torch.zeros(S, B, Hq, device=dev)
+        o_final = torch.zeros(B, Hq, 1, D, device=dev)
+
+        def share():
+            rtp.sparse_attn_decode_range(q[:, :Hr], kr, vr, lens, sel, lo, scale, o[:, :Hr], lse[:, :Hr], ws)
+            if l1 > l0:
+                rtp.window_attn(q[:, Hr + l0 * G: Hr + l1 * G], kw[:, l0:l1], vw[:, l0:l1], wl_, W, scale,
+                                o[:, Hr + l0 * G: Hr + l1 * G], wsw)
+            rtp.attn_combine(parts, lses, o_final)
+
+        share_ms = _timed(share, reps)
+        step_ms = sel_ms + share_ms
+        out["ranks"][str(S)] = {"rows_per_rank": rows, "local_kv_heads_per_rank": l1 - l0,
+                                "rank_step_ms": step_ms, "range_and_merge_ms": share_ms,
+                                "tokens_per_s_projected": B / (step_ms * 1e-3)}
+    out["note"] = ("per-rank shares emulated one at a time on one GPU; the all-gather of the partial rows "
+                   "(129 floats per query head and rank) is not included: unmeasured on more than one GPU")
+    del k, v, k_idx, kw, vw
+    torch.cuda.empty_cache()
+    return out
 
 
 def _step_with_events(layer, ev, side):

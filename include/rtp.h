@@ -148,6 +148,43 @@ RTP_API rtp_status rtp_topk_select(const rtp_tensor* q_idx, const rtp_tensor* k_
                                    int32_t k, const rtp_selection* out, void* workspace, size_t workspace_bytes,
                                    rtp_stream_t stream);
 
+/* ---- cache maintenance: appending new tokens --------------------------------
+ *   k_new, v_new [B, H, T, 128]  bf16 or f32, post-rotary keys / values of the
+ *                T new tokens of each sequence (all H KV heads)
+ *   pos          int32[B] device: position of new token 0 in sequence b
+ *   R            the first R KV heads are retrieval heads (0 <= R <= H)
+ *   P            [R, 16, 128] f32 (unused, may be NULL, when R == 0)
+ *   k_cache, v_cache [B, R, N, 128]  full caches of the retrieval heads:
+ *                row pos+t receives token t (tokens outside [0, N) are dropped)
+ *   k_idx        [B, R, N, 16]  projected keys: row pos+t receives P k_t,
+ *                bit-identical to rtp_index_project of that row
+ *   k_ring, v_ring [B, H - R, W, 128]  local heads' rings of W rows: token at
+ *                position p goes to row p mod W (of the T tokens only the last
+ *                W are written)
+ *   lens_out     int32[B] device or NULL (not the pos buffer): receives pos + T,
+ *                clamped to [0, N] when R > 0, i.e. the sequence length after the
+ *                append and the `pos` of the next one
+ *   ring_lens    int32[B] device or NULL (must be NULL when R == H): receives
+ *                min(pos + T, W), the number of ring rows in use, i.e. the
+ *                `lens` of rtp_window_attn over the ring with window W (after
+ *                in-order appends the ring holds exactly the keys of the newest
+ *                token's window, in slot order; attention does not depend on
+ *                the order of its keys)
+ * Caches, rings and P are NULL-able only for the head group that is empty.  All
+ * tensors share the dtype of k_new (P is f32).  pos[b] + T must fit in int32.
+ * pos, lens_out and ring_lens are three distinct buffers.  One launch, one pass
+ * over the new rows.
+ * Errors: INVALID_ARG (NULL pos, R outside [0, H], aliased length buffers),
+ * SHAPE / DTYPE / ALIGNMENT as for the other calls; nothing is written then.
+ * Cites: "RTPurbo: Turning Dense LLMs ...", "Three Key Insights" 1 (retrieval
+ * heads keep the full cache, local heads a local window); "Full Attention
+ * Strikes Back ... (RTPurbo)", TL;DR (a lightweight token indexer).
+ */
+RTP_API rtp_status rtp_kv_append(const rtp_tensor* k_new, const rtp_tensor* v_new, const int32_t* pos, int32_t R,
+                                 const rtp_tensor* P, const rtp_tensor* k_cache, const rtp_tensor* v_cache,
+                                 const rtp_tensor* k_idx, const rtp_tensor* k_ring, const rtp_tensor* v_ring,
+                                 int32_t* lens_out, int32_t* ring_lens, rtp_stream_t stream);
+
 /* ---- a4 (decode): exact attention over each query's selected keys -------
  *   q      [B, Hq, 1, 128]  bf16 or f32 (retrieval query heads)
  *   k, v   [B, Hk, N, 128]  same dtype (full KV cache of the retrieval heads)
@@ -166,6 +203,45 @@ RTP_API rtp_status rtp_sparse_attn_decode(const rtp_tensor* q, const rtp_tensor*
                                   const rtp_tensor* o, void* workspace, size_t workspace_bytes,
                                   rtp_stream_t stream);
 RTP_API size_t rtp_sparse_attn_decode_workspace_size(int64_t B, int64_t Hq, int64_t Hk, int64_t N);
+
+/* ---- a4 (decode) over one key range of longer sequences ------------------
+ * For a sequence whose keys are split by position across devices (each holds
+ * the K/V rows of one contiguous range and the full selection): attention of
+ * each query over its selected keys inside this range, plus the log-sum-exp
+ * that rtp_attn_combine needs to merge the ranges.
+ *   q, sel, scale  as for rtp_sparse_attn_decode (sel covers the whole
+ *          sequence: mask_words * 32 >= key_lo + N)
+ *   k, v   [B, Hk, N, 128]  rows 0 .. N-1 hold keys key_lo .. key_lo + N - 1
+ *   lens   int32[B] device or NULL: whole-sequence lengths (keys at or past
+ *          lens[b] are not attended); NULL means key_lo + N
+ *   key_lo global position of row 0; a multiple of 64, >= 0
+ *   o      [B, Hq, 1, 128] f32 or bf16: attention over the range's selected
+ *          keys, normalised within the range (0 when it has none)
+ *   lse    [B, Hq] f32 (last dim contiguous): ln sum_j exp(scale * q.k_j) over
+ *          those keys (-inf when none)
+ * Workspace: rtp_sparse_attn_decode_workspace_size(B, Hq, Hk, N).  Errors as
+ * rtp_sparse_attn_decode, plus INVALID_ARG for a bad key_lo or a NULL lse.
+ * Cites: "Full Attention Strikes Back ... (RTPurbo)", TL;DR (retrieval heads
+ * attend the indexed tokens of the full cache); softmax over a union of
+ * disjoint key sets is the lse-weighted mean of the per-set results.
+ */
+RTP_API rtp_status rtp_sparse_attn_decode_range(const rtp_tensor* q, const rtp_tensor* k, const rtp_tensor* v,
+                                                const int32_t* lens, const rtp_selection* sel, int64_t key_lo,
+                                                float scale, const rtp_tensor* o, const rtp_tensor* lse,
+                                                void* workspace, size_t workspace_bytes, rtp_stream_t stream);
+
+/* ---- merge of key-range partials ---------------------------------------------
+ *   o_parts   [S, B, Hq, 128] f32: S partial outputs (rtp_sparse_attn_decode_range
+ *             or any attention normalised over its own key set)
+ *   lse_parts [S, B, Hq] f32 (last dim contiguous): their log-sum-exps
+ *   o         [B, Hq, 1, 128] f32 or bf16
+ * o = sum_s exp(lse_s - M) o_s / sum_s exp(lse_s - M), M = max_s lse_s; rows
+ * whose partials are all empty (lse = -inf) get 0.  A partial with lse = 0
+ * and every other -inf passes through unchanged (used for heads that one
+ * device computes alone).  One launch, one warp per row.
+ */
+RTP_API rtp_status rtp_attn_combine(const rtp_tensor* o_parts, const rtp_tensor* lse_parts, const rtp_tensor* o,
+                                    rtp_stream_t stream);
 
 /* ---- a4 (decode) without a caller workspace ------------------------------
  * The pages have no counterpart to this call: it is a library-level variant

@@ -1,6 +1,6 @@
 """Build librtp.so (sm_100a) in-tree with nvcc.
 
-    python -m long_context_sparse_dim_b200.build [-v] [--debug]
+    python -m long_context_sparse_dim_b200.build [-v]
 
 Each ``csrc/*.cu`` compiles to an object under ``_build/`` (skipped when the
 object is newer than its sources), then all objects link into
@@ -60,11 +60,9 @@ def _compile(src: str, extra, verbose: bool) -> str:
     return obj
 
 
-def build(verbose: bool = False, debug: bool = False, ptxas_info: bool = False) -> str:
+def build(verbose: bool = False, ptxas_info: bool = False) -> str:
     os.makedirs(BUILD, exist_ok=True)
     extra = []
-    if debug:
-        extra += ["-DRTP_DEBUG_BOUNDS=1"]
     if ptxas_info:
         extra += ["-Xptxas", "-v"]
     srcs = _sources()
@@ -84,10 +82,9 @@ def build(verbose: bool = False, debug: bool = False, ptxas_info: bool = False) 
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("-v", "--verbose", action="store_true")
-    ap.add_argument("--debug", action="store_true")
     ap.add_argument("--ptxas-info", action="store_true")
     a = ap.parse_args(argv)
-    print(build(a.verbose, a.debug, a.ptxas_info))
+    print(build(a.verbose, a.ptxas_info))
 
 
 if __name__ == "__main__":

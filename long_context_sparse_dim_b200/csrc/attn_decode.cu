@@ -56,6 +56,9 @@ struct AttnArgs {
   float scale_log2;
   MutView4 o;
   int o_bf16;
+  int key_lo;     // global position of key row 0 (a key range of a longer sequence)
+  float* lse;     // [B, Hq] (row stride lse_sb) or null: natural-log sum of exp(scaled scores)
+  int64_t lse_sb; //   over the keys attended
   float* ws_o;    // [groups][splits][kMaxGroup][128]
   float* ws_ml;   // [groups][splits][kMaxGroup][2]
   uint32_t* tickets;  // [groups]
@@ -109,8 +112,8 @@ struct KeyRange {
 };
 
 RTP_DEVICE KeyRange key_range(const AttnArgs& A, int b, int split) {
-  int n_b = A.N;
-  if (A.lens) n_b = min(max(A.lens[b], 0), A.N);
+  int n_b = A.N;  // rows of this call's K/V: keys key_lo .. key_lo + n_b - 1 of the sequence
+  if (A.lens) n_b = min(max(A.lens[b] - A.key_lo, 0), A.N);
   KeyRange r;
   r.hi = n_b;
   r.lo = A.W > 0 ? max(0, n_b - A.W) : 0;
@@ -123,7 +126,7 @@ RTP_DEVICE KeyRange key_range(const AttnArgs& A, int b, int split) {
 // ---- split partial write + last-CTA merge (shared by both variants) --------
 // part_o[h][d] (unnormalised), part_m[h] (log2 domain), part_l[h] are in smem;
 // `scratch` holds at least 2 * kMaxSplits * kMaxGroup + 2 * kMaxGroup floats.
-constexpr int kMaxSplits = 64;
+constexpr int kMaxSplits = 256;  // >= one split per SM for a single (sequence, KV head) group
 
 __device__ void finish_split(const AttnArgs& A, int grp, int split, const float* part_o,
                              const float* part_m, const float* part_l, int* flag_smem, float* scratch) {
@@ -193,6 +196,8 @@ __device__ void finish_split(const AttnArgs& A, int grp, int split, const float*
     const float den = Lh[h];
     const float val = den > 0.f ? num / den : 0.f;
     const int hq = kvh * G + h;
+    if (A.lse && d == 0)  // scores are kept in the log2 domain: ln sum = (M + log2 L) ln 2
+      A.lse[b * A.lse_sb + hq] = den > 0.f ? (Mh[h] + log2f(den)) * 0.69314718055994531f : -INFINITY;
     if (A.o_bf16) {
       __nv_bfloat16* op = static_cast<__nv_bfloat16*>(A.o.data) + b * A.o.sb + hq * A.o.sh;
       op[d] = __float2bfloat16_rn(val);
@@ -222,7 +227,8 @@ attn_decode_bf16_kernel(AttnArgs A) {
 
   const __nv_bfloat16* kbase = static_cast<const __nv_bfloat16*>(A.k.data) + b * A.k.sb + kvh * A.k.sh;
   const __nv_bfloat16* vbase = static_cast<const __nv_bfloat16*>(A.v.data) + b * A.v.sb + kvh * A.v.sh;
-  const uint32_t* mrow0 = sparse ? A.mask + (int64_t)(b * A.Hq + kvh * G) * A.mask_words : nullptr;
+  const uint32_t* mrow0 =
+      sparse ? A.mask + (int64_t)(b * A.Hq + kvh * G) * A.mask_words + (A.key_lo >> 5) : nullptr;
 
   // Q^T as the B operand: column n = head g (zero for g >= G), rows = dims.
   uint32_t qb[8][2];
@@ -460,7 +466,8 @@ attn_decode_f32_kernel(AttnArgs A) {
   const bool sparse = A.W <= 0;
   const float* kbase = static_cast<const float*>(A.k.data) + b * A.k.sb + kvh * A.k.sh;
   const float* vbase = static_cast<const float*>(A.v.data) + b * A.v.sb + kvh * A.v.sh;
-  const uint32_t* mrow0 = sparse ? A.mask + (int64_t)(b * A.Hq + kvh * G) * A.mask_words : nullptr;
+  const uint32_t* mrow0 =
+      sparse ? A.mask + (int64_t)(b * A.Hq + kvh * G) * A.mask_words + (A.key_lo >> 5) : nullptr;
 
   float4 qv[kMaxGroup];
   float m[kMaxGroup], l[kMaxGroup];
@@ -611,6 +618,9 @@ cudaError_t launch_attn_decode(const LaunchAttnDecode& a, cudaStream_t stream) {
   A.scale_log2 = a.scale * kLog2e;
   A.o = a.o;
   A.o_bf16 = a.o_bf16 ? 1 : 0;
+  A.key_lo = (int)a.key_lo;
+  A.lse = a.lse;
+  A.lse_sb = a.lse_sb;
   const size_t o_bytes = (size_t)groups * splits * kMaxGroup * kHeadDim * sizeof(float);
   const size_t ml_bytes = (size_t)groups * splits * kMaxGroup * 2 * sizeof(float);
   char* ws = static_cast<char*>(a.ws);

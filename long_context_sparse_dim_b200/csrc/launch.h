@@ -130,6 +130,9 @@ struct LaunchAttnDecode {
   MutView4 o;            // [B, Hq, 1, 128]
   bool o_bf16;
   void* ws;
+  int64_t key_lo = 0;    // sparse mode: global position of key row 0 (multiple of 64)
+  float* lse = nullptr;  // [B, Hq] (row stride lse_sb) or null: log-sum-exp of the attended scaled scores
+  int64_t lse_sb = 0;
 };
 bool attn_decode_supported(int64_t B, int64_t Hk, int64_t N, int32_t W);
 size_t attn_decode_workspace_bytes(int64_t B, int64_t Hq, int64_t Hk, int64_t N, int32_t W);
@@ -147,6 +150,33 @@ void attn_decode_ticket_range(int64_t B, int64_t Hk, int64_t N, int32_t W, size_
 // 64 columns, 128-byte swizzle).
 bool make_idx_map(CUtensorMap* map, const View4& v, int64_t B, int64_t H, int64_t R, int box_rows);
 bool make_row_map(CUtensorMap* map, const View4& v, int64_t B, int64_t H, int64_t R, int box_rows);
+
+// Merge of key-range attention partials (rtp_attn_combine).
+struct AttnCombineArgs {
+  const float* o_parts;      // [S, B, Hq, 128] f32, strides ps, pb, ph (elements)
+  int64_t ps, pb, ph;
+  const float* lse;          // [S, B, Hq] f32, strides ls, lb, 1
+  int64_t ls, lb;
+  int S, B, Hq;
+  MutView4 o;                // [B, Hq, 1, 128]
+  int o_bf16;
+};
+cudaError_t launch_attn_combine(const AttnCombineArgs& a, cudaStream_t stream);
+
+// Cache append (rtp_kv_append): the first R KV heads go to the full caches
+// (and the projected-key cache), the others to W-row rings.
+struct KvAppendArgs {
+  View4 k_new, v_new;        // [B, H, T, 128]
+  const int32_t* pos;        // [B] device: position of token 0
+  const float* P;            // [R, 16, 128]
+  MutView4 k_cache, v_cache; // [B, R, N, 128]
+  MutView4 k_idx;            // [B, R, N, 16]
+  MutView4 k_ring, v_ring;   // [B, H - R, W, 128]
+  int32_t* lens_out;         // [B] or null: pos + T (clamped to [0, N] when R > 0)
+  int32_t* ring_lens;        // [B] or null: min(pos + T, W)
+  int B, H, T, R, N, W;
+};
+cudaError_t launch_kv_append(const KvAppendArgs& a, bool bf16, cudaStream_t stream);
 
 // Records a CUDA error for rtp_last_cuda_error() on this thread.
 void set_last_cuda_error(int32_t e);

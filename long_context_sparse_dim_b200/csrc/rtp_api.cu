@@ -38,6 +38,18 @@ rtp_status check4(const rtp_tensor* t, int64_t last) {
   return RTP_OK;
 }
 
+// An f32 tensor of `nd` dims with a contiguous last dim (log-sum-exp rows).
+rtp_status check_f32_rows(const rtp_tensor* t, int32_t nd) {
+  if (!t || !t->data) return RTP_ERR_INVALID_ARG;
+  if (t->ndim != nd) return RTP_ERR_SHAPE;
+  if (t->dtype != RTP_F32) return RTP_ERR_DTYPE;
+  for (int i = 0; i < nd; ++i)
+    if (t->shape[i] < 0 || t->stride[i] < 0) return RTP_ERR_SHAPE;
+  if (t->shape[nd - 1] > 1 && t->stride[nd - 1] != 1) return RTP_ERR_ALIGNMENT;
+  if (((uintptr_t)t->data) % 4) return RTP_ERR_ALIGNMENT;
+  return RTP_OK;
+}
+
 rtp::View4 view(const rtp_tensor* t) { return rtp::View4{t->data, t->stride[0], t->stride[1], t->stride[2]}; }
 rtp::MutView4 mview(const rtp_tensor* t) {
   return rtp::MutView4{t->data, t->stride[0], t->stride[1], t->stride[2]};
@@ -222,6 +234,62 @@ rtp_status rtp_topk_select(const rtp_tensor* q_idx, const rtp_tensor* k_idx, con
   return cuda_status(rtp::launch_topp_decode(a, (cudaStream_t)stream));
 }
 
+// ---- cache maintenance ---------------------------------------------------------------
+rtp_status rtp_kv_append(const rtp_tensor* k_new, const rtp_tensor* v_new, const int32_t* pos, int32_t R,
+                         const rtp_tensor* P, const rtp_tensor* k_cache, const rtp_tensor* v_cache,
+                         const rtp_tensor* k_idx, const rtp_tensor* k_ring, const rtp_tensor* v_ring,
+                         int32_t* lens_out, int32_t* ring_lens, rtp_stream_t stream) {
+  rtp_status s;
+  if ((s = check_kv(k_new, v_new)) != RTP_OK) return s;
+  if (!pos) return RTP_ERR_INVALID_ARG;
+  if ((void*)lens_out == (const void*)pos || (void*)ring_lens == (const void*)pos) return RTP_ERR_INVALID_ARG;
+  if (lens_out && lens_out == ring_lens) return RTP_ERR_INVALID_ARG;
+  const int64_t B = k_new->shape[0], H = k_new->shape[1], T = k_new->shape[2];
+  if (R < 0 || R > H) return RTP_ERR_INVALID_ARG;
+  if (R == H && ring_lens) return RTP_ERR_INVALID_ARG;  // no local heads, no ring
+  if (B > INT32_MAX || H > INT32_MAX || T > INT32_MAX) return RTP_ERR_SHAPE;
+  int64_t N = 0, W = 1;
+  if (R > 0) {
+    if ((s = check_kv(k_cache, v_cache)) != RTP_OK) return s;
+    if ((s = check4(k_idx, 16)) != RTP_OK) return s;
+    if (!P || !P->data) return RTP_ERR_INVALID_ARG;
+    if (P->dtype != RTP_F32) return RTP_ERR_DTYPE;
+    if (P->ndim != 3 || P->shape[0] != R || P->shape[1] != 16 || P->shape[2] != 128) return RTP_ERR_SHAPE;
+    if (P->stride[2] != 1 || P->stride[1] != 128 || P->stride[0] != 16 * 128) return RTP_ERR_ALIGNMENT;
+    if (((uintptr_t)P->data) % 16) return RTP_ERR_ALIGNMENT;
+    if (k_cache->shape[0] != B || k_cache->shape[1] != R) return RTP_ERR_SHAPE;
+    if (k_idx->shape[0] != B || k_idx->shape[1] != R || k_idx->shape[2] != k_cache->shape[2]) return RTP_ERR_SHAPE;
+    if (k_cache->dtype != k_new->dtype || k_idx->dtype != k_new->dtype) return RTP_ERR_DTYPE;
+    N = k_cache->shape[2];
+  }
+  if (R < H) {
+    if ((s = check_kv(k_ring, v_ring)) != RTP_OK) return s;
+    if (k_ring->shape[0] != B || k_ring->shape[1] != H - R || k_ring->shape[2] < 1) return RTP_ERR_SHAPE;
+    if (k_ring->dtype != k_new->dtype) return RTP_ERR_DTYPE;
+    if (k_ring->shape[2] > INT32_MAX) return RTP_ERR_SHAPE;
+    W = k_ring->shape[2];
+  }
+  rtp::KvAppendArgs a;
+  a.k_new = view(k_new);
+  a.v_new = view(v_new);
+  a.pos = pos;
+  a.P = R > 0 ? static_cast<const float*>(P->data) : nullptr;
+  a.k_cache = R > 0 ? mview(k_cache) : rtp::MutView4{nullptr, 0, 0, 0};
+  a.v_cache = R > 0 ? mview(v_cache) : rtp::MutView4{nullptr, 0, 0, 0};
+  a.k_idx = R > 0 ? mview(k_idx) : rtp::MutView4{nullptr, 0, 0, 0};
+  a.k_ring = R < H ? mview(k_ring) : rtp::MutView4{nullptr, 0, 0, 0};
+  a.v_ring = R < H ? mview(v_ring) : rtp::MutView4{nullptr, 0, 0, 0};
+  a.lens_out = lens_out;
+  a.ring_lens = ring_lens;
+  a.B = (int)B;
+  a.H = (int)H;
+  a.T = (int)T;
+  a.R = R;
+  a.N = (int)N;
+  a.W = (int)W;
+  return cuda_status(rtp::launch_kv_append(a, k_new->dtype == RTP_BF16, (cudaStream_t)stream));
+}
+
 // ---- a4 decode -------------------------------------------------------------------
 size_t rtp_sparse_attn_decode_workspace_size(int64_t B, int64_t Hq, int64_t Hk, int64_t N) {
   return rtp::attn_decode_workspace_bytes(B, Hq, Hk, N, 0);
@@ -289,6 +357,55 @@ rtp_status rtp_sparse_attn_decode(const rtp_tensor* q, const rtp_tensor* k, cons
   if ((s = check_workspace(workspace, workspace_bytes, need)) != RTP_OK) return s;
   a.ws = workspace;
   return cuda_status(rtp::launch_attn_decode(a, (cudaStream_t)stream));
+}
+
+rtp_status rtp_sparse_attn_decode_range(const rtp_tensor* q, const rtp_tensor* k, const rtp_tensor* v,
+                                        const int32_t* lens, const rtp_selection* sel, int64_t key_lo,
+                                        float scale, const rtp_tensor* o, const rtp_tensor* lse,
+                                        void* workspace, size_t workspace_bytes, rtp_stream_t stream) {
+  rtp::LaunchAttnDecode a;
+  rtp_status s;
+  if (key_lo < 0 || key_lo % 64) return RTP_ERR_INVALID_ARG;
+  if ((s = check_f32_rows(lse, 2)) != RTP_OK) return s;
+  if ((s = rtp::check_sparse_attn_decode(q, k, v, lens, sel, scale, o, &a)) != RTP_OK) return s;
+  if (lse->shape[0] != a.B || lse->shape[1] != a.Hq) return RTP_ERR_SHAPE;
+  if (key_lo + a.N > INT32_MAX) return RTP_ERR_SHAPE;
+  if (sel->mask_words < (key_lo + a.N + 31) / 32) return RTP_ERR_SHAPE;  // masks cover the whole sequence
+  const size_t need = rtp_sparse_attn_decode_workspace_size(a.B, a.Hq, a.Hk, a.N);
+  if ((s = check_workspace(workspace, workspace_bytes, need)) != RTP_OK) return s;
+  a.ws = workspace;
+  a.key_lo = key_lo;
+  a.lse = static_cast<float*>(lse->data);
+  a.lse_sb = lse->stride[0];
+  return cuda_status(rtp::launch_attn_decode(a, (cudaStream_t)stream));
+}
+
+rtp_status rtp_attn_combine(const rtp_tensor* o_parts, const rtp_tensor* lse_parts, const rtp_tensor* o,
+                            rtp_stream_t stream) {
+  rtp_status s;
+  if ((s = check4(o_parts, 128)) != RTP_OK) return s;
+  if ((s = check4(o, 128)) != RTP_OK) return s;
+  if ((s = check_f32_rows(lse_parts, 3)) != RTP_OK) return s;
+  if (o_parts->dtype != RTP_F32) return RTP_ERR_DTYPE;
+  if (o_parts->shape[0] < 1 || o_parts->shape[0] > INT32_MAX || o_parts->shape[1] != o->shape[0] ||
+      o_parts->shape[2] != o->shape[1] || o->shape[2] != 1)
+    return RTP_ERR_SHAPE;
+  for (int i = 0; i < 3; ++i)
+    if (lse_parts->shape[i] != o_parts->shape[i]) return RTP_ERR_SHAPE;
+  rtp::AttnCombineArgs a;
+  a.o_parts = static_cast<const float*>(o_parts->data);
+  a.ps = o_parts->stride[0];
+  a.pb = o_parts->stride[1];
+  a.ph = o_parts->stride[2];
+  a.lse = static_cast<const float*>(lse_parts->data);
+  a.ls = lse_parts->stride[0];
+  a.lb = lse_parts->stride[1];
+  a.S = (int)o_parts->shape[0];
+  a.B = (int)o->shape[0];
+  a.Hq = (int)o->shape[1];
+  a.o = mview(o);
+  a.o_bf16 = o->dtype == RTP_BF16;
+  return cuda_status(rtp::launch_attn_combine(a, (cudaStream_t)stream));
 }
 
 // ---- a4 prefill --------------------------------------------------------------------

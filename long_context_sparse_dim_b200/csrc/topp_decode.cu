@@ -31,6 +31,11 @@
 // Every mass is a 64-bit fixed-point integer sum, so the result does not depend
 // on thread order.  No spin waits: all synchronisation is the hardware cluster
 // barrier.
+// Caches longer than 16 CTAs x 32768 keys (up to 4x that) give each CTA more
+// keys than its shared memory holds: the first 32768 scores stay on chip and
+// the rest are recomputed from the projected keys (L2-resident after the first
+// pass) by every pass that reads them -- the same function of the same bits,
+// so the cut is the one the stored scores would give.
 #include <cooperative_groups.h>
 
 #include <math.h>
@@ -49,6 +54,7 @@ constexpr int kFinePerBin = 16;
 constexpr int kFineBins = kBins * kFinePerBin;
 constexpr int kMaxCluster = 16;
 constexpr int kMaxKeysPerCta = 32768;       // scores of one CTA held in shared memory (128 KB)
+constexpr int kMaxStream = 4;               // keys per CTA at most kMaxStream x the resident ones
 constexpr float kCoarsePerNat = 16.f;       // coarse bin width 1/16 nat
 constexpr float kFinePerNat = 256.f;        // fine bin width 1/256 nat
 constexpr float kSubPerNat = 65536.f;       // rank 0's sub-bin width 1/65536 nat
@@ -392,6 +398,14 @@ topp_query_kernel(View4 qv, View4 kv, const int32_t* __restrict__ lens, int Hq, 
   load_idx_row<T>(static_cast<const T*>(qv.data) + b * qv.sb + h * qv.sh, qf);
   const T* kb = static_cast<const T*>(kv.data) + b * kv.sb + kvh * kv.sh;
   float lmax = -INFINITY;
+  const int n_res = min(n_chunk, kMaxKeysPerCta);  // keys whose scores stay in shared memory
+  // score of local key i: stored, or recomputed (identical bits) past the resident ones
+  auto score_of = [&](int i) -> float {
+    if (i < n_res) return scores[i];
+    float kf[kIdxDim];
+    load_idx_row<T>(kb + (int64_t)(c0 + i) * kv.sn, kf);
+    return indexer_dot16(qf, kf);
+  };
   constexpr int U = sizeof(T) == 2 ? 4 : 2;
   for (int base = 0; base < nloc; base += U * kSelThreads) {
     IdxRaw<T> raw[U];
@@ -407,7 +421,7 @@ topp_query_kernel(View4 qv, View4 kv, const int32_t* __restrict__ lens, int Hq, 
         float kf[kIdxDim];
         idx_raw_to_float<T>(raw[u], kf);
         const float sc = indexer_dot16(qf, kf);
-        scores[i] = sc;
+        if (i < n_res) scores[i] = sc;
         lmax = fmaxf(lmax, sc);
       }
     }
@@ -432,7 +446,7 @@ topp_query_kernel(View4 qv, View4 kv, const int32_t* __restrict__ lens, int Hq, 
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int i = base + u * kSelThreads + tid;
-      sc[u] = i < nloc ? scores[i] : 0.f;
+      sc[u] = i < nloc ? score_of(i) : 0.f;
     }
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
@@ -494,7 +508,7 @@ topp_query_kernel(View4 qv, View4 kv, const int32_t* __restrict__ lens, int Hq, 
         for (int u = 0; u < 4; ++u) {
           const int i = base + u * kSelThreads + tid;
           const bool valid = i < nloc;
-          const float sc = valid ? scores[i] : 0.f;
+          const float sc = valid ? score_of(i) : 0.f;
           const int f = valid ? fine_bin(sc, m) : kFineBins;
           const uint32_t word = __ballot_sync(0xffffffffu, f < fb);
           const int wpos = base + u * kSelThreads + warp * 32;
@@ -559,7 +573,7 @@ topp_query_kernel(View4 qv, View4 kv, const int32_t* __restrict__ lens, int Hq, 
     }
     __syncwarp();
     for (int i = tid; i < nloc; i += kSelThreads) {
-      const float sc = scores[i];
+      const float sc = score_of(i);
       if (coarse_bin(sc, m) == lin) {
         const uint32_t k = score_key(sc);
         if (k >= kbase && (uint64_t)k < kend) {
@@ -590,7 +604,7 @@ topp_query_kernel(View4 qv, View4 kv, const int32_t* __restrict__ lens, int Hq, 
   const float tau = key_score(tau_key);
   uint32_t ngt = 0, neq = 0;
   for (int i = tid; i < nloc; i += kSelThreads) {
-    const uint32_t k = score_key(scores[i]);
+    const uint32_t k = score_key(score_of(i));
     ngt += k > tau_key;
     neq += k == tau_key;
   }
@@ -635,7 +649,7 @@ topp_query_kernel(View4 qv, View4 kv, const int32_t* __restrict__ lens, int Hq, 
   for (int base = 0; base < n_chunk; base += kSelThreads) {
     const int i = base + tid;
     const bool valid = i < nloc;
-    const uint32_t k = valid ? score_key(scores[i]) : 0u;
+    const uint32_t k = valid ? score_key(score_of(i)) : 0u;
     const bool gt = valid && k > tau_key;
     bool sel = gt;
     if (my_ties) {
@@ -667,7 +681,7 @@ topp_query_kernel(View4 qv, View4 kv, const int32_t* __restrict__ lens, int Hq, 
   }
 }
 
-bool topp_decode_supported(int64_t N) { return N <= (int64_t)kMaxKeysPerCta * kMaxCluster; }
+bool topp_decode_supported(int64_t N) { return N <= (int64_t)kMaxKeysPerCta * kMaxCluster * kMaxStream; }
 
 static int sm_count() {
   int dev = 0, sms = 148;
@@ -700,8 +714,8 @@ cudaError_t launch_topp_decode(const LaunchToppDecode& a, cudaStream_t stream) {
   int64_t n_chunk = (a.N + C - 1) / C;
   n_chunk = (n_chunk + 31) / 32 * 32;
   if (n_chunk == 0) n_chunk = 32;
-  if (n_chunk > kMaxKeysPerCta) return cudaErrorInvalidValue;
-  const size_t smem = sizeof(SelSmem) + (size_t)n_chunk * sizeof(float);
+  if (n_chunk > (int64_t)kMaxKeysPerCta * kMaxStream) return cudaErrorInvalidValue;
+  const size_t smem = sizeof(SelSmem) + (size_t)(n_chunk < kMaxKeysPerCta ? n_chunk : kMaxKeysPerCta) * sizeof(float);
   if (a.bf16)
     return launch_cluster(topp_query_kernel<__nv_bfloat16>, (int)(Q * C), C, smem, stream, a.q_idx, a.k_idx, a.lens,
                           (int)a.Hq, G, (int)a.N, (int)n_chunk, a.p, (int)a.topk, two_pow_frac, a.tau_bits, a.tiepos,

@@ -10,7 +10,9 @@ selection, outputs, workspaces) and issues the calls of one decode step:
 
 The first R KV heads are the retrieval heads ("RTPurbo: Turning Dense LLMs
 into Sparse Attention Models ...", "Three Key Insights" 1); every step of the
-computation runs in librtp.so.
+computation runs in librtp.so.  ``DecodeLayer`` works on a resident cache of
+all heads, ``CachedDecodeLayer`` keeps its own caches (full for the retrieval
+heads, a W-row ring for the local heads) and appends each step's new token.
 """
 from __future__ import annotations
 
@@ -168,4 +170,133 @@ class PrefillLayer:
                             self.ws_loc, stream)
         if side_stream is not None and self.Hkv > self.R:
             main.wait_stream(side_stream)
+        return self.o
+
+
+class CachedDecodeLayer:
+    """Decode over caches the layer keeps itself: every step appends the new
+    token's keys and values, then attends with it.
+
+        rtp_kv_append       new K/V -> retrieval heads' full caches and projected
+                            keys, local heads' W-row rings (one launch)
+        a1  rtp_index_project   queries of the retrieval heads -> q_idx
+        a3  rtp_topp_select     top-p over the retrieval heads' caches
+        a4  rtp_sparse_attn_decode   attention over the selected keys
+        a5  rtp_window_attn     the local heads over their rings
+
+    Retrieval heads (the first R KV heads) keep the full cache, local heads only
+    the last W tokens ("RTPurbo: Turning Dense LLMs into Sparse Attention Models
+    ...", "Three Key Insights" 1), so a local head's cache is W rows whatever the
+    context length.  Sequence lengths live on the device (two buffers used in
+    turn: one is an append's ``pos``, the other its ``lens_out``); the host never
+    reads them.  Inputs of a step go into ``q`` [B, Hq, 1, D], ``k_new`` and
+    ``v_new`` [B, Hkv, 1, D] (in place, or through the arguments of ``step``).
+    """
+
+    def __init__(self, B: int, Hq: int, Hkv: int, N: int, R: int, W: int, p: float, P: torch.Tensor,
+                 dtype: torch.dtype = torch.bfloat16, out_dtype: torch.dtype = torch.float32,
+                 scale: Optional[float] = None, device=None, D: int = 128):
+        dev = P.device if device is None else torch.device(device)
+        if Hq % Hkv or not 0 <= R <= Hkv or W < 1:
+            raise ValueError("need Hkv | Hq, 0 <= R <= Hkv and W >= 1")
+        self.B, self.Hq, self.Hkv, self.N, self.D = B, Hq, Hkv, N, D
+        self.G = G = Hq // Hkv
+        self.R, self.W, self.p = R, W, float(p)
+        self.scale = (D ** -0.5) if scale is None else scale
+        self.P = P
+        L = Hkv - R
+        self.k_cache = torch.zeros(B, R, N, D, dtype=dtype, device=dev)
+        self.v_cache = torch.zeros(B, R, N, D, dtype=dtype, device=dev)
+        self.k_idx = torch.zeros(B, R, N, 16, dtype=dtype, device=dev)
+        self.k_ring = torch.zeros(B, L, W, D, dtype=dtype, device=dev)
+        self.v_ring = torch.zeros(B, L, W, D, dtype=dtype, device=dev)
+        self._lens = [torch.zeros(B, dtype=torch.int32, device=dev) for _ in range(2)]
+        self.ring_lens = torch.zeros(B, dtype=torch.int32, device=dev)
+        self._cur = 0
+        self.q = torch.zeros(B, Hq, 1, D, dtype=dtype, device=dev)
+        self.k_new = torch.zeros(B, Hkv, 1, D, dtype=dtype, device=dev)
+        self.v_new = torch.zeros(B, Hkv, 1, D, dtype=dtype, device=dev)
+        self.q_idx = torch.zeros(B, R * G, 1, 16, dtype=dtype, device=dev)
+        self.o = torch.zeros(B, Hq, 1, D, dtype=out_dtype, device=dev)
+        self.sel = rtp.Selection.empty(B * R * G, N, dev)
+        self.ws_sel = rtp.workspace(rtp.topp_select_workspace_size(B, R * G, 1, R, N), dev)
+        self.ws_ret = rtp.workspace(rtp.sparse_attn_decode_workspace_size(B, R * G, R, N), dev) if R else None
+        self.ws_loc = (rtp.workspace(rtp.window_attn_workspace_size(B, Hq - R * G, 1, L, W, W), dev)
+                       if L else None)
+        self._plans = {}
+
+    @property
+    def lens(self) -> torch.Tensor:
+        """Device lengths of the sequences (tokens appended so far, capped at N)."""
+        return self._lens[self._cur]
+
+    def cache_bytes(self) -> int:
+        """Device bytes of the K/V caches, rings and projected keys."""
+        return sum(t.numel() * t.element_size() for t in (self.k_cache, self.v_cache, self.k_idx,
+                                                         self.k_ring, self.v_ring))
+
+    def set_lengths(self, lens: torch.Tensor) -> None:
+        """Declare how many tokens each sequence holds (for caches filled by the caller)."""
+        self._lens[self._cur].copy_(lens.to(torch.int32))
+        self.ring_lens.copy_(torch.clamp(lens.to(torch.int32), 0, self.W))
+
+    def append(self, k_new: torch.Tensor, v_new: torch.Tensor, stream=None) -> None:
+        """Append T tokens [B, Hkv, T, D] to every sequence (a chunk of prefill);
+        tokens beyond the cache's N rows are dropped."""
+        R, L = self.R, self.Hkv - self.R
+        cur = self._cur
+        rtp.kv_append(k_new, v_new, self._lens[cur], R, self.P if R else None,
+                      self.k_cache if R else None, self.v_cache if R else None, self.k_idx if R else None,
+                      self.k_ring if L else None, self.v_ring if L else None, self._lens[1 - cur],
+                      self.ring_lens if L else None, stream)
+        self._cur = 1 - cur
+
+    def _plan(self, cur: int, main: torch.cuda.Stream, side: Optional[torch.cuda.Stream]):
+        R, G, L = self.R, self.G, self.Hkv - self.R
+        pos, lens = self._lens[cur], self._lens[1 - cur]
+        pre, win, chain = [], [], []
+        pre.append(rtp.bind_kv_append(self.k_new, self.v_new, pos, R, self.P if R else None,
+                                      self.k_cache if R else None, self.v_cache if R else None,
+                                      self.k_idx if R else None, self.k_ring if L else None,
+                                      self.v_ring if L else None, lens, self.ring_lens if L else None, main))
+        if R:
+            pre.append(rtp.bind_index_project(self.q[:, : R * G], self.P, self.q_idx, main))
+            chain.append(rtp.bind_topp_select(self.q_idx, self.k_idx, lens, self.p, self.sel, self.ws_sel, main))
+            chain.append(rtp.bind_sparse_attn_decode(self.q[:, : R * G], self.k_cache, self.v_cache, lens, self.sel,
+                                                     self.scale, self.o[:, : R * G], self.ws_ret, main))
+        if L:
+            win.append(rtp.bind_window_attn(self.q[:, R * G:], self.k_ring, self.v_ring, self.ring_lens, self.W,
+                                            self.scale, self.o[:, R * G:], self.ws_loc,
+                                            main if side is None else side))
+        return pre, win, chain
+
+    def step(self, q: Optional[torch.Tensor] = None, k_new: Optional[torch.Tensor] = None,
+             v_new: Optional[torch.Tensor] = None, stream=None,
+             side_stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+        """Append the new token of every sequence and decode it; returns o [B, Hq, 1, D].
+        With ``side_stream`` the local heads' window attention runs there."""
+        for dst, src in ((self.q, q), (self.k_new, k_new), (self.v_new, v_new)):
+            if src is not None:
+                dst.copy_(src)
+        main = torch.cuda.current_stream() if stream is None else stream
+        key = (self._cur, main.cuda_stream, None if side_stream is None else side_stream.cuda_stream)
+        plan = self._plans.get(key)
+        if plan is None:
+            plan = self._plans[key] = self._plan(self._cur, main, side_stream)
+        pre, win, chain = plan
+        for call in pre:
+            call()
+        if win and side_stream is not None:
+            side_stream.wait_stream(main)
+            for call in win:
+                call()
+            for call in chain:
+                call()
+            main.wait_stream(side_stream)
+        else:
+            for call in chain:
+                call()
+            for call in win:
+                call()
+        self._cur = 1 - self._cur
         return self.o

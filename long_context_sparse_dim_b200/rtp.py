@@ -27,7 +27,7 @@ EXPORTED = ("rtp_index_project", "rtp_topp_select", "rtp_topp_select_workspace_s
             "rtp_sparse_attn_decode", "rtp_sparse_attn_decode_workspace_size", "rtp_sparse_attn_decode_noalloc",
             "rtp_sparse_attn_prefill", "rtp_sparse_attn_prefill_workspace_size",
             "rtp_window_attn", "rtp_window_attn_workspace_size",
-            "rtp_poll_device_error", "rtp_set_wait_budget_cycles", "rtp_status_string", "rtp_last_cuda_error",
+            "rtp_kv_append", "rtp_sparse_attn_decode_range", "rtp_attn_combine", "rtp_poll_device_error", "rtp_set_wait_budget_cycles", "rtp_status_string", "rtp_last_cuda_error",
             "rtp_version")
 
 
@@ -69,6 +69,9 @@ def _load() -> ctypes.CDLL:
         "rtp_sparse_attn_prefill_workspace_size": ([i64, i64, i64, i64, i64], sz),
         "rtp_window_attn": ([T, T, T, vp, i32, f32, T, vp, sz, vp], i32),
         "rtp_window_attn_workspace_size": ([i64, i64, i64, i64, i64, i32], sz),
+        "rtp_sparse_attn_decode_range": ([T, T, T, vp, S, i64, f32, T, T, vp, sz, vp], i32),
+        "rtp_attn_combine": ([T, T, T, vp], i32),
+        "rtp_kv_append": ([T, T, vp, i32, T, T, T, T, T, T, vp, vp, vp], i32),
         "rtp_poll_device_error": ([P(i32)], i32),
         "rtp_set_wait_budget_cycles": ([i64], i32),
         "rtp_status_string": ([i32], ctypes.c_char_p),
@@ -171,12 +174,38 @@ def _ws(ws: Optional[torch.Tensor]):
 
 
 # --------------------------------------------------------------------------
-# the five calls
+# the calls
 # --------------------------------------------------------------------------
 
 def index_project(x: torch.Tensor, P: torch.Tensor, x_idx: torch.Tensor, stream=None) -> None:
     _check(_lib.rtp_index_project(ctypes.byref(tensor_desc(x)), ctypes.byref(tensor_desc(P, 3)),
                                   ctypes.byref(tensor_desc(x_idx)), _stream(stream)), "rtp_index_project")
+
+
+def _opt_desc(t: Optional[torch.Tensor], ndim: int = 4, keep=None):
+    if t is None:
+        return None
+    d = tensor_desc(t, ndim)
+    if keep is not None:
+        keep.append(d)
+    return ctypes.byref(d)
+
+
+def _kv_append_args(k_new, v_new, pos, R, P, k_cache, v_cache, k_idx, k_ring, v_ring, lens_out, ring_lens,
+                    stream, keep):
+    return [_opt_desc(k_new, keep=keep), _opt_desc(v_new, keep=keep), _ptr(pos), ctypes.c_int32(int(R)),
+            _opt_desc(P, 3, keep), _opt_desc(k_cache, keep=keep), _opt_desc(v_cache, keep=keep),
+            _opt_desc(k_idx, keep=keep), _opt_desc(k_ring, keep=keep), _opt_desc(v_ring, keep=keep),
+            _ptr(lens_out), _ptr(ring_lens), _stream(stream)]
+
+
+def kv_append(k_new, v_new, pos, R: int, P=None, k_cache=None, v_cache=None, k_idx=None, k_ring=None,
+              v_ring=None, lens_out=None, ring_lens=None, stream=None) -> None:
+    """Append T new tokens per sequence: retrieval heads (the first R KV heads)
+    to the full caches and the projected-key cache, local heads to W-row rings."""
+    keep = []
+    _check(_lib.rtp_kv_append(*_kv_append_args(k_new, v_new, pos, R, P, k_cache, v_cache, k_idx, k_ring, v_ring,
+                                               lens_out, ring_lens, stream, keep)), "rtp_kv_append")
 
 
 def topp_select_workspace_size(B, Hq, T, Hk, N) -> int:
@@ -212,6 +241,25 @@ def sparse_attn_decode(q, k, v, lens, sel: Selection, scale: float, o, ws=None, 
 
 
 NOALLOC_SCRATCH_BYTES = 4 << 20
+
+
+def sparse_attn_decode_range(q, k, v, lens, sel: Selection, key_lo: int, scale: float, o, lse, ws=None,
+                            stream=None) -> None:
+    """Attention over the selected keys among rows key_lo .. key_lo + N - 1 of
+    each sequence (k, v hold just those rows); lse [B, Hq] f32 (last dim
+    contiguous) receives the log-sum-exp for rtp_attn_combine."""
+    w, nb = _ws(ws)
+    _check(_lib.rtp_sparse_attn_decode_range(ctypes.byref(tensor_desc(q)), ctypes.byref(tensor_desc(k)),
+                                             ctypes.byref(tensor_desc(v)), _ptr(lens), ctypes.byref(sel.desc()),
+                                             int(key_lo), float(scale), ctypes.byref(tensor_desc(o)),
+                                             ctypes.byref(tensor_desc(lse, 2)), w, nb, _stream(stream)),
+           "rtp_sparse_attn_decode_range")
+
+
+def attn_combine(o_parts, lse_parts, o, stream=None) -> None:
+    """o [B, Hq, 1, 128] from S partials o_parts [S, B, Hq, 128] f32 and lse_parts [S, B, Hq] f32."""
+    _check(_lib.rtp_attn_combine(ctypes.byref(tensor_desc(o_parts)), ctypes.byref(tensor_desc(lse_parts, 3)),
+                                 ctypes.byref(tensor_desc(o)), _stream(stream)), "rtp_attn_combine")
 
 
 def sparse_attn_decode_noalloc(q, k, v, lens, sel: Selection, scale: float, o, stream=None) -> None:
@@ -308,6 +356,29 @@ def bind_window_attn(q, k, v, lens, W: int, scale: float, o, ws=None, stream=Non
                  [_ref(tensor_desc(q), keep), _ref(tensor_desc(k), keep), _ref(tensor_desc(v), keep), _ptr(lens),
                   ctypes.c_int32(W), ctypes.c_float(scale), _ref(tensor_desc(o), keep), w, ctypes.c_size_t(nb),
                   _stream(stream)], keep)
+
+
+def bind_kv_append(k_new, v_new, pos, R: int, P=None, k_cache=None, v_cache=None, k_idx=None, k_ring=None,
+                   v_ring=None, lens_out=None, ring_lens=None, stream=None) -> Bound:
+    keep = [k_new, v_new, pos, P, k_cache, v_cache, k_idx, k_ring, v_ring, lens_out, ring_lens]
+    return Bound("rtp_kv_append", _kv_append_args(k_new, v_new, pos, R, P, k_cache, v_cache, k_idx, k_ring,
+                                                  v_ring, lens_out, ring_lens, stream, keep), keep)
+
+
+def bind_sparse_attn_decode_range(q, k, v, lens, sel: Selection, key_lo: int, scale: float, o, lse, ws=None,
+                                  stream=None) -> Bound:
+    keep = [q, k, v, lens, sel, o, lse, ws]
+    w, nb = _ws(ws)
+    return Bound("rtp_sparse_attn_decode_range",
+                 [_ref(tensor_desc(q), keep), _ref(tensor_desc(k), keep), _ref(tensor_desc(v), keep), _ptr(lens),
+                  _ref(sel.desc(), keep), ctypes.c_int64(key_lo), ctypes.c_float(scale), _ref(tensor_desc(o), keep),
+                  _ref(tensor_desc(lse, 2), keep), w, ctypes.c_size_t(nb), _stream(stream)], keep)
+
+
+def bind_attn_combine(o_parts, lse_parts, o, stream=None) -> Bound:
+    keep = [o_parts, lse_parts, o]
+    return Bound("rtp_attn_combine", [_ref(tensor_desc(o_parts), keep), _ref(tensor_desc(lse_parts, 3), keep),
+                                      _ref(tensor_desc(o), keep), _stream(stream)], keep)
 
 
 def poll_device_error() -> int:

@@ -195,6 +195,32 @@ def attend(q: np.ndarray, K: np.ndarray, V: np.ndarray, idx: np.ndarray, scale: 
     return (e[:, None] * Vs).sum(axis=0) / e.sum()
 
 
+def attend_lse(q: np.ndarray, K: np.ndarray, V: np.ndarray, idx: np.ndarray,
+               scale: float) -> Tuple[np.ndarray, float]:
+    """attend() over idx, and ln sum_j exp(q . K[j] * scale) over the same keys
+    (-inf for an empty set): what one device reports for the keys it holds
+    when a sequence's keys are split by position over several devices."""
+    o = attend(q, K, V, idx, scale)
+    idx = np.asarray(idx, dtype=np.int64)
+    if idx.size == 0:
+        return o, -np.inf
+    logits = (np.asarray(K[idx], dtype=np.float64) @ np.asarray(q, dtype=np.float64)) * scale
+    m = logits.max()
+    return o, float(m + np.log(np.exp(logits - m).sum()))
+
+
+def combine_partials(parts: Sequence[Tuple[np.ndarray, float]]) -> np.ndarray:
+    """Attention over a union of disjoint key sets from the per-set results
+    (o_s, lse_s): softmax weights over the union split as exp(lse_s) per set,
+    so o = sum_s exp(lse_s) o_s / sum_s exp(lse_s); all sets empty gives 0."""
+    lses = np.array([lse for _, lse in parts], dtype=np.float64)
+    if lses.size == 0 or np.all(np.isneginf(lses)):
+        return np.zeros(np.asarray(parts[0][0]).shape if parts else 0, dtype=np.float64)
+    m = lses.max()
+    w = np.exp(lses - m)
+    return sum(wi * np.asarray(o, dtype=np.float64) for wi, (o, _) in zip(w, parts)) / w.sum()
+
+
 def window_keys(pos: int, W: int) -> np.ndarray:
     """Local-head keys of a query at ``pos``: the last W positions up to pos ([B] insight 1, R6)."""
     if W < 1:

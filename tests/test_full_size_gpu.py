@@ -1,8 +1,9 @@
 """GPU parity at the full workload sizes, in the launch configuration bench.py
 times: decode of 4 sequences of 131072 keys (three top-p masses), causal
 prefill of 32768 tokens, and the last 8192 tokens against a 1,048,576-token
-cache.  Prefill checks a seeded sample of query tokens (always the first and
-the last) over every head; decode checks every query."""
+cache (and one decode query against a cache of that length).  Prefill checks a
+seeded sample of query tokens (32 of them besides the first and the last) over
+every head; decode checks every query."""
 import numpy as np
 import pytest
 import torch
@@ -74,15 +75,16 @@ def test_prefill_t32768_causal_sampled():
 
 
 def test_prefill_chunk_t8192_n1048576_sampled():
-    _prefill_full(wl.PREFILL_CHUNK_1M, 6, 1)
+    _prefill_full(wl.PREFILL_CHUNK_1M, 32, 1)
 
 
-def test_decode_b1_n524288_longest_supported():
-    # the longest decode context: one retrieval KV head (4 query heads, one
-    # 16-CTA cluster each in the selection) and one local KV head; the sparse
-    # attention needs its largest chunk (8192 keys x 64 splits)
+def test_decode_b1_n1048576():
+    # a million-key decode context: one retrieval KV head (4 query heads, one
+    # 16-CTA cluster each in the selection, each CTA recomputing the scores it
+    # cannot keep on chip) and one local KV head; the sparse attention splits the
+    # keys over 256 CTAs of 4096
     from long_context_sparse_dim_b200.layer import DecodeLayer
-    w = wl.DECODE_B4_N128K.replace(name="decode_b1_n524288", B=1, N=524288, Hq=8, Hkv=2, R=1, needles=64,
+    w = wl.DECODE_B4_N128K.replace(name="decode_b1_n1048576", B=1, N=1 << 20, Hq=8, Hkv=2, R=1, needles=64,
                                    p=0.95, seed=21)
     inst = wl.generate(w)
     q, k, v, P, lens = upload(inst)

@@ -320,3 +320,69 @@ def test_topk_select_validation():
     assert L.rtp_topk_select(by(qi), by(ki), None, 5, None, None, 0, None) == 1           # no selection
     assert L.rtp_topk_select(by(_desc(rtp, [2, 8, 3, 16])), by(ki), None, 5, by(s), None, 0, None) == 7  # T != 1
     assert L.rtp_topk_select(by(_desc(rtp, [2, 7, 1, 16])), by(ki), None, 5, by(s), None, 0, None) == 2
+
+
+def test_kv_append_validation():
+    rtp = _lib()
+    L = rtp.lib()
+    by = ctypes.byref
+    B, H, R, T, N, W = 2, 4, 1, 3, 64, 16
+    kn = _desc(rtp, [B, H, T, 128])
+    P = _desc(rtp, [R, 16, 128], dtype=0)
+    kc = _desc(rtp, [B, R, N, 128])
+    ki = _desc(rtp, [B, R, N, 16])
+    kr = _desc(rtp, [B, H - R, W, 128])
+    pos, out, rl = ctypes.c_void_p(0x20000), ctypes.c_void_p(0x30000), ctypes.c_void_p(0x40000)
+    fn = L.rtp_kv_append
+
+    def call(pos=pos, R=R, P=by(P), kc=by(kc), ki=by(ki), kr=by(kr), out=out, rl=rl, kn=by(kn)):
+        return fn(kn, kn, pos, R, P, kc, kc, ki, kr, kr, out, rl, None)
+
+    assert call(pos=None) == 1                                    # no positions
+    assert call(R=5) == 1 and call(R=-1) == 1                     # R outside [0, H]
+    assert call(out=pos) == 1 and call(rl=pos) == 1 and call(out=rl) == 1   # aliased length buffers
+    assert call(P=None) == 1                                      # retrieval heads need P
+    assert call(kr=None) == 1                                     # local heads need a ring
+    assert call(P=by(_desc(rtp, [2, 16, 128], dtype=0))) == 2     # one P per retrieval head
+    assert call(P=by(_desc(rtp, [R, 16, 128]))) == 3              # P is f32
+    assert call(kc=by(_desc(rtp, [B, 2, N, 128]))) == 2           # cache heads != R
+    assert call(ki=by(_desc(rtp, [B, R, N + 1, 16]))) == 2        # projected rows != cache rows
+    assert call(kc=by(_desc(rtp, [B, R, N, 128], dtype=0))) == 3  # cache dtype != new rows
+    assert call(kr=by(_desc(rtp, [B, H - R, 0, 128]))) == 2       # an empty ring
+    assert call(kr=by(_desc(rtp, [B + 1, H - R, W, 128]))) == 2   # ring batch != B
+    assert call(kn=by(_desc(rtp, [B, H, T, 64]))) == 2            # head dim 128
+    # all heads retrieval heads: no ring, and no ring lengths
+    assert fn(by(kn), by(kn), pos, H, by(_desc(rtp, [H, 16, 128], dtype=0)), by(_desc(rtp, [B, H, N, 128])),
+              by(_desc(rtp, [B, H, N, 128])), by(_desc(rtp, [B, H, N, 16])), None, None, out, rl, None) == 1
+
+
+def test_cached_decode_layer_marshals_append_then_the_step():
+    import torch
+    rtp = _lib()
+    from long_context_sparse_dim_b200.layer import CachedDecodeLayer
+    B, Hq, Hkv, N, D, R, W = 2, 8, 2, 300, 128, 1, 64
+    G = Hq // Hkv
+    P = torch.zeros(R, 16, D)
+    layer = CachedDecodeLayer(B, Hq, Hkv, N, R, W, 0.9, P, device="cpu")
+    main, side = _FakeStream(11), _FakeStream(22)
+    for cur in (0, 1):
+        pre, win, chain = layer._plan(cur, main, side)
+        assert [c._name for c in pre] == ["rtp_kv_append", "rtp_index_project"]
+        assert [c._name for c in win] == ["rtp_window_attn"]
+        assert [c._name for c in chain] == ["rtp_topp_select", "rtp_sparse_attn_decode"]
+        app = pre[0]._args
+        pos, lens = layer._lens[cur], layer._lens[1 - cur]
+        assert app[2].value == pos.data_ptr() and app[10].value == lens.data_ptr()
+        assert app[11].value == layer.ring_lens.data_ptr() and app[3].value == R
+        kn, vn, Pd, kc, vc, ki, kr, vr = _descs(pre[0], rtp)
+        assert list(kn.shape) == [B, Hkv, 1, D] and kn.data == layer.k_new.data_ptr()
+        assert list(kc.shape) == [B, R, N, D] and list(kr.shape) == [B, Hkv - R, W, D]
+        assert list(ki.shape) == [B, R, N, 16] and Pd.ndim == 3
+        # the selection and sparse attention read the lengths the append writes
+        assert chain[0]._args[2].value == lens.data_ptr() and chain[1]._args[3].value == lens.data_ptr()
+        # the window attention reads the ring with its lengths, window W
+        wq, wk, wv, wo = _descs(win[0], rtp)
+        assert wk.data == layer.k_ring.data_ptr() and list(wk.shape) == [B, Hkv - R, W, D]
+        assert win[0]._args[3].value == layer.ring_lens.data_ptr() and win[0]._args[4].value == W
+        assert wq.data == layer.q.data_ptr() + R * G * D * 2 and win[0]._args[-1].value == 22
+    assert layer.cache_bytes() == 2 * B * R * N * D * 2 + B * R * N * 16 * 2 + 2 * B * (Hkv - R) * W * D * 2

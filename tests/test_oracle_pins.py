@@ -446,3 +446,47 @@ def test_needle_recall_hand_case():
            (0, 5, 0): oracle.QueryResult(np.zeros(4), None, None)}
     needles = [(0, 0, 0, 0, 4), (0, 0, 0, 0, 2), (0, 1, 5, 0, 3)]
     assert oracle.needle_recall(res, needles) == (1, 2)
+
+
+# --------------------------------------------------------------------------
+# keys split by position over devices: per-range results and their merge
+# --------------------------------------------------------------------------
+
+def test_lse_closed_forms():
+    rng = np.random.default_rng(40)
+    q = rng.standard_normal(128)
+    K = np.tile(rng.standard_normal(128), (5, 1))          # five identical keys
+    V = rng.standard_normal((5, 128))
+    scale = 1 / math.sqrt(128)
+    a = float(K[0] @ q) * scale
+    o, lse = oracle.attend_lse(q, K, V, np.arange(5), scale)
+    assert lse == pytest.approx(a + math.log(5), rel=0, abs=1e-12)      # n equal logits: a + ln n
+    np.testing.assert_allclose(o, V.mean(axis=0), rtol=1e-12, atol=1e-12)
+    o1, lse1 = oracle.attend_lse(q, K, V, np.array([3]), scale)
+    assert lse1 == pytest.approx(a, abs=1e-12)
+    np.testing.assert_array_equal(o1, V[3])
+    o0, lse0 = oracle.attend_lse(q, K, V, np.array([], dtype=np.int64), scale)
+    assert lse0 == -np.inf and not o0.any()
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_range_partials_merge_to_attention_over_the_union(seed):
+    # softmax over a union of disjoint sets: independent check with torch's fp64
+    # attention over the union, the set split into ranges (one of them empty)
+    rng = np.random.default_rng(50 + seed)
+    n = 300
+    q = rng.standard_normal(128)
+    K = 2.0 * rng.standard_normal((n, 128))
+    V = rng.standard_normal((n, 128))
+    idx = np.sort(rng.choice(n, size=170, replace=False))
+    scale = 1 / math.sqrt(128)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q[None, None]), torch.from_numpy(K[idx][None]), torch.from_numpy(V[idx][None]),
+        scale=scale)[0, 0].numpy()
+    bounds = [0, 64, 64, 192, n]                           # [64, 64) is empty
+    parts = [oracle.attend_lse(q, K, V, idx[(idx >= lo) & (idx < hi)], scale) for lo, hi in zip(bounds, bounds[1:])]
+    assert parts[1][1] == -np.inf
+    np.testing.assert_allclose(oracle.combine_partials(parts), ref, rtol=1e-12, atol=1e-12)
+    # a lone partial with lse 0 passes through unchanged
+    np.testing.assert_array_equal(oracle.combine_partials([(parts[0][0], 0.0), (parts[2][0], -np.inf)]), parts[0][0])
+    assert not oracle.combine_partials([(parts[1][0], -np.inf), (parts[1][0], -np.inf)]).any()

@@ -128,3 +128,30 @@ def test_select_mixed_rows_in_one_launch():
     d[7] = 25.0
     _check_rows(np.stack([a, b, c, d]), 0.9, "mixed p=0.9")
     _check_rows(np.stack([a, b, c, d]), 0.99999, "mixed p=0.99999")
+
+
+def test_select_scores_streamed_past_the_resident_ones():
+    # 700000 keys: 16 CTAs of 43776 keys, of which each keeps 32768 scores in
+    # shared memory and recomputes the rest in every pass.  Random rows, a tie
+    # group placed inside the recomputed parts with the cut in its middle, and a
+    # row whose first-pass bin overflows (key-space passes over both parts)
+    rng = np.random.default_rng(17)
+    N, chunk = 700000, 43776
+    a = rng.standard_normal(N).astype(np.float32)
+    streamed = np.concatenate([np.arange(r * chunk + 32768, min((r + 1) * chunk, N)) for r in range(16)])
+    tie_pos = np.sort(rng.choice(streamed, size=40, replace=False))
+    t = rng.standard_normal(N).astype(np.float32)
+    v = np.float32(np.sort(t)[N - 3000])
+    t[t == v] = np.float32(v + 1e-3)
+    t[tie_pos] = v
+    t64 = t.astype(np.float64)
+    order = np.lexsort((np.arange(N), -t64))
+    w = np.exp(t64[order] - t64.max())
+    cum = np.cumsum(w)
+    k20 = int(np.flatnonzero(order == tie_pos[19])[0])
+    p_tie = float(np.float32((cum[k20] - 0.5 * w[k20]) / cum[-1]))
+    _check_rows(a[None], 0.9, "streamed normal")
+    (ref, mask, count, tau, tp), = _check_rows(t[None], p_tie, "streamed ties")
+    assert tau == v and tp == tie_pos[19] and count == ref.count
+    u = rng.uniform(0.0, 0.06, size=(1, N)).astype(np.float32)
+    _check_rows(u, 0.5, "streamed overflow")
