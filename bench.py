@@ -744,6 +744,27 @@ def _cpu_baseline_prefill(inst, wl, budget_s):
                       f"projected-key cache prebuilt, {dt:.1f} s"}
 
 
+def _needle_recall(layer, inst, wl):
+    """Planted needles whose key is in their query's selected set, read from the
+    selection's threshold form (score > tau, or == tau at a position <= tiepos);
+    scores recomputed from the stored projected vectors in fp64 (a tie-band
+    difference from the GPU's fp32 score can only move needles at the cut)."""
+    if not inst.needles:
+        return None
+    import torch
+    nd = np.array(inst.needles, dtype=np.int64)                 # (b, kv head, q head, t, key position)
+    b, kvh, h, t, j = nd.T
+    Hr = wl.R * wl.G
+    qi = layer.q_idx[torch.from_numpy(b), torch.from_numpy(h), torch.from_numpy(t)].double().cpu().numpy()
+    ki = layer.k_idx[torch.from_numpy(b), torch.from_numpy(kvh), torch.from_numpy(j)].double().cpu().numpy()
+    s = (qi * ki).sum(axis=1) / 4.0
+    rows = torch.from_numpy((b * Hr + h) * wl.T + t)
+    tau = layer.sel.tau_bits[rows].cpu().numpy().view(np.float32).astype(np.float64)
+    tp = layer.sel.tiepos[rows].cpu().numpy()
+    hit = (s > tau) | ((s == tau) & (j <= tp))
+    return {"recalled": int(hit.sum()), "needles": int(hit.size), "fraction": float(hit.mean())}
+
+
 def measure_prefill(args, wl, dev, world, steps, warmup, with_cpu):
     """One prefill workload measured on this rank: the JSON fields of its line."""
     import torch
@@ -795,6 +816,7 @@ def measure_prefill(args, wl, dev, world, steps, warmup, with_cpu):
 
     G, R = wl.G, wl.R
     T, N = wl.T, wl.N
+    needle = _needle_recall(layer, inst, wl)
     counts = layer.sel.count.cpu().numpy().astype(np.int64)
     admitted = int(counts.sum())                       # (query, key) pairs the sparse attention runs
     pos = np.arange(T) + N - T
@@ -828,7 +850,7 @@ def measure_prefill(args, wl, dev, world, steps, warmup, with_cpu):
                        "pairs_per_s": causal / (kernels_ms["topp_select"] * 1e-3)},
         "kernels_ms": kernels_ms,
         "kernels_tflops": {n: flop[n] / (kernels_ms[n] * 1e-3) / 1e12 for n in flop if n in kernels_ms},
-        "selection": {"mean_selected_fraction": admitted / max(causal, 1)},
+        "selection": {"mean_selected_fraction": admitted / max(causal, 1), "needle_recall": needle},
         "gpu_launches": len(calls) * steps,
         "streams": "window attention (local heads) forked onto a second stream inside each step",
         "clocks": clock_info,

@@ -210,7 +210,8 @@ RTP_API size_t rtp_sparse_attn_decode_workspace_size(int64_t B, int64_t Hq, int6
  * each query over its selected keys inside this range, plus the log-sum-exp
  * that rtp_attn_combine needs to merge the ranges.
  *   q, sel, scale  as for rtp_sparse_attn_decode (sel covers the whole
- *          sequence: mask_words * 32 >= key_lo + N)
+ *          sequence; keys past mask_words * 32 count as not selected, so the
+ *          last range may run past the sequence's end)
  *   k, v   [B, Hk, N, 128]  rows 0 .. N-1 hold keys key_lo .. key_lo + N - 1
  *   lens   int32[B] device or NULL: whole-sequence lengths (keys at or past
  *          lens[b] are not attended); NULL means key_lo + N

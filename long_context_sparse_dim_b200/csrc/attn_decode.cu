@@ -114,6 +114,8 @@ struct KeyRange {
 RTP_DEVICE KeyRange key_range(const AttnArgs& A, int b, int split) {
   int n_b = A.N;  // rows of this call's K/V: keys key_lo .. key_lo + n_b - 1 of the sequence
   if (A.lens) n_b = min(max(A.lens[b] - A.key_lo, 0), A.N);
+  // a key range may run past the keys the selection covers: those are not selected
+  if (A.W <= 0) n_b = (int)min((int64_t)n_b, max(A.mask_words * 32 - A.key_lo, (int64_t)0));
   KeyRange r;
   r.hi = n_b;
   r.lo = A.W > 0 ? max(0, n_b - A.W) : 0;

@@ -42,7 +42,7 @@ extern "C" rtp_status rtp_sparse_attn_decode_noalloc(const rtp_tensor* q, const 
                                                      const rtp_tensor* o, rtp_stream_t stream) {
   // every argument check first: an invalid call launches and writes nothing
   rtp::LaunchAttnDecode a;
-  const rtp_status s = rtp::check_sparse_attn_decode(q, k, v, lens, sel, scale, o, &a);
+  const rtp_status s = rtp::check_sparse_attn_decode(q, k, v, lens, sel, scale, o, &a, false);
   if (s != RTP_OK) return s;
   const size_t need = rtp_sparse_attn_decode_workspace_size(a.B, a.Hq, a.Hk, a.N);
   if (need > (size_t)RTP_NOALLOC_SCRATCH_BYTES) return RTP_ERR_UNSUPPORTED;

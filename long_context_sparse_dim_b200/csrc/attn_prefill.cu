@@ -100,15 +100,35 @@ RTP_DEVICE float max3f(float a, float b, float c) {
   return r;
 }
 
-RTP_DEVICE void named_sync(int id, int n) { asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(n) : "memory"); }
-
-// Bits j of a 32-key chunk with lo <= j <= hi.
-RTP_DEVICE uint32_t band32(int lo, int hi) {
-  if (hi < 0 || lo > 31 || hi < lo) return 0u;
-  const int l = max(lo, 0), r = min(hi, 31);
-  const uint32_t upto = r >= 31 ? 0xffffffffu : ((1u << (r + 1)) - 1u);
-  return upto & ~((1u << l) - 1u);
+// (a * s + c, b * s + c) in one packed fp32x2 fused multiply-add.
+RTP_DEVICE void fma2(float a, float b, float sc, float c, float& ra, float& rb) {
+  uint64_t x, y, z, r;
+  asm("mov.b64 %0, {%1, %2};\n" : "=l"(x) : "f"(a), "f"(b));
+  asm("mov.b64 %0, {%1, %2};\n" : "=l"(y) : "f"(sc), "f"(sc));
+  asm("mov.b64 %0, {%1, %2};\n" : "=l"(z) : "f"(c), "f"(c));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;\n" : "=l"(r) : "l"(x), "l"(y), "l"(z));
+  asm("mov.b64 {%0, %1}, %2;\n" : "=f"(ra), "=f"(rb) : "l"(r));
 }
+
+// (acc0, acc1) += (a, b) in one packed fp32x2 add.
+RTP_DEVICE void add2(float& acc0, float& acc1, float a, float b) {
+  uint64_t x, y, r;
+  asm("mov.b64 %0, {%1, %2};\n" : "=l"(x) : "f"(acc0), "f"(acc1));
+  asm("mov.b64 %0, {%1, %2};\n" : "=l"(y) : "f"(a), "f"(b));
+  asm("add.rn.f32x2 %0, %1, %2;\n" : "=l"(r) : "l"(x), "l"(y));
+  asm("mov.b64 {%0, %1}, %2;\n" : "=f"(acc0), "=f"(acc1) : "l"(r));
+}
+
+// (a - c, b - d) in one packed fp32x2 subtract.
+RTP_DEVICE void sub2p(float a, float b, float c, float d, float& ra, float& rb) {
+  uint64_t x, y, r;
+  asm("mov.b64 %0, {%1, %2};\n" : "=l"(x) : "f"(a), "f"(b));
+  asm("mov.b64 %0, {%1, %2};\n" : "=l"(y) : "f"(c), "f"(d));
+  asm("sub.rn.f32x2 %0, %1, %2;\n" : "=l"(r) : "l"(x), "l"(y));
+  asm("mov.b64 {%0, %1}, %2;\n" : "=f"(ra), "=f"(rb) : "l"(r));
+}
+
+RTP_DEVICE void named_sync(int id, int n) { asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(n) : "memory"); }
 
 }  // namespace
 
@@ -255,47 +275,63 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
     const int h = kvh * A.G + (in_block ? row / TB : 0);
     const int t = in_block ? t0 + row % TB : A.T;
     const int pos = t < A.T ? qbase + t : -1;  // -1: no keys
-    float vtau = 0.f;  // raw indexer accumulator of the cut score (4 tau, an exact scaling)
+    float vtau = 0.f;     // raw indexer accumulator of the cut score (4 tau, an exact scaling)
+    float vtau_lo = 0.f;  // the float just below it: x >= vtau  <=>  x > vtau_lo
     int tpos = -1;
     if (SPARSE && pos >= 0) {
       const int64_t qrow = ((int64_t)b * A.Hq + h) * A.T + t;
       vtau = __fmul_rn(__uint_as_float(A.tau_bits[qrow]), 4.f);
+      vtau_lo = nextafterf(vtau, -INFINITY);
       tpos = A.tiepos[qrow];
     }
+    const int wlo = pos - A.W + 1;  // window: first key a local row sees (may be negative)
     const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16) + 64u * (uint32_t)hf;
     float m_run = -INFINITY;  // running maximum of the scaled logits (log2 units)
+    // The logits of 16 keys from k0 on, with the keys the row does not attend set to -inf.
+    // Sparse: key k is attended iff k <= pos and (x > vtau or (x == vtau and k <= tpos)), x
+    // its indexer accumulator; inside the causal prefix and away from the tie position that
+    // is one compare against vtau or vtau_lo.  Window: wlo <= k <= pos.
+    // Returns whether any of the 16 was masked.
+    auto admit16 = [&](uint32_t (&v)[16], const uint32_t (&x)[16], int k0) -> bool {
+      uint32_t any = 0u;
+      if (SPARSE) {
+        if (k0 + 15 <= pos && (k0 > tpos || k0 + 15 <= tpos)) {
+          const float th = k0 > tpos ? vtau : vtau_lo;
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const bool out = !(__uint_as_float(x[j]) > th);
+            any |= (uint32_t)out;
+            v[j] = out ? 0xff800000u : v[j];
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const float xf = __uint_as_float(x[j]);
+            const int k = k0 + j;
+            const bool out = !(k <= pos && (xf > vtau || (xf == vtau && k <= tpos)));
+            any |= (uint32_t)out;
+            v[j] = out ? 0xff800000u : v[j];
+          }
+        }
+      } else if (!(k0 >= wlo && k0 + 15 <= pos)) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const bool out = !(k0 + j >= wlo && k0 + j <= pos);
+          any |= (uint32_t)out;
+          v[j] = out ? 0xff800000u : v[j];
+        }
+      }
+      return any != 0u;
+    };
     for (int i = 0; i < ntiles; ++i) {
       const int bi = i & 1;
       const int kh = (tile0 + i) * kAtKeys + 64 * hf;  // first key of this thread's half
-      // admission bits of this row over the half's 64 keys
-      uint32_t adm[2];
       if (SPARSE) {
         const bool ok = __all_sync(0xffffffffu, mbar_wait(&S.idx_full, (uint32_t)i & 1u, alive, A.err, A.budget));
         if (!ok) {
           alive = false;
           break;
         }
-        tc_fence_after();
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          uint32_t v[32];
-          tmem_ld32(lane_base + kTmemIdx + 32u * (uint32_t)c, v);
-          tmem_ld_wait();
-          uint32_t bits = 0u;
-#pragma unroll
-          for (int jj = 0; jj < 32; ++jj) {
-            const float x = __uint_as_float(v[jj]);
-            bits |= (uint32_t)(x > vtau || (x == vtau && kh + 32 * c + jj <= tpos)) << jj;
-          }
-          adm[c] = bits & band32(0, pos - kh - 32 * c);
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&S.idx_free);
-      } else {
-#pragma unroll
-        for (int c = 0; c < 2; ++c)
-          adm[c] = pos < 0 ? 0u : band32(max(pos - A.W + 1, 0) - kh - 32 * c, pos - kh - 32 * c);
       }
       const bool ok =
           __all_sync(0xffffffffu, mbar_wait(&S.s_full[bi], (uint32_t)(i >> 1) & 1u, alive, A.err, A.budget));
@@ -305,17 +341,28 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
       }
       tc_fence_after();
       const uint32_t sb = lane_base + kTmemS + (uint32_t)bi * kAtKeys;
-      // pass 1: the maximum of the admitted logits, over both halves of the row
+      const uint32_t ib = lane_base + kTmemIdx;
+      // pass 1: the logits the row does not attend are overwritten with -inf in place (so
+      // that pass 2 needs no admission test and the indexer tile is free for the next one),
+      // and the maximum of the rest is taken over both halves of the row
       float tmax = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t v[32];
-        tmem_ld32(sb + 32u * (uint32_t)c, v);
+      for (int q = 0; q < 4; ++q) {
+        uint32_t v[16], x[16];
+        tmem_ld16(sb + 16u * (uint32_t)q, v);
+        if (SPARSE) tmem_ld16(ib + 16u * (uint32_t)q, x);
         tmem_ld_wait();
+        // (the store is warp-collective: taken by every lane when any lane masked a logit)
+        if (__any_sync(0xffffffffu, admit16(v, x, kh + 16 * q))) tmem_st16(sb + 16u * (uint32_t)q, v);
 #pragma unroll
-        for (int jj = 0; jj < 32; jj += 2)
-          tmax = max3f(tmax, ((adm[c] >> jj) & 1u) ? __uint_as_float(v[jj]) : -INFINITY,
-                       ((adm[c] >> (jj + 1)) & 1u) ? __uint_as_float(v[jj + 1]) : -INFINITY);
+        for (int jj = 0; jj < 16; jj += 2)
+          tmax = max3f(tmax, __uint_as_float(v[jj]), __uint_as_float(v[jj + 1]));
+      }
+      tmem_st_wait();
+      if (SPARSE) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.idx_free);
       }
       S.pmax[bi][hf][row] = tmax;
       named_sync(1 + quad, 64);  // warps quad and quad + 4
@@ -327,29 +374,30 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
       // pass 2: P = 2^(s * scale * log2 e - m_new) as bf16 hi + lo, written over S
       // (16 keys at a time: slice q of 16 keys, which occupied columns
       // 16q .. 16q+15 as S, keeps its 8 hi words in 16q .. 16q+7 and its 8 lo
-      // words in 16q+8 .. 16q+15, so a store only overwrites what was just read)
-      float lsum = 0.f;
+      // words in 16q+8 .. 16q+15, so a store only overwrites what was just read).
+      // Pairs of keys go through packed fp32x2 instructions.
+      float l0 = 0.f, l1 = 0.f;
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        const int c = q >> 1, sub = q & 1;
         uint32_t v[16];
         tmem_ld16(sb + 16u * (uint32_t)q, v);
         tmem_ld_wait();
         uint32_t hi[8], lo[8];
 #pragma unroll
         for (int jj = 0; jj < 8; ++jj) {
-          const int k0 = 16 * sub + 2 * jj;
-          const float x0 = ((adm[c] >> k0) & 1u) ? __uint_as_float(v[2 * jj]) : -INFINITY;
-          const float x1 = ((adm[c] >> (k0 + 1)) & 1u) ? __uint_as_float(v[2 * jj + 1]) : -INFINITY;
-          const float p0 = ex2a(__fmaf_rn(x0, A.scale_log2, -m_ref));
-          const float p1 = ex2a(__fmaf_rn(x1, A.scale_log2, -m_ref));
-          lsum += p0 + p1;
+          float y0, y1, p0, p1, r0, r1;
+          fma2(__uint_as_float(v[2 * jj]), __uint_as_float(v[2 * jj + 1]), A.scale_log2, -m_ref, y0, y1);
+          p0 = ex2a(y0);
+          p1 = ex2a(y1);
+          add2(l0, l1, p0, p1);
           hi[jj] = pack_bf16x2(p0, p1);
-          lo[jj] = pack_bf16x2(p0 - bf16_lo(hi[jj]), p1 - bf16_hi(hi[jj]));
+          sub2p(p0, p1, bf16_lo(hi[jj]), bf16_hi(hi[jj]), r0, r1);
+          lo[jj] = pack_bf16x2(r0, r1);
         }
         tmem_st8(sb + 16u * (uint32_t)q, hi);
         tmem_st8(sb + 16u * (uint32_t)q + 8u, lo);
       }
+      const float lsum = l0 + l1;
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();

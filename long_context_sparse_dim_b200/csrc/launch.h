@@ -141,7 +141,7 @@ cudaError_t launch_attn_decode(const LaunchAttnDecode& a, cudaStream_t stream);
 // *a holds the launch arguments (a->ws still to be set).  Nothing is launched.
 rtp_status check_sparse_attn_decode(const rtp_tensor* q, const rtp_tensor* k, const rtp_tensor* v,
                                     const int32_t* lens, const rtp_selection* sel, float scale,
-                                    const rtp_tensor* o, LaunchAttnDecode* a);
+                                    const rtp_tensor* o, LaunchAttnDecode* a, bool key_range);
 // Byte range of the completion tickets inside a decode-attention workspace.
 void attn_decode_ticket_range(int64_t B, int64_t Hk, int64_t N, int32_t W, size_t* offset, size_t* bytes);
 

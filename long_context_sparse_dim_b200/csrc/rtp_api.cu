@@ -316,13 +316,14 @@ static rtp_status check_decode_common(const rtp_tensor* q, const rtp_tensor* k, 
 namespace rtp {
 rtp_status check_sparse_attn_decode(const rtp_tensor* q, const rtp_tensor* k, const rtp_tensor* v,
                                     const int32_t* lens, const rtp_selection* sel, float scale,
-                                    const rtp_tensor* o, LaunchAttnDecode* a) {
+                                    const rtp_tensor* o, LaunchAttnDecode* a, bool key_range) {
   rtp_status s;
   if ((s = check_decode_common(q, k, v, o, scale)) != RTP_OK) return s;
   if (q->shape[2] != 1) return RTP_ERR_SHAPE;
   if (!sel || !sel->mask) return RTP_ERR_INVALID_ARG;
   const int64_t N = k->shape[2];
-  if (sel->mask_words < (N + 31) / 32) return RTP_ERR_SHAPE;
+  // a key range's rows past the selection's keys count as not selected (the kernel clamps)
+  if (!key_range && sel->mask_words < (N + 31) / 32) return RTP_ERR_SHAPE;
   if (!attn_decode_supported(q->shape[0], k->shape[1], N, 0)) return RTP_ERR_UNSUPPORTED;
   a->q = view(q);
   a->k = view(k);
@@ -352,7 +353,7 @@ rtp_status rtp_sparse_attn_decode(const rtp_tensor* q, const rtp_tensor* k, cons
                                   rtp_stream_t stream) {
   rtp::LaunchAttnDecode a;
   rtp_status s;
-  if ((s = rtp::check_sparse_attn_decode(q, k, v, lens, sel, scale, o, &a)) != RTP_OK) return s;
+  if ((s = rtp::check_sparse_attn_decode(q, k, v, lens, sel, scale, o, &a, false)) != RTP_OK) return s;
   const size_t need = rtp_sparse_attn_decode_workspace_size(a.B, a.Hq, a.Hk, a.N);
   if ((s = check_workspace(workspace, workspace_bytes, need)) != RTP_OK) return s;
   a.ws = workspace;
@@ -367,10 +368,9 @@ rtp_status rtp_sparse_attn_decode_range(const rtp_tensor* q, const rtp_tensor* k
   rtp_status s;
   if (key_lo < 0 || key_lo % 64) return RTP_ERR_INVALID_ARG;
   if ((s = check_f32_rows(lse, 2)) != RTP_OK) return s;
-  if ((s = rtp::check_sparse_attn_decode(q, k, v, lens, sel, scale, o, &a)) != RTP_OK) return s;
+  if ((s = rtp::check_sparse_attn_decode(q, k, v, lens, sel, scale, o, &a, true)) != RTP_OK) return s;
   if (lse->shape[0] != a.B || lse->shape[1] != a.Hq) return RTP_ERR_SHAPE;
   if (key_lo + a.N > INT32_MAX) return RTP_ERR_SHAPE;
-  if (sel->mask_words < (key_lo + a.N + 31) / 32) return RTP_ERR_SHAPE;  // masks cover the whole sequence
   const size_t need = rtp_sparse_attn_decode_workspace_size(a.B, a.Hq, a.Hk, a.N);
   if ((s = check_workspace(workspace, workspace_bytes, need)) != RTP_OK) return s;
   a.ws = workspace;

@@ -140,6 +140,25 @@ RTP_DEVICE void sub2(float a, float b, float c, float& ra, float& rb) {
   asm("mov.b64 {%0, %1}, %2;\n" : "=f"(ra), "=f"(rb) : "l"(z));
 }
 
+// (c - a·s, c - b·s) in one packed fp32x2 fused multiply-add.
+RTP_DEVICE void cms2(float a, float b, float s, float c, float& ra, float& rb) {
+  uint64_t x, y, z, r;
+  asm("mov.b64 %0, {%1, %2};\n" : "=l"(x) : "f"(a), "f"(b));
+  asm("mov.b64 %0, {%1, %2};\n" : "=l"(y) : "f"(-s), "f"(-s));
+  asm("mov.b64 %0, {%1, %2};\n" : "=l"(z) : "f"(c), "f"(c));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;\n" : "=l"(r) : "l"(x), "l"(y), "l"(z));
+  asm("mov.b64 {%0, %1}, %2;\n" : "=f"(ra), "=f"(rb) : "l"(r));
+}
+
+// (a·s, b·s) in one packed fp32x2 multiply.
+RTP_DEVICE void mul2(float a, float b, float s, float& ra, float& rb) {
+  uint64_t x, y, r;
+  asm("mov.b64 %0, {%1, %2};\n" : "=l"(x) : "f"(a), "f"(b));
+  asm("mov.b64 %0, {%1, %2};\n" : "=l"(y) : "f"(s), "f"(s));
+  asm("mul.rn.f32x2 %0, %1, %2;\n" : "=l"(r) : "l"(x), "l"(y));
+  asm("mov.b64 {%0, %1}, %2;\n" : "=f"(ra), "=f"(rb) : "l"(r));
+}
+
 RTP_DEVICE float max3f(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;\n" : "=f"(r) : "f"(a), "f"(b), "f"(c));
@@ -354,7 +373,32 @@ topp_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
               m = max3f(m, max3f(a0, a1, a2), a3);
             }
           } else if (level == kLvLin0) {
-            if (own && nv > 0) {
+            if (own && nv >= 32) {
+              // the whole chunk is inside the prefix, so every u = m - v is >= 0: per pair of keys
+              // c0 u in one packed multiply-add (c0 a power of two: the same bits as c0 (m - v)),
+              // the weights' scalings in packed multiplies, and the two read-modify-writes
+              // overlapped (a pair in one bin is added as one update)
+              uint64_t* H = &S.hist[half][0][row];
+              const float mc = __fmul_rn(mh, A.c0), wmc = __fdiv_rn(wmul, A.c0);
+#pragma unroll
+              for (int j = 0; j < 32; j += 2) {
+                float u0, u1, x0, x1, e0, e1, y0, y1;
+                cms2(__uint_as_float(v[j]), __uint_as_float(v[j + 1]), A.c0, mc, u0, u1);
+                const int d0 = __float_as_int(__fadd_rd(fminf(u0, 31.f), 8388608.f)) - 0x4B000000;
+                const int d1 = __float_as_int(__fadd_rd(fminf(u1, 31.f), 8388608.f)) - 0x4B000000;
+                mul2(u0, u1, wmc, x0, x1);
+                asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(e0) : "f"(x0));
+                asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(e1) : "f"(x1));
+                y0 = __fmul_rn(e0, A.two_pow_frac);
+                y1 = __fmul_rn(e1, A.two_pow_frac);
+                const uint64_t w0 = __float2ull_rn(y0), w1 = __float2ull_rn(y1);
+                const uint64_t h0 = H[d0 * kPfRows], h1 = H[d1 * kPfRows];
+                const uint64_t s0 = h0 + w0;
+                const uint64_t s1 = (d0 == d1 ? s0 : h1) + w1;
+                H[d0 * kPfRows] = s0;
+                H[d1 * kPfRows] = s1;  // after s0: a pair in one bin ends as h + w0 + w1
+              }
+            } else if (own && nv > 0) {
               // every key lands in a bin; consecutive keys are taken in pairs so that the two
               // read-modify-writes overlap (a pair in one bin is added as one update)
               uint64_t* H = &S.hist[half][0][row];

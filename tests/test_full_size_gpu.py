@@ -64,8 +64,10 @@ def _prefill_full(w, n_sample, seed):
     for r_i, (h, t) in enumerate((h, t) for h in range(Hr) for t in toks):
         n = L.pos(0, t) + 1
         compare_selection(res[(0, h, t)], mask[r_i], n, int(count[r_i]), f"{w.name} h{h} t{t}")
+    # needle recall is a property of the method on this workload (the pages report > 90%), gated
+    # only where the sampled tokens hold enough needles to estimate it
     needles = [n for n in inst.needles if n[3] in set(toks)]
-    if needles:
+    if len(needles) >= 20:
         hit, tot = oracle.needle_recall(res, needles)
         assert hit / tot >= 0.9
 
