@@ -13,8 +13,9 @@ runs its own replica of the workload (weak scaling, no data-path collective).
 
 ``value`` is decode tokens/s (sequences advanced by one token per second,
 summed over ranks).  ``e2e`` is the same metric through the public API with
-host buffers: each step copies the new token's q/k/v from pinned host memory,
-makes the C-ABI calls, and reads the output back.  ``--impl reference`` times
+host buffers (``DecodeLayer.host_step``): each step copies the new token's
+q/k/v from pinned host memory, makes the C-ABI calls and reads the output
+back, replayed as one CUDA graph, with the host waiting for every token.  ``--impl reference`` times
 the CPU oracle on the same workload instead (rank 0 only).
 """
 from __future__ import annotations
@@ -678,21 +679,15 @@ def _e2e(layer, inst, wl, dev, steps):
     h_o = torch.empty(layer.o.shape, dtype=layer.o.dtype).pin_memory()
     h2d = h_q.numel() * h_q.element_size() + 2 * h_k.numel() * h_k.element_size()
     d2h = h_o.numel() * h_o.element_size()
-    side = torch.cuda.Stream(dev)
-    layer.step(side_stream=side)       # marshals the step's calls for this stream pair (untimed)
+    layer.host_step(h_q, h_k, h_v, h_o)      # captures the step's graph for these buffers (untimed)
     torch.cuda.synchronize()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record()
     for _ in range(steps):
-        layer.q.copy_(h_q, non_blocking=True)
-        layer.k[:, :, n - 1: n].copy_(h_k, non_blocking=True)
-        layer.v[:, :, n - 1: n].copy_(h_v, non_blocking=True)
-        layer.step(side_stream=side)
-        h_o.copy_(layer.o, non_blocking=True)
-        torch.cuda.current_stream().synchronize()
+        layer.host_step(h_q, h_k, h_v, h_o)  # copies in, the step, copy out, host waits for the output
     t1.record()
-    torch.cuda.synchronize()
+    t1.synchronize()
     ms = t0.elapsed_time(t1) / steps
     return {"value": wl.B / (ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
             "d2h_bytes_per_step": int(d2h), "ms_per_step": ms, "steps": steps}

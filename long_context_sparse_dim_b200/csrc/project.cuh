@@ -55,17 +55,18 @@ RTP_DEVICE void halve(float (&v)[kIdxDim], int lane, int bit) {
   }
 }
 
-// Lane l holds x[4l .. 4l+3] in xv and P[j][4l .. 4l+3] in Pl[j]; the warp writes
-// the 16 outputs of the row to out[0 .. 15].
-template <typename Tout>
-RTP_DEVICE void project_row(const float (&Pl)[kIdxDim][4], const float (&xv)[4], int lane, Tout* out) {
+// Lane l holds x[4l .. 4l+3] in xv and reads P[j][4l .. 4l+3] as pl(j) (a float4:
+// registers, or a load); the warp writes the 16 outputs of the row to out[0 .. 15].
+template <typename Tout, typename PL>
+RTP_DEVICE void project_row_with(PL pl, const float (&xv)[4], int lane, Tout* out) {
   float acc[kIdxDim];
 #pragma unroll
   for (int j = 0; j < kIdxDim; ++j) {
-    float a = __fmul_rn(Pl[j][0], xv[0]);
-    a = __fmaf_rn(Pl[j][1], xv[1], a);
-    a = __fmaf_rn(Pl[j][2], xv[2], a);
-    acc[j] = __fmaf_rn(Pl[j][3], xv[3], a);
+    const float4 pj = pl(j);
+    float a = __fmul_rn(pj.x, xv[0]);
+    a = __fmaf_rn(pj.y, xv[1], a);
+    a = __fmaf_rn(pj.z, xv[2], a);
+    acc[j] = __fmaf_rn(pj.w, xv[3], a);
   }
   halve<16>(acc, lane, 16);
   halve<8>(acc, lane, 8);
@@ -76,6 +77,13 @@ RTP_DEVICE void project_row(const float (&Pl)[kIdxDim][4], const float (&xv)[4],
     const int j = ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 + ((lane >> 1) & 1);
     store1<Tout>(out + j, y);
   }
+}
+
+// The same with P's block held in registers: Pl[j] = P[j][4l .. 4l+3].
+template <typename Tout>
+RTP_DEVICE void project_row(const float (&Pl)[kIdxDim][4], const float (&xv)[4], int lane, Tout* out) {
+  project_row_with<Tout>([&](int j) { return make_float4(Pl[j][0], Pl[j][1], Pl[j][2], Pl[j][3]); }, xv, lane,
+                         out);
 }
 
 }  // namespace rtp

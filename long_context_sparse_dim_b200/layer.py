@@ -115,6 +115,53 @@ class DecodeLayer:
                 call()
         return self.o
 
+    def host_step(self, h_q: torch.Tensor, h_k: torch.Tensor, h_v: torch.Tensor, h_o: torch.Tensor) -> torch.Tensor:
+        """One decode step end to end from host memory: copy the new token's
+        queries h_q [B, Hq, 1, D] and key/value rows h_k, h_v [B, Hkv, 1, D] (pinned
+        host tensors of the cache dtype) in, run the step, copy the output to h_o
+        [B, Hq, 1, D] (pinned) and wait for it.  The new rows land at each
+        sequence's last position.  The first call with a set of buffers captures
+        the copies and the calls in one CUDA graph (with the window attention on a
+        forked stream); later calls replay it, so a token costs one graph launch
+        and one synchronisation on the host."""
+        key = (h_q.data_ptr(), h_k.data_ptr(), h_v.data_ptr(), h_o.data_ptr())
+        ent = self._host_graphs.get(key) if hasattr(self, "_host_graphs") else None
+        if ent is None:
+            ent = self._capture_host(h_q, h_k, h_v, h_o)
+            self._host_graphs = getattr(self, "_host_graphs", {})
+            self._host_graphs[key] = ent
+        graph, stream = ent
+        graph.replay()
+        stream.synchronize()
+        return h_o
+
+    def _capture_host(self, h_q, h_k, h_v, h_o):
+        for t in (h_q, h_k, h_v, h_o):
+            if t.device.type != "cpu" or not t.is_pinned():
+                raise ValueError("host_step takes pinned host tensors")
+        dev = self.q.device
+        stream = torch.cuda.Stream(dev)
+        side = torch.cuda.Stream(dev)
+        rows = ([(slice(None), self.N - 1)] if self.lens_host is None else
+                [(slice(b, b + 1), n - 1) for b, n in enumerate(self.lens_host) if n > 0])
+
+        def body():
+            self.q.copy_(h_q, non_blocking=True)
+            for bs, n in rows:
+                self.k[bs, :, n: n + 1].copy_(h_k[bs], non_blocking=True)
+                self.v[bs, :, n: n + 1].copy_(h_v[bs], non_blocking=True)
+            self.step(side_stream=side)
+            h_o.copy_(self.o, non_blocking=True)
+
+        stream.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(stream):
+            body()                                   # marshals the calls for these streams (not captured)
+        stream.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            body()
+        return graph, stream
+
 
 class PrefillLayer:
     """One attention layer's RTPurbo prefill: T query tokens per sequence (the

@@ -175,3 +175,24 @@ def test_decode_side_stream_matches_single_stream():
     layer.step(side_stream=side)
     torch.cuda.synchronize()
     assert torch.equal(layer.o, o1)
+
+
+def test_host_step_matches_device_step():
+    # the end-to-end form (pinned host buffers in and out, one captured graph per
+    # buffer set) gives the device step's bits, on every replay
+    from long_context_sparse_dim_b200.layer import DecodeLayer
+    w = SMALL.replace(name="host_step", B=3, N=2000)
+    inst = wl.generate(w)
+    q, k, v, P, lens = upload(inst)
+    layer = DecodeLayer(q, k, v, P, R=w.R, W=w.W, p=w.p)
+    layer.build_index()
+    o_dev = layer.step().clone()
+    n = w.N
+    h_q = q.cpu().pin_memory()
+    h_k = k[:, :, n - 1: n].cpu().pin_memory()
+    h_v = v[:, :, n - 1: n].cpu().pin_memory()
+    h_o = torch.empty(o_dev.shape, dtype=o_dev.dtype).pin_memory()
+    for _ in range(3):
+        h_o.zero_()
+        layer.host_step(h_q, h_k, h_v, h_o)
+        assert torch.equal(h_o, o_dev.cpu())
