@@ -598,9 +598,11 @@ def _key_range_split(dev, N=1 << 20, worlds=(1, 2, 4, 8), reps=50):
     sel = rtp.Selection.empty(B * Hr, N, dev)
     scale = 1 / math.sqrt(D)
 
+    ws_sel = rtp.workspace(rtp.topp_select_workspace_size(B, Hr, 1, R, N), dev)
+
     def select():
         rtp.index_project(q[:, :Hr], P, q_idx)
-        rtp.topp_select(q_idx, k_idx, lens, p, sel)
+        rtp.topp_select(q_idx, k_idx, lens, p, sel, ws_sel)
 
     sel_ms = _timed(select, reps)
     out = {"N": N, "B": B, "W": W, "p": p, "selection_ms": sel_ms,

@@ -124,8 +124,10 @@ RTP_API rtp_status rtp_index_project(const rtp_tensor* x, const rtp_tensor* P, c
  * Query (b, h, t) ranks keys 0 .. pos by s = (q_idx . k_idx[j]) / 4 (fp32, fixed
  * summation order), weights exp(s - max s), and keeps the shortest prefix of
  * the (s desc, position asc) order whose weight reaches p * Z.
- * T == 1 (decode) is implemented for N <= 524288; T > 1 (prefill) uses the
- * tensor-core score tiles.  Workspace: rtp_topp_select_workspace_size().
+ * T == 1 (decode) is implemented for N <= 2097152 (past 524288 keys the
+ * workspace holds the scores the chip cannot keep: 4 bytes per key and query
+ * beyond 524288); T > 1 (prefill) uses the tensor-core score tiles.
+ * Workspace: rtp_topp_select_workspace_size() (0 for prefill and short caches).
  * Cites: "RTPurbo: Turning Dense LLMs ...", "Three Key Insights" 3 (cumulative
  * top-p per query); "Full Attention Strikes Back ... (RTPurbo)", Key findings.
  */

@@ -63,9 +63,11 @@ struct LaunchToppDecode {
   int32_t* count;
   uint32_t* mask;
   int64_t mask_words;
+  float* spill = nullptr;  // workspace: scores past the ones a CTA keeps on chip (long caches)
 };
 cudaError_t launch_topp_decode(const LaunchToppDecode& a, cudaStream_t stream);
 bool topp_decode_supported(int64_t N);
+size_t topp_decode_workspace_bytes(int64_t B, int64_t Hq, int64_t N);
 
 // Top-p selection, prefill form (T query tokens per sequence), tcgen05 score tiles.
 struct LaunchToppPrefill {

@@ -131,9 +131,11 @@ rtp_status rtp_index_project(const rtp_tensor* x, const rtp_tensor* P, const rtp
 
 // ---- a2 + a3 ---------------------------------------------------------------------
 size_t rtp_topp_select_workspace_size(int64_t B, int64_t Hq, int64_t T, int64_t Hk, int64_t N) {
-  (void)B; (void)Hq; (void)Hk; (void)N;
-  if (T <= 1) return 0;  // the decode cut lives entirely in on-chip memory
-  return 0;
+  (void)Hk;
+  if (B < 0 || Hq < 0 || N < 0) return 0;
+  // decode: on chip up to 16 x 32768 keys, past that the scores each CTA cannot keep;
+  // prefill: the cut lives on chip
+  return T <= 1 ? rtp::topp_decode_workspace_bytes(B, Hq, N) : 0;
 }
 
 rtp_status rtp_topp_select(const rtp_tensor* q_idx, const rtp_tensor* k_idx, const int32_t* lens, float p,
@@ -193,6 +195,7 @@ rtp_status rtp_topp_select(const rtp_tensor* q_idx, const rtp_tensor* k_idx, con
   a.count = out->count;
   a.mask = out->mask;
   a.mask_words = out->mask_words;
+  a.spill = static_cast<float*>(workspace);
   return cuda_status(rtp::launch_topp_decode(a, (cudaStream_t)stream));
 }
 
@@ -231,6 +234,7 @@ rtp_status rtp_topk_select(const rtp_tensor* q_idx, const rtp_tensor* k_idx, con
   a.count = out->count;
   a.mask = out->mask;
   a.mask_words = out->mask_words;
+  a.spill = static_cast<float*>(workspace);
   return cuda_status(rtp::launch_topp_decode(a, (cudaStream_t)stream));
 }
 

@@ -33,9 +33,8 @@
 // barrier.
 // Caches longer than 16 CTAs x 32768 keys (up to 4x that) give each CTA more
 // keys than its shared memory holds: the first 32768 scores stay on chip and
-// the rest are recomputed from the projected keys (L2-resident after the first
-// pass) by every pass that reads them -- the same function of the same bits,
-// so the cut is the one the stored scores would give.
+// the rest go to the caller's workspace (written once, read back from L2 by the
+// thread that wrote them in every later pass).
 #include <cooperative_groups.h>
 
 #include <math.h>
@@ -336,7 +335,7 @@ __global__ void __maxnreg__(96)
 topp_query_kernel(View4 qv, View4 kv, const int32_t* __restrict__ lens, int Hq, int G, int N,
                    int n_chunk, float p, int topk, float two_pow_frac, uint32_t* __restrict__ tau_bits,
                    int32_t* __restrict__ tiepos, int32_t* __restrict__ count,
-                   uint32_t* __restrict__ mask, int64_t mask_words) {
+                   uint32_t* __restrict__ mask, int64_t mask_words, float* __restrict__ spill) {
   pdl_wait();
   pdl_release();
   cg::cluster_group cluster = cg::this_cluster();
@@ -399,13 +398,10 @@ topp_query_kernel(View4 qv, View4 kv, const int32_t* __restrict__ lens, int Hq, 
   const T* kb = static_cast<const T*>(kv.data) + b * kv.sb + kvh * kv.sh;
   float lmax = -INFINITY;
   const int n_res = min(n_chunk, kMaxKeysPerCta);  // keys whose scores stay in shared memory
-  // score of local key i: stored, or recomputed (identical bits) past the resident ones
-  auto score_of = [&](int i) -> float {
-    if (i < n_res) return scores[i];
-    float kf[kIdxDim];
-    load_idx_row<T>(kb + (int64_t)(c0 + i) * kv.sn, kf);
-    return indexer_dot16(qf, kf);
-  };
+  // this CTA's scores past the resident ones; every pass maps key i to thread i % kSelThreads, so
+  // each thread reads back only what it wrote
+  float* const gsc = spill ? spill + ((int64_t)qrow * C + rank) * (int64_t)(n_chunk - n_res) : nullptr;
+  auto score_of = [&](int i) -> float { return i < n_res ? scores[i] : gsc[i - n_res]; };
   constexpr int U = sizeof(T) == 2 ? 4 : 2;
   for (int base = 0; base < nloc; base += U * kSelThreads) {
     IdxRaw<T> raw[U];
@@ -421,7 +417,10 @@ topp_query_kernel(View4 qv, View4 kv, const int32_t* __restrict__ lens, int Hq, 
         float kf[kIdxDim];
         idx_raw_to_float<T>(raw[u], kf);
         const float sc = indexer_dot16(qf, kf);
-        if (i < n_res) scores[i] = sc;
+        if (i < n_res)
+          scores[i] = sc;
+        else
+          gsc[i - n_res] = sc;
         lmax = fmaxf(lmax, sc);
       }
     }
@@ -683,6 +682,28 @@ topp_query_kernel(View4 qv, View4 kv, const int32_t* __restrict__ lens, int Hq, 
 
 bool topp_decode_supported(int64_t N) { return N <= (int64_t)kMaxKeysPerCta * kMaxCluster * kMaxStream; }
 
+// CTAs per query (a power of two <= kMaxCluster) and keys per CTA (a multiple of 32).
+static void topp_layout(int64_t Q, int64_t N, int sms, int* C_out, int64_t* n_chunk_out) {
+  int C = 1;
+  while (C < 8 && Q * C < sms) C <<= 1;
+  while ((N + C - 1) / C > kMaxKeysPerCta && C < kMaxCluster) C <<= 1;
+  int64_t n_chunk = (N + C - 1) / C;
+  n_chunk = (n_chunk + 31) / 32 * 32;
+  if (n_chunk == 0) n_chunk = 32;
+  *C_out = C;
+  *n_chunk_out = n_chunk;
+}
+
+size_t topp_decode_workspace_bytes(int64_t B, int64_t Hq, int64_t N) {
+  // the layout depends on the SM count only while every CTA's keys fit on chip; past that
+  // the cluster has kMaxCluster CTAs whatever the SM count
+  int C = 0;
+  int64_t n_chunk = 0;
+  topp_layout(B * Hq, N, 1, &C, &n_chunk);
+  const int64_t per = n_chunk > kMaxKeysPerCta ? (n_chunk - kMaxKeysPerCta) * C : 0;
+  return (size_t)(B * Hq * per) * sizeof(float);
+}
+
 static int sm_count() {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
@@ -709,20 +730,18 @@ cudaError_t launch_topp_decode(const LaunchToppDecode& a, cudaStream_t stream) {
 
   // Query form: one cluster per query.
   int C = 1;
-  while (C < 8 && Q * C < sms) C <<= 1;
-  while ((a.N + C - 1) / C > kMaxKeysPerCta && C < kMaxCluster) C <<= 1;
-  int64_t n_chunk = (a.N + C - 1) / C;
-  n_chunk = (n_chunk + 31) / 32 * 32;
-  if (n_chunk == 0) n_chunk = 32;
+  int64_t n_chunk = 0;
+  topp_layout(Q, a.N, sms, &C, &n_chunk);
   if (n_chunk > (int64_t)kMaxKeysPerCta * kMaxStream) return cudaErrorInvalidValue;
+  if (n_chunk > kMaxKeysPerCta && !a.spill) return cudaErrorInvalidValue;
   const size_t smem = sizeof(SelSmem) + (size_t)(n_chunk < kMaxKeysPerCta ? n_chunk : kMaxKeysPerCta) * sizeof(float);
   if (a.bf16)
     return launch_cluster(topp_query_kernel<__nv_bfloat16>, (int)(Q * C), C, smem, stream, a.q_idx, a.k_idx, a.lens,
                           (int)a.Hq, G, (int)a.N, (int)n_chunk, a.p, (int)a.topk, two_pow_frac, a.tau_bits, a.tiepos,
-                          a.count, a.mask, a.mask_words);
+                          a.count, a.mask, a.mask_words, a.spill);
   return launch_cluster(topp_query_kernel<float>, (int)(Q * C), C, smem, stream, a.q_idx, a.k_idx, a.lens, (int)a.Hq,
                         G, (int)a.N, (int)n_chunk, a.p, (int)a.topk, two_pow_frac, a.tau_bits, a.tiepos, a.count,
-                        a.mask, a.mask_words);
+                        a.mask, a.mask_words, a.spill);
 }
 
 }  // namespace rtp

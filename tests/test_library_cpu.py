@@ -386,3 +386,20 @@ def test_cached_decode_layer_marshals_append_then_the_step():
         assert win[0]._args[3].value == layer.ring_lens.data_ptr() and win[0]._args[4].value == W
         assert wq.data == layer.q.data_ptr() + R * G * D * 2 and win[0]._args[-1].value == 22
     assert layer.cache_bytes() == 2 * B * R * N * D * 2 + B * R * N * 16 * 2 + 2 * B * (Hkv - R) * W * D * 2
+
+
+def test_decode_selection_workspace_for_long_caches():
+    # up to 16 x 32768 keys the decode cut lives on chip; past that the workspace holds the
+    # scores each of a query's 16 CTAs cannot keep (4 bytes per key beyond 16 x 32768)
+    rtp = _lib()
+    assert rtp.topp_select_workspace_size(8, 32, 1, 8, 32768) == 0
+    assert rtp.topp_select_workspace_size(1, 8, 1, 2, 524288) == 0
+    assert rtp.topp_select_workspace_size(1, 8, 1, 2, 1 << 20) == 8 * 16 * (65536 - 32768) * 4
+    assert rtp.topp_select_workspace_size(1, 8, 4096, 2, 1 << 20) == 0      # prefill
+    L = rtp.lib()
+    by = ctypes.byref
+    qi = _desc(rtp, [1, 8, 1, 16])
+    ki = _desc(rtp, [1, 2, 1 << 20, 16])
+    s = _sel(rtp, words=(1 << 20) // 32)
+    assert L.rtp_topp_select(by(qi), by(ki), None, 0.9, by(s), None, 0, None) == 5          # no workspace
+    assert L.rtp_topk_select(by(qi), by(ki), None, 10, by(s), None, 0, None) == 5
