@@ -30,7 +30,9 @@
 //            keys, whose cut can lie deeper), the last one the tail, with
 //            64-bit fixed-point masses; Z is their sum
 //   LIN 1-3  32 sub-bins of the previous cut bin (each level 32 times finer;
-//            power-of-two rescaling of u is exact), masses and counts
+//            power-of-two rescaling of u is exact), masses; a cut bin whose mass
+//            is at most 32 times the least weight a key of it can have holds at
+//            most 32 keys
 //   COLLECT  once the cut bin holds <= 32 keys, their (v, position) pairs are
 //            kept and sorted by (score desc, position asc) to finish the cut
 //   MASK     (only when a mask is requested) one more sweep writes it
@@ -84,7 +86,6 @@ struct PfSmem {
   alignas(1024) uint8_t qtile[kPfRows * kIdxDim * 2];  // A operand, 4 KB
   alignas(1024) uint8_t ktile[kPfStages][kPfTileBytes];  // B operand ring
   uint64_t hist[2][kPfBins][kPfRows];  // per half: bin masses, or candidates (COLLECT)
-  uint8_t hcnt[2][kPfBins][kPfRows];   // per half: bin counts (saturating at 255)
   PfRowState rs[kPfRows];
   float xs[16][kPfEpiWarps * 32];  // per epilogue thread: 16 keys of a chunk, for picking keys by column
   float pmax[kPfRows];  // half 1's partial maximum
@@ -275,7 +276,6 @@ topp_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
 #pragma unroll 4
       for (int i = 0; i < kPfBins; ++i) {
         S.hist[half][i][row] = 0;
-        S.hcnt[half][i][row] = 0;
       }
     }
     ncand = 0;
@@ -470,8 +470,6 @@ topp_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
                 if (level == kLvLin) {
                   const int d = min(max((int)__fmul_rn(u, dscale) - 32 * prefix, 0), kPfBins - 1);
                   hist_add(&S.hist[half][d][row], pf_weight_u(u, wmul, A.two_pow_frac));
-                  const uint8_t cc = S.hcnt[half][d][row];
-                  S.hcnt[half][d][row] = cc == 255 ? cc : (uint8_t)(cc + 1);
                 } else if (level == kLvKey) {
                   const uint32_t k = score_key(canon_score(x));
                   if (k >= kbase && (uint64_t)k < kend) {
@@ -593,11 +591,7 @@ topp_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
           const uint64_t tg = tt >= (double)Z ? Z : (uint64_t)tt;
           target = tg < 1 ? 1 : tg;
         } else {
-          for (int i = 0; i < kPfBins; ++i) {
-            S.hist[0][i][row] += S.hist[1][i][row];
-            const int cc = (int)S.hcnt[0][i][row] + (int)S.hcnt[1][i][row];
-            S.hcnt[0][i][row] = (uint8_t)(cc > 255 ? 255 : cc);
-          }
+          for (int i = 0; i < kPfBins; ++i) S.hist[0][i][row] += S.hist[1][i][row];
         }
         // the first bin (in score order) where the cumulative mass reaches the target; should
         // rounding ever leave it short, the last non-empty bin
@@ -636,13 +630,17 @@ topp_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
             vhi = vmax_u_ge(m, u_tail);
             level = kLvKey;
           } else {
-            const int in_bin = level == kLvLin0 ? 255 : (int)S.hcnt[0][cut][row];  // level 0 keeps no counts
             prefix = level == kLvLin0 ? cut : 32 * prefix + cut;  // full bin index at level `lin`
             const float ulo = (float)prefix / dscale;             // exact: dscale is a power of two
             const float uhi = (float)(prefix + 1) / dscale;
             vlo = vmax_u_ge(m, uhi);
             vhi = vmax_u_ge(m, ulo);
-            if (in_bin <= kPfBins) {
+            // every key of the cut bin has u < uhi, so weighs at least the weight at uhi: the bin's
+            // mass bounds how many keys it holds (2^-20 covers the rounding of the exponential)
+            const uint64_t w_lo = pf_weight_u(uhi, wmul, A.two_pow_frac);
+            const bool few = w_lo > 0 && (double)S.hist[0][cut][row] <=
+                                             (double)kPfBins * (double)w_lo * (1.0 - 9.5367431640625e-07);
+            if (few) {
               level = kLvCollect;
             } else if (lin < 3) {
               ++lin;

@@ -54,6 +54,7 @@ class DecodeLayer:
         self.ws_loc = (rtp.workspace(rtp.window_attn_workspace_size(B, Hq - R * G, 1, Hkv - R, N, W), dev)
                        if Hkv > R else None)
         self._plans = {}
+        self._host_graphs = {}  # host_step: (graph, stream) per set of host buffers
 
     def build_index(self, stream=None) -> None:
         """Project every cached key of the retrieval heads (done once, before decoding)."""
@@ -125,11 +126,9 @@ class DecodeLayer:
         forked stream); later calls replay it, so a token costs one graph launch
         and one synchronisation on the host."""
         key = (h_q.data_ptr(), h_k.data_ptr(), h_v.data_ptr(), h_o.data_ptr())
-        ent = self._host_graphs.get(key) if hasattr(self, "_host_graphs") else None
+        ent = self._host_graphs.get(key)
         if ent is None:
-            ent = self._capture_host(h_q, h_k, h_v, h_o)
-            self._host_graphs = getattr(self, "_host_graphs", {})
-            self._host_graphs[key] = ent
+            ent = self._host_graphs[key] = self._capture_host(h_q, h_k, h_v, h_o)
         graph, stream = ent
         graph.replay()
         stream.synchronize()
