@@ -133,8 +133,9 @@ kv_append_kernel(KvAppendArgs A) {
 
 cudaError_t launch_kv_append(const KvAppendArgs& a, bool bf16, cudaStream_t stream) {
   const int64_t rows = (int64_t)a.B * a.H * a.T;
-  if (rows == 0) return cudaSuccess;
+  if (a.B == 0 || (rows == 0 && !a.lens_out && !a.ring_lens)) return cudaSuccess;
   int64_t blocks = (rows + kAppUnroll * (kAppThreads / 32) - 1) / (kAppUnroll * (kAppThreads / 32));
+  if (blocks < 1) blocks = 1;  // an empty append still writes the lengths
   if (blocks > 148 * 16) blocks = 148 * 16;
   const size_t smem = a.R <= kAppSmemHeads ? (size_t)a.R * kIdxDim * kHeadDim * sizeof(float) : 0;
   if (bf16) {

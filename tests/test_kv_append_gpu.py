@@ -185,3 +185,27 @@ def test_cached_decode_matches_resident_cache_layer():
     ring = 2 * w.B * (w.Hkv - w.R) * w.W * 128 * 2
     full_ret = 2 * w.B * w.R * w.N * 128 * 2 + w.B * w.R * w.N * 16 * 2
     assert layer.cache_bytes() == full_ret + ring
+
+
+def test_empty_append_and_one_row_ring():
+    # T = 0 writes only the lengths; W = 1 keeps the newest token's row
+    dev = "cuda"
+    B, H, R, N, D = 2, 3, 1, 16, 128
+    k_full = torch.randn(B, H, 20, D, device=dev).to(torch.bfloat16)
+    P = torch.randn(R, 16, D, device=dev)
+    kc = torch.zeros(B, R, N, D, dtype=torch.bfloat16, device=dev)
+    vc, ki = torch.zeros_like(kc), torch.zeros(B, R, N, 16, dtype=torch.bfloat16, device=dev)
+    kr = torch.zeros(B, H - R, 1, D, dtype=torch.bfloat16, device=dev)
+    vr = torch.zeros_like(kr)
+    pos = torch.tensor([5, 0], dtype=torch.int32, device=dev)
+    out = torch.full((B,), -1, dtype=torch.int32, device=dev)
+    rl = torch.full((B,), -1, dtype=torch.int32, device=dev)
+    empty = k_full[:, :, :0]  # a zero-length view (its data pointer is valid)
+    rtp.kv_append(empty, empty, pos, R, P, kc, vc, ki, kr, vr, out, rl)
+    torch.cuda.synchronize()
+    assert out.cpu().tolist() == [5, 0] and rl.cpu().tolist() == [1, 0]
+    assert not kc.any() and not kr.any()
+    rtp.kv_append(_chunk(k_full, [5, 0], 3), _chunk(k_full, [5, 0], 3), pos, R, P, kc, vc, ki, kr, vr, out, rl)
+    torch.cuda.synchronize()
+    assert out.cpu().tolist() == [8, 3] and rl.cpu().tolist() == [1, 1]
+    assert torch.equal(kr[0, :, 0], k_full[0, R:, 7]) and torch.equal(kr[1, :, 0], k_full[1, R:, 2])
