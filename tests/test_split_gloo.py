@@ -90,7 +90,7 @@ def _rank(rank, world, port, out_dir):
 
 
 @pytest.mark.timeout(600)
-@pytest.mark.parametrize("world", [2, 3])
+@pytest.mark.parametrize("world", [2, 3, 4])
 def test_split_decode_matches_the_unsplit_oracle(world, tmp_path):
     import oracle
     mp.start_processes(_rank, args=(world, _free_port(), str(tmp_path)), nprocs=world, start_method="spawn",
