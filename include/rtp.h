@@ -19,7 +19,8 @@
  *   - Tensors are described by rtp_tensor: 4-D, strides in elements, the last
  *     dimension contiguous (stride[3] == 1), base address and every other
  *     stride 16-byte aligned.  Layout [B, H, N or T, D] ("head major"); any
- *     other memory order is expressed through the strides.
+ *     other memory order is expressed through the strides.  An empty tensor
+ *     (a zero among its first three dimensions) may have a NULL base.
  *   - Every pointer is a DEVICE pointer on the current device, allocated and
  *     owned by the caller.  The library allocates nothing on any call: calls
  *     that need scratch take a caller workspace (256-byte aligned) whose size

@@ -21,17 +21,20 @@ int64_t elt_size(int32_t dt) { return dt == RTP_F32 ? 4 : 2; }
 bool dtype_ok(int32_t dt) { return dt == RTP_F32 || dt == RTP_BF16; }
 
 // A 4-D tensor with the given last dimension, contiguous last dim, 16-byte
-// aligned base and (for dims longer than 1) 16-byte aligned strides.
+// aligned base and (for dims longer than 1) 16-byte aligned strides.  An empty
+// tensor (a zero dimension) may have a NULL base: nothing is read or written.
 rtp_status check4(const rtp_tensor* t, int64_t last) {
-  if (!t || !t->data) return RTP_ERR_INVALID_ARG;
+  if (!t) return RTP_ERR_INVALID_ARG;
   if (t->ndim != 4) return RTP_ERR_SHAPE;
   if (!dtype_ok(t->dtype)) return RTP_ERR_DTYPE;
   for (int i = 0; i < 4; ++i)
     if (t->shape[i] < 0 || t->stride[i] < 0) return RTP_ERR_SHAPE;
+  const bool empty = t->shape[0] == 0 || t->shape[1] == 0 || t->shape[2] == 0;
+  if (!t->data && !empty) return RTP_ERR_INVALID_ARG;
   if (t->shape[3] != last) return RTP_ERR_SHAPE;
   if (t->shape[0] > INT32_MAX || t->shape[1] > INT32_MAX || t->shape[2] > INT32_MAX) return RTP_ERR_SHAPE;
   if (t->stride[3] != 1) return RTP_ERR_ALIGNMENT;
-  if (((uintptr_t)t->data) % 16) return RTP_ERR_ALIGNMENT;
+  if (((uintptr_t)t->data) % 16) return RTP_ERR_ALIGNMENT;  // (NULL passes: an empty tensor)
   const int64_t es = elt_size(t->dtype);
   for (int i = 0; i < 3; ++i)
     if (t->shape[i] > 1 && (t->stride[i] * es) % 16) return RTP_ERR_ALIGNMENT;

@@ -403,3 +403,15 @@ def test_decode_selection_workspace_for_long_caches():
     s = _sel(rtp, words=(1 << 20) // 32)
     assert L.rtp_topp_select(by(qi), by(ki), None, 0.9, by(s), None, 0, None) == 5          # no workspace
     assert L.rtp_topk_select(by(qi), by(ki), None, 10, by(s), None, 0, None) == 5
+
+
+def test_empty_tensors_may_have_a_null_base():
+    # a zero among the first three dimensions: nothing is read or written, no launch
+    rtp = _lib()
+    L = rtp.lib()
+    by = ctypes.byref
+    x = _desc(rtp, [2, 4, 0, 128], data=0)
+    xi = _desc(rtp, [2, 4, 0, 16], data=0)
+    P = _desc(rtp, [4, 16, 128], dtype=0)
+    assert L.rtp_index_project(by(x), by(P), by(xi), None) == 0
+    assert L.rtp_index_project(by(_desc(rtp, [2, 4, 3, 128], data=0)), by(P), by(xi), None) == 1  # not empty
