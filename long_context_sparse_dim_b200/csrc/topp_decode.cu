@@ -24,9 +24,10 @@
 //            the keys of the cut sub-bin by (score desc, position asc), walks
 //            their weights to the cut and sets the candidates' mask bits.
 // If the cut lies in the tail bin or the fine cut bin holds more than 512
-// keys (heavy ties), narrowing continues in key space instead: 256 bins over
-// the order-preserving uint32 image of the fp32 score (8-bit digits of the
-// offset inside the coarse cut bin) until the bracket is one score value tau;
+// keys (long caches, heavy ties), narrowing continues in key space instead:
+// 256 bins over the order-preserving uint32 image of the fp32 score (8-bit
+// digits of the offset inside the fine cut bin, or the coarse tail bin) until
+// the bracket is one score value tau;
 // ties at tau are resolved by position with a prefix count over the cluster.
 // Every mass is a 64-bit fixed-point integer sum, so the result does not depend
 // on thread order.  No spin waits: all synchronisation is the hardware cluster
@@ -469,6 +470,7 @@ topp_query_kernel(View4 qv, View4 kv, const int32_t* __restrict__ lens, int Hq, 
   }
   uint64_t target = 0, mass_above = 0;
   const int lin = cluster_cut(S, cluster, S.hist[0], true, true, p, topk, target, mass_above);
+  int fine = -1;  // the fine cut bin, when the key-space narrowing below starts from it
 
   if (lin < kBins - 1) {
     // ---- the fine bin of the cut, from the 16 fine bins under coarse bin lin --
@@ -545,19 +547,23 @@ topp_query_kernel(View4 qv, View4 kv, const int32_t* __restrict__ lens, int Hq, 
       return;
     }
     cluster_wait();  // more candidates than rank 0 takes: narrow in key space below
+    fine = fb;       // inside the fine cut bin, 16 times narrower than the coarse one
+    mass_above = S.fine_above;
   }
 
-  // ---- key-space narrowing inside coarse bin lin -----------------------------
-  // key window holding every score of coarse bin `lin` (with a margin)
+  // ---- key-space narrowing inside the fine cut bin (or coarse bin lin for the tail) ----
+  // key window holding every score of that bin (with a margin)
   uint32_t kbase;
   uint64_t kend;
   int shift = 0;
   {
-    const float hi_s = m - (float)lin / kCoarsePerNat;
-    const float lo_s = m - (float)(lin + 1) / kCoarsePerNat;
-    const float mg = 1e-5f * (fabsf(m) + (float)(lin + 1) / kCoarsePerNat) + 1e-30f;
+    const float per_nat = fine >= 0 ? kFinePerNat : kCoarsePerNat;
+    const int bin = fine >= 0 ? fine : lin;
+    const float hi_s = m - (float)bin / per_nat;
+    const float lo_s = m - (float)(bin + 1) / per_nat;
+    const float mg = 1e-5f * (fabsf(m) + (float)(bin + 1) / per_nat) + 1e-30f;
     const uint32_t khi = score_key(__fadd_rn(hi_s + mg, 0.0f));
-    const uint32_t klo = lin == kBins - 1 ? 0u : score_key(__fadd_rn(lo_s - mg, 0.0f));
+    const uint32_t klo = fine < 0 && lin == kBins - 1 ? 0u : score_key(__fadd_rn(lo_s - mg, 0.0f));
     kbase = klo;
     kend = (uint64_t)khi + 1;
     const uint64_t range = kend - klo;
@@ -573,7 +579,7 @@ topp_query_kernel(View4 qv, View4 kv, const int32_t* __restrict__ lens, int Hq, 
     __syncwarp();
     for (int i = tid; i < nloc; i += kSelThreads) {
       const float sc = score_of(i);
-      if (coarse_bin(sc, m) == lin) {
+      if (fine >= 0 ? fine_bin(sc, m) == fine : coarse_bin(sc, m) == lin) {
         const uint32_t k = score_key(sc);
         if (k >= kbase && (uint64_t)k < kend) {
           const int d = (int)((uint64_t)(k - kbase) >> shift);
