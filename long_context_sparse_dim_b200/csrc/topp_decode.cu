@@ -24,7 +24,8 @@
 //            the keys of the cut sub-bin by (score desc, position asc), walks
 //            their weights to the cut and sets the candidates' mask bits.
 // If the cut lies in the tail bin or the fine cut bin holds more than 512
-// keys (long caches, heavy ties), narrowing continues in key space instead:
+// keys (long caches, heavy ties), narrowing continues in key space instead (at
+// once, without the scan, when the fine bin's mass already proves it too full):
 // 256 bins over the order-preserving uint32 image of the fp32 score (8-bit
 // digits of the offset inside the fine cut bin, or the coarse tail bin) until
 // the bracket is one score value tau;
@@ -93,6 +94,7 @@ struct SelSmem {
   uint64_t cut_above;
   int fine_cut;                      // fine bin holding the cut
   uint64_t fine_above;               // mass of the fine bins above it
+  uint64_t fine_mass;                // mass of the fine cut bin
   // rank 0: filled by every CTA between the fine cut and the candidate barrier
   uint32_t ncand;                    // candidates sent (may exceed kCandCap)
   uint32_t nabove;                   // keys above the fine cut bin
@@ -492,10 +494,26 @@ topp_query_kernel(View4 qv, View4 kv, const int32_t* __restrict__ lens, int Hq, 
       if (lane < kFinePerBin && incl - a < need && need <= incl) {
         S.fine_cut = lin * kFinePerBin + lane;
         S.fine_above = mass_above + (incl - a);
+        S.fine_mass = a;
       }
     }
     __syncthreads();
     const int fb = S.fine_cut;
+    // A fine bin whose mass exceeds kCandCap times the largest weight a key of it can have (at its
+    // upper end, u = fb / 256) certainly holds more candidates than rank 0 takes: skip the candidate
+    // scan and narrow in key space at once (the same decision on every CTA of the cluster).
+    {
+      const double w_max = unit ? 1.0
+                                : (double)__float2ull_rn(__fmul_rn(
+                                      ex2f_fast(__fmul_rn(-(float)fb / kFinePerNat, 1.4426950408889634f)),
+                                      two_pow_frac)) * (1.0 + 9.5367431640625e-07);
+      if ((double)S.fine_mass > (double)kCandCap * w_max) {
+        fine = fb;
+        mass_above = S.fine_above;
+        cluster.sync();  // every CTA has read the others' fine bins before the passes below reuse them
+        goto key_space;
+      }
+    }
 
     // ---- one scan: mask words of the keys above the fine cut bin; its keys
     //      (the candidates) and the count of keys above it go to rank 0 ------
@@ -551,6 +569,7 @@ topp_query_kernel(View4 qv, View4 kv, const int32_t* __restrict__ lens, int Hq, 
     mass_above = S.fine_above;
   }
 
+key_space:
   // ---- key-space narrowing inside the fine cut bin (or coarse bin lin for the tail) ----
   // key window holding every score of that bin (with a margin)
   uint32_t kbase;
