@@ -61,17 +61,28 @@ class DecodeLayer:
         if self.R:
             rtp.index_project(self.k_ret, self.P, self.k_idx, stream)
 
-    def _plan(self, main: torch.cuda.Stream, side: Optional[torch.cuda.Stream]):
+    def _plan(self, main: torch.cuda.Stream, side: Optional[torch.cuda.Stream], new_rows=None):
         """The step's C-ABI calls with their arguments marshalled once, for
         this pair of streams: projections, window attention, and the chain
-        selection -> sparse attention."""
+        selection -> sparse attention.  With ``new_rows`` = (k_new, v_new, pos)
+        the step first appends each sequence's new K/V row (staged on the
+        device) at position pos[b] with rtp_kv_append, which also writes its
+        projected key, in place of the projection of a row already in the cache."""
         pre, win, chain = [], [], []
+        R, H = self.R, self.Hkv
+        if new_rows is not None:
+            k_new, v_new, pos = new_rows
+            # the local heads' full caches serve as rings of N rows: position p goes to row p mod N = p
+            pre.append(rtp.bind_kv_append(k_new, v_new, pos, R, self.P if R else None,
+                                          self.k_ret if R else None, self.v_ret if R else None,
+                                          self.k_idx if R else None, self.k_loc if H > R else None,
+                                          self.v_loc if H > R else None, None, None, main))
         if self.R:
-            if self.lens_host is None:
+            if new_rows is None and self.lens_host is None:
                 n = self.N
                 pre.append(rtp.bind_index_project(self.k_ret[:, :, n - 1: n], self.P, self.k_idx[:, :, n - 1: n],
                                                   main))
-            else:
+            elif new_rows is None:
                 for b, n in enumerate(self.lens_host):
                     if n > 0:
                         pre.append(rtp.bind_index_project(self.k_ret[b: b + 1, :, n - 1: n], self.P,
@@ -99,6 +110,11 @@ class DecodeLayer:
         plan = self._plans.get(key)
         if plan is None:
             plan = self._plans[key] = self._plan(main, side_stream)
+        self._run(plan, main, side_stream)
+        return self.o
+
+    @staticmethod
+    def _run(plan, main, side_stream) -> None:
         pre, win, chain = plan
         for call in pre:
             call()
@@ -114,17 +130,18 @@ class DecodeLayer:
                 call()
             for call in win:
                 call()
-        return self.o
 
     def host_step(self, h_q: torch.Tensor, h_k: torch.Tensor, h_v: torch.Tensor, h_o: torch.Tensor) -> torch.Tensor:
         """One decode step end to end from host memory: copy the new token's
         queries h_q [B, Hq, 1, D] and key/value rows h_k, h_v [B, Hkv, 1, D] (pinned
         host tensors of the cache dtype) in, run the step, copy the output to h_o
         [B, Hq, 1, D] (pinned) and wait for it.  The new rows land at each
-        sequence's last position.  The first call with a set of buffers captures
-        the copies and the calls in one CUDA graph (with the window attention on a
-        forked stream); later calls replay it, so a token costs one graph launch
-        and one synchronisation on the host."""
+        sequence's last position: they are copied to a contiguous device staging
+        buffer and rtp_kv_append writes them into the caches together with the
+        projected key (one launch, no strided host copies).  The first call with a
+        set of buffers captures the copies and the calls in one CUDA graph (with
+        the window attention on a forked stream); later calls replay it, so a token
+        costs one graph launch and one synchronisation on the host."""
         key = (h_q.data_ptr(), h_k.data_ptr(), h_v.data_ptr(), h_o.data_ptr())
         ent = self._host_graphs.get(key)
         if ent is None:
@@ -141,15 +158,17 @@ class DecodeLayer:
         dev = self.q.device
         stream = torch.cuda.Stream(dev)
         side = torch.cuda.Stream(dev)
-        rows = ([(slice(None), self.N - 1)] if self.lens_host is None else
-                [(slice(b, b + 1), n - 1) for b, n in enumerate(self.lens_host) if n > 0])
+        k_new = torch.empty(self.B, self.Hkv, 1, self.D, dtype=self.k.dtype, device=dev)
+        v_new = torch.empty_like(k_new)
+        lens = [self.N] * self.B if self.lens_host is None else self.lens_host
+        pos = torch.tensor([n - 1 for n in lens], dtype=torch.int32, device=dev)  # -1 (empty): nothing written
+        plan = self._plan(stream, side, new_rows=(k_new, v_new, pos))
 
         def body():
             self.q.copy_(h_q, non_blocking=True)
-            for bs, n in rows:
-                self.k[bs, :, n: n + 1].copy_(h_k[bs], non_blocking=True)
-                self.v[bs, :, n: n + 1].copy_(h_v[bs], non_blocking=True)
-            self.step(side_stream=side)
+            k_new.copy_(h_k, non_blocking=True)
+            v_new.copy_(h_v, non_blocking=True)
+            self._run(plan, stream, side)
             h_o.copy_(self.o, non_blocking=True)
 
         stream.wait_stream(torch.cuda.current_stream(dev))

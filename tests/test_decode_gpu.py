@@ -196,3 +196,39 @@ def test_host_step_matches_device_step():
         h_o.zero_()
         layer.host_step(h_q, h_k, h_v, h_o)
         assert torch.equal(h_o, o_dev.cpu())
+
+
+def test_host_step_appends_the_new_rows_ragged():
+    # host_step writes each sequence's new K/V row (and its projected key) at its last
+    # position: over caches that lack those rows it gives the device step's bits over the
+    # complete caches; an empty sequence receives nothing
+    from long_context_sparse_dim_b200.layer import DecodeLayer
+    w = SMALL.replace(name="host_step_ragged", B=3, N=2000)
+    inst = wl.generate(w)
+    q, k, v, P, _ = upload(inst)
+    ln = [2000, 1500, 0]
+    lens = torch.tensor(ln, dtype=torch.int32, device=q.device)
+    full = DecodeLayer(q, k, v, P, R=w.R, W=w.W, p=w.p, lens=lens)
+    full.build_index()
+    o_dev = full.step().clone()
+    k2, v2 = k.clone(), v.clone()
+    for b, n in enumerate(ln):
+        if n > 0:
+            k2[b, :, n - 1] = 0
+            v2[b, :, n - 1] = 0
+    layer = DecodeLayer(q, k2, v2, P, R=w.R, W=w.W, p=w.p, lens=lens)
+    layer.build_index()
+    h_q = q.cpu().pin_memory()
+    rows_k = torch.stack([k[b, :, max(n - 1, 0)] for b, n in enumerate(ln)]).unsqueeze(2)
+    rows_v = torch.stack([v[b, :, max(n - 1, 0)] for b, n in enumerate(ln)]).unsqueeze(2)
+    rows_k[2] = 7.0  # the empty sequence's row is never written
+    rows_v[2] = -7.0
+    h_k = rows_k.cpu().pin_memory()
+    h_v = rows_v.cpu().pin_memory()
+    h_o = torch.empty(o_dev.shape, dtype=o_dev.dtype).pin_memory()
+    for _ in range(2):
+        h_o.zero_()
+        layer.host_step(h_q, h_k, h_v, h_o)
+        assert torch.equal(h_o, o_dev.cpu())
+    assert torch.equal(k2, k) and torch.equal(v2, v)
+    assert torch.equal(layer.k_idx, full.k_idx)
