@@ -14,9 +14,12 @@ runs its own replica of the workload (weak scaling, no data-path collective).
 ``value`` is decode tokens/s (sequences advanced by one token per second,
 summed over ranks).  ``e2e`` is the same metric through the public API with
 host buffers (``DecodeLayer.host_step``): each step copies the new token's
-q/k/v from pinned host memory, makes the C-ABI calls and reads the output
-back, replayed as one CUDA graph, with the host waiting for every token.  ``--impl reference`` times
-the CPU oracle on the same workload instead (rank 0 only).
+q/k/v from pinned host memory, appends the new K/V rows (rtp_kv_append),
+makes the other C-ABI calls and reads the output back, replayed as one CUDA
+graph, with the host waiting for every token; the prefill object's ``e2e``
+uses ``PrefillLayer.host_step``, whose copies run pipelined with the work on
+two streams.  ``--impl reference`` times the CPU oracle on the same workload
+instead (rank 0 only).
 """
 from __future__ import annotations
 
@@ -862,7 +865,7 @@ def measure_prefill(args, wl, dev, world, steps, warmup, with_cpu):
                                "flop": 4.0 * 128 * int((pos + 1).sum()) * wl.Hq,
                                "pages": PAGES_SPEEDUP}
     del o_dense
-    out["e2e"] = _e2e_prefill(layer, inst, dev, side, max(1, min(steps, 3)))
+    out["e2e"] = _e2e_prefill(layer, inst, max(1, min(steps, 3)))
     if with_cpu:
         out["cpu_baseline"] = cpu_baseline_prefill(inst, wl, args.cpu_budget)
     del layer, q, k, v
@@ -887,7 +890,7 @@ def run_prefill(args, wl, rank, world, local_rank):
     return 0
 
 
-def _e2e_prefill(layer, inst, dev, side, steps):
+def _e2e_prefill(layer, inst, steps):
     import torch
     h_q = torch.from_numpy(inst.q).to(torch.bfloat16).pin_memory()
     h_k = torch.from_numpy(inst.k).to(torch.bfloat16).pin_memory()
@@ -898,14 +901,11 @@ def _e2e_prefill(layer, inst, dev, side, steps):
     torch.cuda.synchronize()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
+    layer.host_step(h_q, h_k, h_v, h_o)  # untimed: first use of the host streams
+    torch.cuda.synchronize()
     t0.record()
     for _ in range(steps):
-        layer.q.copy_(h_q, non_blocking=True)
-        layer.k.copy_(h_k, non_blocking=True)
-        layer.v.copy_(h_v, non_blocking=True)
-        layer.step(side_stream=side)
-        h_o.copy_(layer.o, non_blocking=True)
-        torch.cuda.current_stream().synchronize()
+        layer.host_step(h_q, h_k, h_v, h_o)  # copies in, the step, copy out (pipelined), host waits
     t1.record()
     torch.cuda.synchronize()
     ms = t0.elapsed_time(t1) / steps

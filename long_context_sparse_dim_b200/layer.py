@@ -237,6 +237,57 @@ class PrefillLayer:
             main.wait_stream(side_stream)
         return self.o
 
+    def host_step(self, h_q: torch.Tensor, h_k: torch.Tensor, h_v: torch.Tensor, h_o: torch.Tensor) -> torch.Tensor:
+        """One prefill end to end from host memory: h_q [B, Hq, T, D], h_k, h_v
+        [B, Hkv, N, D] (pinned, the layer's dtypes) in, the output to h_o [B, Hq,
+        T, D] (pinned), then wait for it.  The copies are pipelined with the
+        work: the retrieval heads' inputs cross first and their chain (projection,
+        selection, sparse attention, output copy) starts at once on one stream,
+        while the local heads' inputs, their window attention and their output
+        copy run on a second stream beside the selection."""
+        for t in (h_q, h_k, h_v, h_o):
+            if t.device.type != "cpu" or not t.is_pinned():
+                raise ValueError("host_step takes pinned host tensors")
+        for h, d in ((h_q, self.q), (h_k, self.k), (h_v, self.v), (h_o, self.o)):
+            if h.shape != d.shape or h.dtype != d.dtype or not h.is_contiguous():
+                raise ValueError("host buffers must be contiguous and match the layer's tensors")
+        dev = self.q.device
+        if getattr(self, "_host_streams", None) is None:
+            self._host_streams = (torch.cuda.Stream(dev), torch.cuda.Stream(dev))
+        main, side = self._host_streams
+        main.wait_stream(torch.cuda.current_stream(dev))
+        R, RG, H = self.R, self.R * self.G, self.Hkv
+        with torch.cuda.stream(main):
+            for b in range(self.B):  # per sequence: contiguous slices on both sides
+                if R:
+                    self.q[b, :RG].copy_(h_q[b, :RG], non_blocking=True)
+                    self.k[b, :R].copy_(h_k[b, :R], non_blocking=True)
+                    self.v[b, :R].copy_(h_v[b, :R], non_blocking=True)
+        if H > R:
+            side.wait_stream(main)  # the retrieval inputs cross first
+            with torch.cuda.stream(side):
+                for b in range(self.B):
+                    self.q[b, RG:].copy_(h_q[b, RG:], non_blocking=True)
+                    self.k[b, R:].copy_(h_k[b, R:], non_blocking=True)
+                    self.v[b, R:].copy_(h_v[b, R:], non_blocking=True)
+                rtp.window_attn(self.q_loc, self.k_loc, self.v_loc, self.lens, self.W, self.scale, self.o_loc,
+                                self.ws_loc, side)
+                for b in range(self.B):
+                    h_o[b, RG:].copy_(self.o[b, RG:], non_blocking=True)
+        if R:
+            with torch.cuda.stream(main):
+                rtp.index_project(self.k_ret, self.P, self.k_idx, main)
+                rtp.index_project(self.q_ret, self.P, self.q_idx, main)
+                rtp.topp_select(self.q_idx, self.k_idx, self.lens, self.p, self.sel, None, main)
+                rtp.sparse_attn_prefill(self.q_ret, self.k_ret, self.v_ret, self.q_idx, self.k_idx, self.lens,
+                                        self.sel, self.scale, self.o_ret, None, main)
+                for b in range(self.B):
+                    h_o[b, :RG].copy_(self.o[b, :RG], non_blocking=True)
+        if H > R:
+            main.wait_stream(side)
+        main.synchronize()
+        return h_o
+
 
 class CachedDecodeLayer:
     """Decode over caches the layer keeps itself: every step appends the new

@@ -101,3 +101,26 @@ def test_prefill_bf16_output_and_determinism():
     torch.cuda.synchronize()
     assert torch.equal(layer.o, o1) and torch.equal(layer.sel.mask, m1)
     _check(inst, layer, o1, tol=6e-3)
+
+
+def test_prefill_host_step_matches_step():
+    # the end-to-end form (pinned host buffers in and out, copies pipelined with the work on
+    # two streams) gives the device step's bits, ragged batch included
+    from long_context_sparse_dim_b200.layer import PrefillLayer
+    inst = wl.generate(SMALL.replace(name="pf_host", B=2, N=400, T=300))
+    w = inst.wl
+    q, k, v, P, lens = upload(inst)
+    layer = PrefillLayer(q, k, v, P, R=w.R, W=w.W, p=w.p, lens=lens)
+    o_dev = layer.step().clone()
+    torch.cuda.synchronize()
+    h_q, h_k, h_v = (x.cpu().pin_memory() for x in (q, k, v))
+    h_o = torch.empty(o_dev.shape, dtype=o_dev.dtype).pin_memory()
+    layer.q.zero_()
+    layer.k.zero_()
+    layer.v.zero_()
+    layer.o.zero_()
+    for _ in range(2):
+        h_o.zero_()
+        layer.host_step(h_q, h_k, h_v, h_o)
+        assert torch.equal(h_o, o_dev.cpu())
+    assert rtp.poll_device_error() == 0
