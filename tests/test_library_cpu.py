@@ -244,6 +244,62 @@ def test_decode_layer_marshals_each_call_of_the_step():
     assert list(ao.shape) == [B, R * G, 1, D] and ao.data == layer.o.data_ptr()
 
 
+def test_decode_layer_host_plan_appends_the_new_rows():
+    # the host-buffer step appends the staged new rows with rtp_kv_append (retrieval
+    # heads to their caches and projected keys, local heads to their full caches used
+    # as rings of N rows) and then projects only the queries
+    import torch
+    rtp = _lib()
+    from long_context_sparse_dim_b200.layer import DecodeLayer
+    B, Hq, Hkv, N, D, R, W = 2, 8, 2, 300, 128, 1, 64
+    G = Hq // Hkv
+    q = torch.zeros(B, Hq, 1, D, dtype=torch.bfloat16)
+    k = torch.zeros(B, Hkv, N, D, dtype=torch.bfloat16)
+    v = torch.zeros(B, Hkv, N, D, dtype=torch.bfloat16)
+    P = torch.zeros(R, 16, D)
+    layer = DecodeLayer(q, k, v, P, R=R, W=W, p=0.9)
+    k_new = torch.zeros(B, Hkv, 1, D, dtype=torch.bfloat16)
+    v_new = torch.zeros_like(k_new)
+    pos = torch.tensor([N - 1, N - 1], dtype=torch.int32)
+    main, side = _FakeStream(11), _FakeStream(22)
+    pre, win, chain = layer._plan(main, side, new_rows=(k_new, v_new, pos))
+    assert [c._name for c in pre] == ["rtp_kv_append", "rtp_index_project"]
+    assert [c._name for c in win] == ["rtp_window_attn"]
+    assert [c._name for c in chain] == ["rtp_topp_select", "rtp_sparse_attn_decode"]
+    app = pre[0]._args
+    assert app[2].value == pos.data_ptr() and app[3].value == R
+    assert app[10] is None and app[11] is None and app[-1].value == 11  # no lengths written
+    kn, vn, Pd, kc, vc, ki, kr, vr = _descs(pre[0], rtp)
+    assert kn.data == k_new.data_ptr() and vn.data == v_new.data_ptr()
+    assert kc.data == k.data_ptr() and list(kc.shape) == [B, R, N, D]
+    assert ki.data == layer.k_idx.data_ptr() and list(ki.shape) == [B, R, N, 16]
+    assert kr.data == k.data_ptr() + R * N * D * 2 and list(kr.shape) == [B, Hkv - R, N, D]
+    assert vr.data == v.data_ptr() + R * N * D * 2
+    qx, _, qo = _descs(pre[1], rtp)
+    assert list(qx.shape) == [B, R * G, 1, D] and qo.data == layer.q_idx.data_ptr()
+    # every head a retrieval head: no rings
+    layer2 = DecodeLayer(q, k, v, torch.zeros(Hkv, 16, D), R=Hkv, W=W, p=0.9)
+    pre2, win2, _ = layer2._plan(main, side, new_rows=(k_new, v_new, pos))
+    assert win2 == [] and pre2[0]._args[8] is None and pre2[0]._args[9] is None
+
+
+def test_host_steps_take_pinned_buffers_only():
+    import torch
+    _lib()
+    from long_context_sparse_dim_b200.layer import DecodeLayer, PrefillLayer
+    B, Hq, Hkv, N, T, D = 1, 8, 2, 256, 256, 128
+    q = torch.zeros(B, Hq, T, D, dtype=torch.bfloat16)
+    k = torch.zeros(B, Hkv, N, D, dtype=torch.bfloat16)
+    v = torch.zeros(B, Hkv, N, D, dtype=torch.bfloat16)
+    P = torch.zeros(1, 16, D)
+    pl = PrefillLayer(q, k, v, P, R=1, W=64, p=0.9)
+    with pytest.raises(ValueError):
+        pl.host_step(q, k, v, torch.zeros(B, Hq, T, D))  # not pinned
+    dl = DecodeLayer(q[:, :, :1], k, v, P, R=1, W=64, p=0.9)
+    with pytest.raises(ValueError):
+        dl.host_step(q[:, :, :1], k[:, :, :1], v[:, :, :1], torch.zeros(B, Hq, 1, D))
+
+
 def test_header_is_plain_c_and_links_against_the_library(tmp_path):
     # include/rtp.h is a C header (C99, no C++), and a C program links
     # against librtp.so by the names it declares
