@@ -7,11 +7,12 @@
 // Hundred Training Steps", "Three Key Insights" 2-3: a 16-dim indexer ranks the
 // tokens and each query keeps the cumulative top-p of that ranking.
 //
-// Design (B200): a CTA takes one query head and 128 consecutive query tokens;
-// token r of the block is TMEM lane r.  A score tile of 128 tokens x 128 keys
+// Design (B200): a CTA takes the G query heads of one KV head x 128/G
+// consecutive query tokens (128 rows, row r = TMEM lane r), so every key tile
+// it streams serves the whole GQA group.  A score tile of 128 rows x 128 keys
 // is ONE tcgen05.mma (kind::f16, M=128, N=128, K=16): the projected queries
 // (A) stay in shared memory, 128-key tiles of the projected-key cache (B) are
-// streamed by TMA (32-byte swizzle, no multicast) through a 4-stage ring, and
+// streamed by TMA (32-byte swizzle, no multicast) through a 2-stage ring, and
 // the fp32 accumulators alternate between two TMEM buffers so the next MMA
 // runs while the epilogue reads the previous tile.  Warp roles (two CTAs per
 // SM):
@@ -29,6 +30,9 @@
 //   LIN0     32 bins of u, 1/4 nat each (1/2 nat for caches longer than 2^17
 //            keys, whose cut can lie deeper), the last one the tail, with
 //            64-bit fixed-point masses; Z is their sum
+//   TAIL     a cut in the last (tail) bin: the next 31 bins of the same width
+//            further out, the last one again the rest (repeated up to 5 times,
+//            far past the depth where a 64-bit fixed-point weight is still > 0)
 //   LIN 1-3  32 sub-bins of the previous cut bin (each level 32 times finer;
 //            power-of-two rescaling of u is exact), masses; a cut bin whose mass
 //            is at most 32 times the least weight a key of it can have holds at
@@ -36,8 +40,8 @@
 //   COLLECT  once the cut bin holds <= 32 keys, their (v, position) pairs are
 //            kept and sorted by (score desc, position asc) to finish the cut
 //   MASK     (only when a mask is requested) one more sweep writes it
-// Fallbacks: a cut in the tail bin, or a bin still too full after LIN 3,
-// continue with 5-bit digits of the order-preserving uint32 image of the score
+// Fallbacks: a cut past the last TAIL level, or a bin still too full after
+// LIN 3, continue with 5-bit digits of the order-preserving uint32 image of the score
 // (KEY) until one value is left; a TIE sweep then counts the keys above it and
 // locates the ties in position order.
 // Every bracket is an interval (vlo, vhi] of raw accumulators, precomputed
@@ -65,7 +69,11 @@ constexpr int kPfTileBytes = kPfKeys * kIdxDim * 2;  // 4 KB
 constexpr int kPfTmemCols = 2 * kPfKeys;             // two accumulator buffers
 constexpr int kPfMaxSweeps = 24;
 
-enum PfLevel : int { kLvMax, kLvLin0, kLvLin, kLvKey, kLvCollect, kLvTie, kLvMask, kLvDone };
+enum PfLevel : int { kLvMax, kLvLin0, kLvTail, kLvLin, kLvKey, kLvCollect, kLvTie, kLvMask, kLvDone };
+
+// A cut past the first level's 31 bins of u is binned again at the same width (TAIL), 31 bins further
+// each time, up to this offset in first-level bins; past it the exact score-key digits take over.
+constexpr int kPfMaxTailOff = 5 * 31;
 
 // The part of a row's state that its half-1 thread needs in the next sweep
 // (written by the row's half-0 thread after every sweep).
@@ -74,7 +82,7 @@ struct PfRowState {
   float m;         // raw row maximum
   float vlo, vhi;  // bracket: raw accumulators v with vlo < v <= vhi
   float dscale;    // LIN: c0 * 32^lin
-  int prefix;      // LIN: full bin index of the bracket at the previous level
+  int prefix;      // LIN: full bin index of the bracket at the previous level; TAIL: first-level bin of bin 0
   uint32_t kbase;  // KEY: lowest score key of the digit range
   int shift;       // KEY: digit shift
   uint64_t kend;   // KEY: one past the highest score key
@@ -272,7 +280,7 @@ topp_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
     const int more = __syncthreads_or(level != kLvDone);
     const int abort = __syncthreads_or(!alive);
     if (!more || abort || ntiles == 0) break;
-    if (epi && (level == kLvLin0 || level == kLvLin || level == kLvKey)) {
+    if (epi && (level == kLvLin0 || level == kLvTail || level == kLvLin || level == kLvKey)) {
 #pragma unroll 4
       for (int i = 0; i < kPfBins; ++i) {
         S.hist[half][i][row] = 0;
@@ -320,7 +328,7 @@ topp_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
     } else {
       // ---------------- epilogue: two threads per query row ----------------
       const float mh = m;
-      const bool bracket = level == kLvLin || level == kLvKey || level == kLvCollect;
+      const bool bracket = level == kLvLin || level == kLvTail || level == kLvKey || level == kLvCollect;
       // the screen: past the first linear level (a bracket 1/32 as wide or less) and with
       // finite bounds; bhw is the half width plus a margin for the rounding of x - c
       const bool screen = (level == kLvCollect || (level == kLvLin && dscale > 32.f * A.c0)) &&
@@ -467,8 +475,9 @@ topp_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
                 hb &= hb - 1u;
                 const float x = S.xs[j - 16 * hh][tid];
                 const float u = __fsub_rn(mh, x);
-                if (level == kLvLin) {
-                  const int d = min(max((int)__fmul_rn(u, dscale) - 32 * prefix, 0), kPfBins - 1);
+                if (level == kLvLin || level == kLvTail) {
+                  const int d = min(max((int)__fmul_rn(u, dscale) - (level == kLvTail ? prefix : 32 * prefix), 0),
+                                    kPfBins - 1);
                   hist_add(&S.hist[half][d][row], pf_weight_u(u, wmul, A.two_pow_frac));
                 } else if (level == kLvKey) {
                   const uint32_t k = score_key(canon_score(x));
@@ -579,7 +588,7 @@ topp_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
         A.tiepos[qrow] = tiepos;
         A.count[qrow] = gt_all + taken;
         level = mrow ? kLvMask : kLvDone;  // the selection mask needs one more sweep
-      } else {  // LIN0, LIN or KEY: find the cut bin
+      } else {  // LIN0, TAIL, LIN or KEY: find the cut bin
         if (level == kLvLin0) {
           uint64_t Z = 0;
           for (int i = 0; i < kPfBins; ++i) {
@@ -616,10 +625,18 @@ topp_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
           cum = cum_nz;
         }
         mass_above += cum;
-        if (level == kLvLin0 || level == kLvLin) {
-          if (level == kLvLin0 && cut == kPfBins - 1) {
-            // tail bin (u >= 31 / c0, i.e. s <= max s - 7.75 / c0): exact digits over its keys
-            const float u_tail = 31.f / A.c0;  // exact: c0 is a power of two
+        if (level == kLvLin0 || level == kLvTail || level == kLvLin) {
+          const int off = level == kLvTail ? prefix : 0;  // first-level bin of this level's bin 0
+          if (level != kLvLin && cut == kPfBins - 1 && off + 31 <= kPfMaxTailOff) {
+            // the cut lies past this level's 31 bins (c0 u >= off + 31): the next 31 bins of the same
+            // width, over the keys from there on (the last bin again holds the rest)
+            prefix = off + 31;
+            vlo = -INFINITY;
+            vhi = vmax_u_ge(m, (float)prefix / A.c0);  // exact: c0 is a power of two
+            level = kLvTail;
+          } else if (level != kLvLin && cut == kPfBins - 1) {
+            // still further out: exact digits over the keys past the last binned range
+            const float u_tail = (float)(off + 31) / A.c0;
             const float hi_s = __fmul_rn(__fsub_rn(m, u_tail), 0.25f);
             const float mg = 1e-5f * (fabsf(hi_s) + 8.f) + 1e-30f;
             kbase = 0u;
@@ -630,7 +647,7 @@ topp_prefill_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_const
             vhi = vmax_u_ge(m, u_tail);
             level = kLvKey;
           } else {
-            prefix = level == kLvLin0 ? cut : 32 * prefix + cut;  // full bin index at level `lin`
+            prefix = level == kLvLin ? 32 * prefix + cut : off + cut;  // full bin index at level `lin`
             const float ulo = (float)prefix / dscale;             // exact: dscale is a power of two
             const float uhi = (float)(prefix + 1) / dscale;
             vlo = vmax_u_ge(m, uhi);
