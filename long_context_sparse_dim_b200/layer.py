@@ -214,6 +214,7 @@ class PrefillLayer:
         self.sel = rtp.Selection.empty(B * R * G * T, N, dev, with_mask=with_mask)
         self.ws_loc = (rtp.workspace(rtp.window_attn_workspace_size(B, Hq - R * G, T, Hkv - R, N, W), dev)
                        if Hkv > R else None)
+        self._host_streams = None  # host_step: its two streams, made on first use
 
     def step(self, stream=None, side_stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
         main = torch.cuda.current_stream() if stream is None else stream
@@ -252,7 +253,7 @@ class PrefillLayer:
             if h.shape != d.shape or h.dtype != d.dtype or not h.is_contiguous():
                 raise ValueError("host buffers must be contiguous and match the layer's tensors")
         dev = self.q.device
-        if getattr(self, "_host_streams", None) is None:
+        if self._host_streams is None:
             self._host_streams = (torch.cuda.Stream(dev), torch.cuda.Stream(dev))
         main, side = self._host_streams
         main.wait_stream(torch.cuda.current_stream(dev))
